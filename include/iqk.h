@@ -1,0 +1,206 @@
+/*
+ * iqk.h -- C ABI of the B200 (sm_100a) IQ2_KS / IQ2_K routed-expert library.
+ *
+ * Fused dequantization plus matrix-vector / matrix-matrix products over 2-bit
+ * IQ_K-family weights, as defined on the mlx-iqk 0.1.1 project page
+ * (PKG-INFO), section "Format":
+ *
+ *   a 2-bit weight reconstructs as  d * float(scale_index) * values[4*alphabet + code],
+ *   every step float32, in that order.
+ *
+ * Stream format (one tensor [rows, cols] per expert; experts stacked on a
+ * leading axis; every stream a separate row-major, k-contiguous plane; cols a
+ * multiple of 256):
+ *
+ *   IQ2_KS  qs  uint32 [E][rows][cols/16]   weight k: word k>>4, bits 2*(k&15)..+1
+ *           scl uint32 [E][rows][cols/256]  32-weight sub-block j=k>>5: word j>>3,
+ *                                           nibble j&7 = low 4 bits of the index
+ *           sch uint8  [E][rows][cols/256]  bit j&7 of byte j>>3 = high bit of the index
+ *           sex uint8  [E][rows][cols/256]  bit j&7 of byte j>>3 = alphabet bit
+ *           dv  uint16 [E][rows]            fp16 row scale (bit pattern)
+ *           scale_index = (low4 | high<<4) - 16, in [-16, 15]
+ *           row bytes 2 + 70*cols/256 (2.1875 bits per weight + 16 bits per row)
+ *
+ *   IQ2_K   qs  uint32 [E][rows][cols/16]   as above
+ *           scl uint32 [E][rows][cols/128]  16-weight sub-block j=k>>4: word j>>3,
+ *                                           nibble j&7; scale_index = nibble - 8
+ *           sex uint16 [E][rows][cols/256]  bit j&15 of halfword j>>4 = alphabet bit
+ *           dv  uint16 [E][rows][cols/256]  fp16 scale per 256 weights
+ *           row bytes 76*cols/256 (2.375 bits per weight)
+ *
+ * The page fixes the granularity and content of every stream and that codes
+ * are little-endian in uint32 words; the packing of scl/sch/sex inside their
+ * words, and the offset-16 reading of the IQ2_KS signed index, are this
+ * library's readings (offset-16 mirrors IQ2_K's stated offset-8). The
+ * eight-entry value table (entries 0-3 alphabet 0, 4-7 alphabet 1) is not
+ * printed on the page; every call takes it as an argument.
+ *
+ * Conventions for every entry point:
+ *   - All array pointers are DEVICE pointers owned by the caller, unless the
+ *     parameter says "host". `values` is a host pointer to 8 floats, copied
+ *     into the launch (the caller may reuse it on return).
+ *   - Work is enqueued asynchronously on `stream` (a cudaStream_t; NULL is
+ *     the legacy default stream). Nothing on these paths allocates, frees or
+ *     synchronises; scratch comes from the caller's `workspace`.
+ *   - Arguments are validated on the host before any launch; a call that
+ *     returns an error has enqueued nothing. Device-resident data (expert
+ *     ids) is checked on the device: bad ids are skipped and recorded in the
+ *     workspace status word (iqk_moe_status).
+ *   - bf16 and fp16 values are passed as their 16-bit patterns (uint16_t).
+ */
+#ifndef IQK_H_
+#define IQK_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  IQK_OK = 0,
+  IQK_EINVAL = -1,       /* NULL pointer, bad enum, bad id range, inconsistent shapes */
+  IQK_ESHAPE = -2,       /* cols not a positive multiple of 256, rows <= 0, ... */
+  IQK_EUNSUPPORTED = -3, /* token count / topk / format combination not supported */
+  IQK_ECUDA = -4,        /* a CUDA call failed (see iqk_last_cuda_error) */
+  IQK_ETIMEOUT = -5,     /* a bounded device wait expired */
+  IQK_EWORKSPACE = -6    /* workspace NULL, misaligned (256 B) or too small */
+} iqk_status;
+
+typedef enum { IQK_IQ2_KS = 0, IQK_IQ2_K = 1 } iqk_format;
+
+/* One stacked weight tensor: `experts` matrices of [rows, cols]. */
+typedef struct {
+  int32_t fmt;          /* iqk_format */
+  int32_t experts;      /* >= 1 */
+  int32_t rows;         /* out_features, >= 1 */
+  int32_t cols;         /* in_features, positive multiple of 256 */
+  const uint32_t* qs;   /* [experts][rows][cols/16] */
+  const uint32_t* scl;  /* IQ2_KS [E][rows][cols/256]; IQ2_K [E][rows][cols/128] */
+  const uint8_t* sch;   /* IQ2_KS [E][rows][cols/256]; must be NULL for IQ2_K */
+  const void* sex;      /* IQ2_KS uint8 [E][rows][cols/256]; IQ2_K uint16 [E][rows][cols/256] */
+  const uint16_t* dv;   /* IQ2_KS [E][rows]; IQ2_K [E][rows][cols/256] */
+} iqk_weights;
+
+/* Human-readable text of a status code (static storage). */
+const char* iqk_strerror(int status);
+/* Text of the last CUDA error seen by this library in this thread ("" if none). */
+const char* iqk_last_cuda_error(void);
+/* Library ABI version: 1. */
+int iqk_version(void);
+
+/*
+ * Stream bytes of one row (all planes), or -1 for a bad format / width.
+ * Page: "IQ2_KS rows cost 2 + 70*n/256 bytes, IQ2_K rows cost 76*n/256 bytes".
+ */
+int64_t iqk_row_bytes(int32_t fmt, int32_t cols);
+
+/*
+ * iqk_dequant -- reconstruct expert `expert` of `w` to float32, bit-exact.
+ * Defines: the reconstruction formula above (page section "Format").
+ * out:    device float32 [rows][cols], row-major, written completely.
+ * Each weight is (d * (float)scale_index) * values[4*alphabet + code] with
+ * both products rounded to nearest even in float32 (no fused multiply-add,
+ * no flush of subnormals), so the result equals the CPU dequantizer's.
+ * Errors: IQK_EINVAL (NULL, bad fmt, expert out of range), IQK_ESHAPE.
+ */
+int iqk_dequant(const iqk_weights* w, int32_t expert, const float* values /* host [8] */,
+                float* out, void* stream);
+
+/*
+ * iqk_dequant_bf16 -- as iqk_dequant, then rounded to bfloat16 (nearest even):
+ * out[r][k] = bf16_rn(w_fp32[r][k]). This is the operand the prefill
+ * tensor-core path consumes, exposed so it can be checked bit for bit.
+ * out: device uint16 [rows][cols].
+ */
+int iqk_dequant_bf16(const iqk_weights* w, int32_t expert, const float* values /* host [8] */,
+                     uint16_t* out, void* stream);
+
+/*
+ * iqk_gemv -- y[t][o] = sum_k w[o][k] * x[t][k] for one expert, t < T.
+ * Defines: the fused decode GEMV of the page's "Surface" section (few
+ * token-expert pairs, one pass over the reduction axis).
+ * x: device bf16 [T][cols]; y: device float32 [T][rows]; 1 <= T <= 64.
+ * Accuracy: |y - y_exact| <= 2e-3 * sum_k |w[o][k] * x[t][k]| (weights enter the
+ * tensor-core reduction as bfloat16 of (scale_index * value) with d applied
+ * in float32; float32 accumulation).
+ * workspace: >= iqk_gemv_workspace_bytes(T, rows, cols) bytes, 256-B aligned.
+ */
+size_t iqk_gemv_workspace_bytes(int32_t T, int32_t rows, int32_t cols);
+int iqk_gemv(const iqk_weights* w, int32_t expert, const float* values /* host [8] */,
+             const uint16_t* x, int32_t T, float* y, void* workspace, size_t ws_bytes,
+             void* stream);
+
+/*
+ * Routed-expert block (gate/up GEMV, SwiGLU, down GEMV, weighted combine).
+ * Geometry on the page: 256 experts, six selected, gate and up [2048 x 4096],
+ * down [4096 x 2048]; any experts >= 1, hidden and inter multiples of 256.
+ *
+ *   gate, up: [E][inter][hidden];  down: [E][hidden][inter]  (same E)
+ *   x:   device bf16 [T][hidden]
+ *   ids: device int32 [T][topk], expert of slot j of token t (0 <= id < E;
+ *        ids within a token should be distinct -- duplicates are computed as
+ *        separate pairs)
+ *   p:   device float32 [T][topk], routing weight of each slot
+ *   y:   device bf16 [T][hidden], written completely:
+ *        y[t] = bf16_rn( sum_j p[t][j] * down_e( bf16_rn( silu(gate_e x_t) * up_e x_t ) ) )
+ *        with silu(g) = g / (1 + exp(-g)), e = ids[t][j].
+ *   1 <= topk <= 16.
+ *
+ * iqk_moe_decode: few tokens (1 <= T <= 64); one weight read per distinct
+ *   expert per call, shared by the tokens routed to it.
+ * iqk_moe_prefill: many tokens (1 <= T <= 65536); pairs grouped by expert,
+ *   weights dequantized once per expert into bfloat16 tensor-core operands.
+ *
+ * workspace: >= iqk_moe_workspace_bytes(...) bytes, 256-B aligned, owned by
+ * the caller, not shared by concurrent calls. mode 0 = decode, 1 = prefill.
+ */
+size_t iqk_moe_workspace_bytes(int32_t mode, int32_t T, int32_t topk, int32_t experts,
+                               int32_t hidden, int32_t inter);
+int iqk_moe_decode(const iqk_weights* gate, const iqk_weights* up, const iqk_weights* down,
+                   const float* values /* host [8] */, const uint16_t* x, int32_t T,
+                   const int32_t* ids, const float* p, int32_t topk, uint16_t* y,
+                   void* workspace, size_t ws_bytes, void* stream);
+int iqk_moe_prefill(const iqk_weights* gate, const iqk_weights* up, const iqk_weights* down,
+                    const float* values /* host [8] */, const uint16_t* x, int32_t T,
+                    const int32_t* ids, const float* p, int32_t topk, uint16_t* y,
+                    void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * iqk_moe_status -- synchronises `stream`, then reads the status word a
+ * decode/prefill call left in `workspace`: IQK_OK, or IQK_EINVAL if any
+ * expert id was outside [0, E) (those pairs were skipped), or IQK_ETIMEOUT.
+ */
+int iqk_moe_status(const void* workspace, void* stream);
+
+/*
+ * iqk_moe_route -- the prefill grouping step on its own (for inspection):
+ * counts[e] = number of (token, slot) pairs routed to e; offsets[e] =
+ * exclusive prefix sum (offsets[E] = number of valid pairs); perm[i] = pair
+ * index t*topk + j of the i-th pair in expert order, ties in pair order.
+ * counts: device int32 [E]; offsets: device int32 [E+1]; perm: device int32 [T*topk].
+ * Page: prefill "honouring the caller's sort flag so each expert's weights are
+ * read once per sorted prefill" (section "Surface").
+ */
+int iqk_moe_route(const int32_t* ids, int32_t T, int32_t topk, int32_t experts, int32_t* counts,
+                  int32_t* offsets, int32_t* perm, void* workspace, size_t ws_bytes,
+                  void* stream);
+
+/*
+ * iqk_floor -- the deleted-decode address floor used for pricing (page section
+ * "Pricing": identical loads, decode removed, an integer accumulator reaching
+ * the output). For each listed expert it streams every byte of every stream
+ * of every row with the same access pattern as the decode kernels and writes
+ * out[i][r] = XOR over the row's bytes, byte b of a stream folded into byte
+ * (b & 3) of a little-endian word.
+ * expert_list: device int32 [n_experts]; out: device uint32 [n_experts][rows].
+ */
+int iqk_floor(const iqk_weights* w, const int32_t* expert_list, int32_t n_experts, uint32_t* out,
+              void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* IQK_H_ */

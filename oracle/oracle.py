@@ -1,0 +1,243 @@
+"""CPU oracle for the IQ2_KS / IQ2_K routed-expert path.
+
+TEST INFRASTRUCTURE ONLY. Only the tests, the package smoke check and the
+benchmark's CPU-baseline leg may import this module; the product path never
+does, and this module imports nothing from the CUDA library. It shares no
+code, header, table or constant generator with it.
+
+What it computes, and where each step is defined:
+
+* ``dequant``: the page's reconstruction ``d * float(scale_index) *
+  values[4*alphabet + code]`` in float32, each product rounded once, in that
+  order (mlx-iqk 0.1.1 PKG-INFO, section "Format", the paragraph after the
+  stream tables). Implemented in plain C (``iqk_oracle.c``), built with
+  ``-ffp-contract=off``.
+* ``gemv``: the plain definition ``y[t,o] = sum_k w[o,k] * x[t,k]`` in float64
+  (a library matmul as the one step), plus ``S[t,o] = sum_k |w[o,k] * x[t,k]|``,
+  the scale of the stated tolerance ``|y - y_ref| <= 2e-3 * S``.
+* ``moe``: the routed-expert block the page's geometry describes (gate/up,
+  SwiGLU, down, weighted combine; section "Surface" and the benchmark geometry
+  paragraph). The page does not write the block out; the plain reading used
+  here: ``g = Wg x``, ``u = Wu x``, ``h = bf16_rn(float32(silu(g) * u))`` with
+  ``silu(g) = g / (1 + exp(-g))`` in float64, ``y = sum_j p_j * (Wd_j h_j)`` in
+  float64, output ``bf16_rn(float32(y))``. Prefill is the same per token.
+* ``route_prep``: expert histogram, exclusive prefix sum and the stable
+  permutation of (token, slot) pairs sorted by expert -- what "grouped by
+  expert ... each expert's weights read once" requires (section "Surface").
+* ``floor_xor``: the deleted-decode address floor's checksum (section
+  "Pricing": identical loads, decode removed, an integer accumulator).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "iqk_oracle.c")
+_SO = os.path.join(_HERE, "_build", "liboracle.so")
+_lock = threading.Lock()
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile the C part of the oracle (plain gcc, strict float semantics)."""
+    os.makedirs(os.path.dirname(_SO), exist_ok=True)
+    if force or not os.path.exists(_SO) or os.path.getmtime(_SO) < os.path.getmtime(_SRC):
+        tmp = _SO + f".{os.getpid()}.tmp"
+        subprocess.check_call(["gcc", "-O2", "-std=c99", "-ffp-contract=off", "-fno-fast-math",
+                               "-fPIC", "-shared", "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, _SO)
+    return _SO
+
+
+def lib():
+    global _lib
+    with _lock:
+        if _lib is None:
+            L = ctypes.CDLL(build())
+            i64, u32p, f32p = ctypes.c_int64, ctypes.c_void_p, ctypes.c_void_p
+            L.oracle_half_to_float.restype = ctypes.c_float
+            L.oracle_half_to_float.argtypes = [ctypes.c_uint16]
+            L.oracle_float_to_bf16.restype = ctypes.c_uint16
+            L.oracle_float_to_bf16.argtypes = [ctypes.c_float]
+            L.oracle_dequant_iq2_ks.restype = ctypes.c_int
+            L.oracle_dequant_iq2_ks.argtypes = [i64, i64] + [ctypes.c_void_p] * 7
+            L.oracle_dequant_iq2_k.restype = ctypes.c_int
+            L.oracle_dequant_iq2_k.argtypes = [i64, i64] + [ctypes.c_void_p] * 6
+            L.oracle_f32_to_bf16_array.argtypes = [ctypes.c_void_p, ctypes.c_void_p, i64]
+            L.oracle_half_to_float_array.argtypes = [ctypes.c_void_p, ctypes.c_void_p, i64]
+            L.oracle_fields_iq2_ks.argtypes = [ctypes.c_void_p] * 4 + [i64] + [ctypes.c_void_p] * 3
+            L.oracle_fields_iq2_k.argtypes = [ctypes.c_void_p] * 3 + [i64] + [ctypes.c_void_p] * 3
+            L.oracle_floor_xor.argtypes = [i64, i64, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]
+            _lib = L
+    return _lib
+
+
+def _p(a: np.ndarray):
+    assert a.flags["C_CONTIGUOUS"], "oracle inputs must be C-contiguous"
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _c(a, dt):
+    return np.ascontiguousarray(a, dtype=dt)
+
+
+# ---------------------------------------------------------------- conversions
+
+def half_to_float(bits) -> np.ndarray:
+    b = _c(bits, np.uint16)
+    out = np.empty(b.shape, np.float32)
+    lib().oracle_half_to_float_array(_p(b), _p(out), b.size)
+    return out
+
+
+def bf16_round(x) -> np.ndarray:
+    """float32 -> bfloat16 bit patterns, round to nearest even."""
+    f = _c(x, np.float32)
+    out = np.empty(f.shape, np.uint16)
+    lib().oracle_f32_to_bf16_array(_p(f), _p(out), f.size)
+    return out
+
+
+def bf16_to_float(bits) -> np.ndarray:
+    """bfloat16 bit patterns -> float32 (exact: the pattern is the upper half)."""
+    return (_c(bits, np.uint16).astype(np.uint32) << 16).view(np.float32)
+
+
+# --------------------------------------------------------------------- fields
+
+def fields(fmt: str, qs_row, scl_row, sch_row, sex_row, k: int):
+    """(code, scale_index, alphabet) of weight ``k`` of one row."""
+    c, i, a = ctypes.c_int32(), ctypes.c_int32(), ctypes.c_int32()
+    L = lib()
+    if fmt == "iq2_ks":
+        q, s, h, x = (_c(qs_row, np.uint32), _c(scl_row, np.uint32), _c(sch_row, np.uint8),
+                      _c(sex_row, np.uint8))
+        L.oracle_fields_iq2_ks(_p(q), _p(s), _p(h), _p(x), k, ctypes.byref(c), ctypes.byref(i),
+                               ctypes.byref(a))
+    elif fmt == "iq2_k":
+        q, s, x = _c(qs_row, np.uint32), _c(scl_row, np.uint32), _c(sex_row, np.uint16)
+        L.oracle_fields_iq2_k(_p(q), _p(s), _p(x), k, ctypes.byref(c), ctypes.byref(i), ctypes.byref(a))
+    else:
+        raise ValueError(fmt)
+    return c.value, i.value, a.value
+
+
+# -------------------------------------------------------------------- dequant
+
+def dequant(fmt: str, rows: int, cols: int, qs, scl, sch, sex, dv, values) -> np.ndarray:
+    """float32 [rows, cols] reconstruction of one matrix (bit-exact reference)."""
+    v = _c(values, np.float32)
+    if v.shape != (8,):
+        raise ValueError("values must hold 8 entries")
+    out = np.empty((rows, cols), np.float32)
+    L = lib()
+    if fmt == "iq2_ks":
+        rc = L.oracle_dequant_iq2_ks(rows, cols, _p(_c(qs, np.uint32)), _p(_c(scl, np.uint32)),
+                                     _p(_c(sch, np.uint8)), _p(_c(sex, np.uint8)),
+                                     _p(_c(dv, np.uint16)), _p(v), _p(out))
+    elif fmt == "iq2_k":
+        rc = L.oracle_dequant_iq2_k(rows, cols, _p(_c(qs, np.uint32)), _p(_c(scl, np.uint32)),
+                                    _p(_c(sex, np.uint16)), _p(_c(dv, np.uint16)), _p(v), _p(out))
+    else:
+        raise ValueError(fmt)
+    if rc != 0:
+        raise ValueError(f"bad shape rows={rows} cols={cols}")
+    return out
+
+
+def dequant_expert(w, e: int, values) -> np.ndarray:
+    """Dequantize expert ``e`` of a stacked-stream object (attributes fmt, rows,
+    cols, qs, scl, sch, sex, dv with a leading expert axis)."""
+    return dequant(w.fmt, w.rows, w.cols, w.qs[e], w.scl[e], None if w.sch is None else w.sch[e],
+                   w.sex[e], w.dv[e], values)
+
+
+# ----------------------------------------------------------------------- gemv
+
+def gemv(w: np.ndarray, x_bits) -> tuple[np.ndarray, np.ndarray]:
+    """y[t, o] = sum_k w[o, k] x[t, k] in float64, and S = sum_k |w x|."""
+    x = bf16_to_float(np.atleast_2d(x_bits)).astype(np.float64)
+    wd = w.astype(np.float64)
+    return x @ wd.T, np.abs(x) @ np.abs(wd).T
+
+
+# ------------------------------------------------------------------------ moe
+
+def silu(g: np.ndarray) -> np.ndarray:
+    return g / (1.0 + np.exp(-g))
+
+
+class _Cache:
+    def __init__(self, w, values):
+        self.w, self.values, self.m = w, values, {}
+
+    def __call__(self, e):
+        e = int(e)
+        if e not in self.m:
+            self.m[e] = dequant_expert(self.w, e, self.values).astype(np.float64)
+        return self.m[e]
+
+
+def moe(gate, up, down, values, x_bits, ids, p, tokens=None):
+    """Routed-expert block for the listed tokens (all by default).
+
+    Returns dict with y_bits (bf16 [n, hidden]), y (float64 before the final
+    rounding), S (tolerance scale, float64) and h_bits (bf16 [n, topk, inter]).
+    """
+    x_bits = np.atleast_2d(x_bits)
+    ids = np.atleast_2d(ids)
+    p = np.atleast_2d(p)
+    toks = list(range(x_bits.shape[0])) if tokens is None else list(tokens)
+    Wg, Wu, Wd = _Cache(gate, values), _Cache(up, values), _Cache(down, values)
+    topk = ids.shape[1]
+    H, F = down.rows, down.cols
+    y = np.zeros((len(toks), H))
+    S = np.zeros((len(toks), H))
+    hb = np.zeros((len(toks), topk, F), np.uint16)
+    for n, t in enumerate(toks):
+        x = bf16_to_float(x_bits[t]).astype(np.float64)
+        for j in range(topk):
+            e = int(ids[t, j])
+            g = Wg(e) @ x
+            u = Wu(e) @ x
+            hb[n, j] = bf16_round((silu(g) * u).astype(np.float32))
+            h = bf16_to_float(hb[n, j]).astype(np.float64)
+            wd = Wd(e)
+            y[n] += float(p[t, j]) * (wd @ h)
+            S[n] += float(p[t, j]) * (np.abs(wd) @ np.abs(h))
+    return dict(y_bits=bf16_round(y.astype(np.float32)), y=y, S=S, h_bits=hb)
+
+
+# ----------------------------------------------------------------- route prep
+
+def route_prep(ids, experts: int):
+    """counts[e], offsets[e] (exclusive prefix sum, offsets[E] = total) and the
+    pair permutation: pair indices t*topk + j sorted by expert, ties in pair
+    order."""
+    flat = np.asarray(ids, np.int64).reshape(-1)
+    if flat.size and (flat.min() < 0 or flat.max() >= experts):
+        raise ValueError("expert id out of range")
+    counts = np.bincount(flat, minlength=experts).astype(np.int32)
+    offsets = np.zeros(experts + 1, np.int32)
+    offsets[1:] = np.cumsum(counts)
+    perm = np.argsort(flat, kind="stable").astype(np.int32)
+    return counts, offsets, perm
+
+
+# ---------------------------------------------------------------------- floor
+
+def floor_xor(w, e: int) -> np.ndarray:
+    """Per-row XOR fold of every stream byte of expert ``e`` (uint32 [rows])."""
+    streams = [a[e] for a in (w.qs, w.scl, w.sch, w.sex, w.dv) if a is not None]
+    rows = w.rows
+    arrs = [np.ascontiguousarray(a).reshape(rows, -1).view(np.uint8) for a in streams]
+    ptrs = (ctypes.c_void_p * len(arrs))(*[a.ctypes.data for a in arrs])
+    rb = np.array([a.shape[1] for a in arrs], np.int64)
+    out = np.empty(rows, np.uint32)
+    lib().oracle_floor_xor(rows, len(arrs), ptrs, _p(rb), _p(out))
+    return out
