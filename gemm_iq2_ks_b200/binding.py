@@ -1,0 +1,249 @@
+"""Thin Python binding of the C ABI in include/iqk.h (argument marshalling only).
+
+Every function here has the C entry point's name and forwards device
+pointers, sizes and the current CUDA stream to ``libiqk.so``; all
+computation happens in the library's CUDA kernels. PyTorch provides device
+memory and streams. There is no fallback: if the library cannot be loaded,
+the call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Sequence
+
+import numpy as np
+
+from . import build as _build
+
+IQK_OK, IQK_EINVAL, IQK_ESHAPE, IQK_EUNSUPPORTED, IQK_ECUDA, IQK_ETIMEOUT, IQK_EWORKSPACE = 0, -1, -2, -3, -4, -5, -6
+FMT = {"iq2_ks": 0, "iq2_k": 1}
+
+EXPORTS = (
+    "iqk_strerror", "iqk_last_cuda_error", "iqk_version", "iqk_row_bytes",
+    "iqk_dequant", "iqk_dequant_bf16", "iqk_gemv_workspace_bytes", "iqk_gemv",
+    "iqk_moe_workspace_bytes", "iqk_moe_decode", "iqk_moe_prefill", "iqk_moe_status",
+    "iqk_route_workspace_bytes", "iqk_moe_route", "iqk_floor",
+)
+
+
+class IqkWeights(ctypes.Structure):
+    _fields_ = [("fmt", ctypes.c_int32), ("experts", ctypes.c_int32), ("rows", ctypes.c_int32),
+                ("cols", ctypes.c_int32), ("qs", ctypes.c_void_p), ("scl", ctypes.c_void_p),
+                ("sch", ctypes.c_void_p), ("sex", ctypes.c_void_p), ("dv", ctypes.c_void_p)]
+
+
+_lib = None
+
+
+def library_path() -> str:
+    return _build.LIB
+
+
+def lib(build_if_missing: bool = True) -> ctypes.CDLL:
+    """Load libiqk.so (building it in-tree first if it is missing or stale)."""
+    global _lib
+    if _lib is None:
+        path = _build.LIB
+        if build_if_missing and not _build.up_to_date():
+            _build.build()
+        if not os.path.exists(path):
+            raise RuntimeError(f"CUDA library not built: {path}")
+        L = ctypes.CDLL(path)
+        vp, i32, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_size_t
+        W = ctypes.POINTER(IqkWeights)
+        sig = {
+            "iqk_strerror": (ctypes.c_char_p, [ctypes.c_int]),
+            "iqk_last_cuda_error": (ctypes.c_char_p, []),
+            "iqk_version": (ctypes.c_int, []),
+            "iqk_row_bytes": (ctypes.c_int64, [i32, i32]),
+            "iqk_dequant": (ctypes.c_int, [W, i32, vp, vp, vp]),
+            "iqk_dequant_bf16": (ctypes.c_int, [W, i32, vp, vp, vp]),
+            "iqk_gemv_workspace_bytes": (sz, [i32, i32, i32]),
+            "iqk_gemv": (ctypes.c_int, [W, i32, vp, vp, i32, vp, vp, sz, vp]),
+            "iqk_moe_workspace_bytes": (sz, [i32, i32, i32, i32, i32, i32]),
+            "iqk_moe_decode": (ctypes.c_int, [W, W, W, vp, vp, i32, vp, vp, i32, vp, vp, sz, vp]),
+            "iqk_moe_prefill": (ctypes.c_int, [W, W, W, vp, vp, i32, vp, vp, i32, vp, vp, sz, vp]),
+            "iqk_moe_status": (ctypes.c_int, [vp, vp]),
+            "iqk_route_workspace_bytes": (sz, [i32, i32, i32]),
+            "iqk_moe_route": (ctypes.c_int, [vp, i32, i32, i32, vp, vp, vp, vp, sz, vp]),
+            "iqk_floor": (ctypes.c_int, [W, vp, i32, vp, vp]),
+        }
+        for name, (res, args) in sig.items():
+            f = getattr(L, name)
+            f.restype = res
+            f.argtypes = args
+        _lib = L
+    return _lib
+
+
+def _check(rc: int, what: str) -> None:
+    if rc == IQK_OK:
+        return
+    L = lib()
+    msg = f"{what}: {L.iqk_strerror(rc).decode()} ({rc})"
+    if rc == IQK_ECUDA:
+        msg += f": {L.iqk_last_cuda_error().decode()}"
+    if rc in (IQK_EINVAL, IQK_ESHAPE):
+        raise ValueError(msg)
+    raise RuntimeError(msg)
+
+
+def _torch():
+    import torch
+    return torch
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    torch = _torch()
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _values(values) -> np.ndarray:
+    v = np.ascontiguousarray(values, dtype=np.float32)
+    if v.shape != (8,):
+        raise ValueError("values must hold 8 floats")
+    return v
+
+
+def _ptr(t) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+class Weights:
+    """Device-resident stacked streams of one weight tensor (torch CUDA tensors)."""
+
+    def __init__(self, fmt: str, experts: int, rows: int, cols: int, qs, scl, sch, sex, dv):
+        self.fmt, self.experts, self.rows, self.cols = fmt, experts, rows, cols
+        self.qs, self.scl, self.sch, self.sex, self.dv = qs, scl, sch, sex, dv
+        self._c = IqkWeights(FMT[fmt], experts, rows, cols, _ptr(qs), _ptr(scl), _ptr(sch), _ptr(sex), _ptr(dv))
+
+    @classmethod
+    def from_host(cls, s, device="cuda") -> "Weights":
+        """Upload host streams (attributes fmt, experts, rows, cols, qs, scl, sch, sex, dv)."""
+        torch = _torch()
+
+        def up(a, dt):
+            if a is None:
+                return None
+            return torch.from_numpy(np.ascontiguousarray(a).view(dt)).to(device)
+
+        return cls(s.fmt, s.experts, s.rows, s.cols, up(s.qs, np.int32), up(s.scl, np.int32),
+                   up(s.sch, np.uint8), up(s.sex, np.uint8 if s.fmt == "iq2_ks" else np.int16),
+                   up(s.dv, np.int16))
+
+    @property
+    def c(self) -> IqkWeights:
+        return self._c
+
+    def nbytes(self) -> int:
+        return sum(t.numel() * t.element_size() for t in (self.qs, self.scl, self.sch, self.sex, self.dv)
+                   if t is not None)
+
+
+def _empty(shape, dtype, device):
+    return _torch().empty(shape, dtype=dtype, device=device)
+
+
+# ------------------------------------------------------------------ entry points
+
+def iqk_row_bytes(fmt: str, cols: int) -> int:
+    return lib().iqk_row_bytes(FMT[fmt], cols)
+
+
+def iqk_dequant(w: Weights, expert: int, values, out=None, stream=None):
+    torch = _torch()
+    out = _empty((w.rows, w.cols), torch.float32, w.qs.device) if out is None else out
+    v = _values(values)
+    _check(lib().iqk_dequant(ctypes.byref(w.c), expert, v.ctypes.data, out.data_ptr(), _stream(stream)),
+           "iqk_dequant")
+    return out
+
+
+def iqk_dequant_bf16(w: Weights, expert: int, values, out=None, stream=None):
+    torch = _torch()
+    out = _empty((w.rows, w.cols), torch.bfloat16, w.qs.device) if out is None else out
+    v = _values(values)
+    _check(lib().iqk_dequant_bf16(ctypes.byref(w.c), expert, v.ctypes.data, out.data_ptr(), _stream(stream)),
+           "iqk_dequant_bf16")
+    return out
+
+
+def iqk_gemv_workspace_bytes(T: int, rows: int, cols: int) -> int:
+    return lib().iqk_gemv_workspace_bytes(T, rows, cols)
+
+
+def workspace(nbytes: int, device="cuda"):
+    """A 256-byte aligned device workspace (torch allocations are)."""
+    return _empty((max(nbytes, 256),), _torch().uint8, device)
+
+
+def iqk_gemv(w: Weights, expert: int, values, x, y=None, ws=None, stream=None):
+    torch = _torch()
+    T = x.shape[0]
+    y = _empty((T, w.rows), torch.float32, x.device) if y is None else y
+    need = iqk_gemv_workspace_bytes(T, w.rows, w.cols)
+    ws = workspace(need, x.device) if ws is None else ws
+    v = _values(values)
+    _check(lib().iqk_gemv(ctypes.byref(w.c), expert, v.ctypes.data, x.data_ptr(), T, y.data_ptr(), ws.data_ptr(),
+                          ws.numel(), _stream(stream)), "iqk_gemv")
+    return y
+
+
+def iqk_moe_workspace_bytes(mode: int, T: int, topk: int, experts: int, hidden: int, inter: int) -> int:
+    return lib().iqk_moe_workspace_bytes(mode, T, topk, experts, hidden, inter)
+
+
+def _moe(fn, mode, gate, up, down, values, x, ids, p, y, ws, stream):
+    torch = _torch()
+    T, topk = ids.shape
+    y = _empty((T, down.rows), torch.bfloat16, x.device) if y is None else y
+    need = iqk_moe_workspace_bytes(mode, T, topk, gate.experts, gate.cols, gate.rows)
+    if need == 0:
+        raise ValueError("unsupported token count / topk for this call")
+    ws = workspace(need, x.device) if ws is None else ws
+    v = _values(values)
+    _check(fn(ctypes.byref(gate.c), ctypes.byref(up.c), ctypes.byref(down.c), v.ctypes.data, x.data_ptr(), T,
+              ids.data_ptr(), p.data_ptr(), topk, y.data_ptr(), ws.data_ptr(), ws.numel(), _stream(stream)),
+           fn.__name__)
+    return y
+
+
+def iqk_moe_decode(gate: Weights, up: Weights, down: Weights, values, x, ids, p, y=None, ws=None, stream=None):
+    return _moe(lib().iqk_moe_decode, 0, gate, up, down, values, x, ids, p, y, ws, stream)
+
+
+def iqk_moe_prefill(gate: Weights, up: Weights, down: Weights, values, x, ids, p, y=None, ws=None, stream=None):
+    return _moe(lib().iqk_moe_prefill, 1, gate, up, down, values, x, ids, p, y, ws, stream)
+
+
+def iqk_moe_status(ws, stream=None) -> int:
+    return lib().iqk_moe_status(ws.data_ptr(), _stream(stream))
+
+
+def iqk_route_workspace_bytes(T: int, topk: int, experts: int) -> int:
+    return lib().iqk_route_workspace_bytes(T, topk, experts)
+
+
+def iqk_moe_route(ids, experts: int, ws=None, stream=None):
+    torch = _torch()
+    T, topk = ids.shape
+    dev = ids.device
+    counts = _empty((experts,), torch.int32, dev)
+    offsets = _empty((experts + 1,), torch.int32, dev)
+    perm = torch.full((T * topk,), -1, dtype=torch.int32, device=dev)
+    ws = workspace(iqk_route_workspace_bytes(T, topk, experts), dev) if ws is None else ws
+    _check(lib().iqk_moe_route(ids.data_ptr(), T, topk, experts, counts.data_ptr(), offsets.data_ptr(),
+                               perm.data_ptr(), ws.data_ptr(), ws.numel(), _stream(stream)), "iqk_moe_route")
+    return counts, offsets, perm, ws
+
+
+def iqk_floor(w: Weights, expert_list, out=None, stream=None):
+    torch = _torch()
+    n = expert_list.numel()
+    out = _empty((n, w.rows), torch.int32, expert_list.device) if out is None else out
+    _check(lib().iqk_floor(ctypes.byref(w.c), expert_list.data_ptr(), n, out.data_ptr(), _stream(stream)),
+           "iqk_floor")
+    return out

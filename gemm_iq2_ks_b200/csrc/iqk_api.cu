@@ -1,0 +1,251 @@
+// C ABI of the library (declared and documented in include/iqk.h).
+// Host-side argument validation, workspace checks and dispatch; no entry
+// point allocates, frees or synchronises except iqk_moe_status, which reads
+// the status word back by design.
+#include <stdio.h>
+#include <string.h>
+
+#include "iqk.h"
+#include "iqk_internal.h"
+
+using namespace iqk;
+
+namespace {
+
+thread_local char g_cuda_err[256] = "";
+
+int cuda_fail(cudaError_t e) {
+  snprintf(g_cuda_err, sizeof(g_cuda_err), "%s: %s", cudaGetErrorName(e), cudaGetErrorString(e));
+  return IQK_ECUDA;
+}
+
+// Launch helpers return -4 on a CUDA failure; record the text.
+int from_launch(int rc) {
+  if (rc == -4) {
+    cudaError_t e = cudaGetLastError();
+    if (e == cudaSuccess) e = cudaErrorUnknown;
+    return cuda_fail(e);
+  }
+  return rc;
+}
+
+int num_sms() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return -1;
+  static int cached[64] = {0};
+  if (dev < 0 || dev >= 64) return -1;
+  if (!cached[dev]) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return -1;
+    cached[dev] = n;
+  }
+  return cached[dev];
+}
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+int check_weights(const iqk_weights* w, WDev* out) {
+  if (!w) return IQK_EINVAL;
+  if (w->fmt != IQK_IQ2_KS && w->fmt != IQK_IQ2_K) return IQK_EINVAL;
+  if (w->experts < 1 || w->rows < 1) return IQK_ESHAPE;
+  if (w->cols <= 0 || w->cols % 256) return IQK_ESHAPE;
+  if (!w->qs || !w->scl || !w->sex || !w->dv) return IQK_EINVAL;
+  if ((w->fmt == IQK_IQ2_KS) != (w->sch != nullptr)) return IQK_EINVAL;
+  if (!aligned(w->qs, 16) || !aligned(w->scl, 4) || !aligned(w->dv, 2)) return IQK_EINVAL;
+  if (w->fmt == IQK_IQ2_K && !aligned(w->sex, 2)) return IQK_EINVAL;
+  if ((int64_t)w->experts * w->rows >= (int64_t)1 << 31) return IQK_ESHAPE;
+  out->qs = w->qs;
+  out->scl = w->scl;
+  out->sch = w->sch;
+  out->sex = w->sex;
+  out->dv = w->dv;
+  out->experts = w->experts;
+  out->rows = w->rows;
+  out->cols = w->cols;
+  return IQK_OK;
+}
+
+int check_values(const float* values, Values* V) {
+  if (!values) return IQK_EINVAL;
+  memcpy(V->v, values, sizeof(V->v));
+  return IQK_OK;
+}
+
+int check_ws(void* ws, size_t have, size_t need) {
+  if (need == 0) return IQK_OK;
+  if (!ws || !aligned(ws, 256) || have < need) return IQK_EWORKSPACE;
+  return IQK_OK;
+}
+
+int check_moe(const iqk_weights* gate, const iqk_weights* up, const iqk_weights* down, WDev* g, WDev* u,
+              WDev* d) {
+  int rc;
+  if ((rc = check_weights(gate, g)) || (rc = check_weights(up, u)) || (rc = check_weights(down, d))) return rc;
+  if (g->experts != u->experts || g->experts != d->experts) return IQK_EINVAL;
+  if (g->rows != u->rows || g->cols != u->cols) return IQK_EINVAL;
+  if (d->rows != g->cols || d->cols != g->rows) return IQK_EINVAL;
+  if (g->rows % 256) return IQK_ESHAPE;  // inter is the down projection's reduction width
+  return IQK_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* iqk_strerror(int s) {
+  switch (s) {
+    case IQK_OK: return "ok";
+    case IQK_EINVAL: return "invalid argument";
+    case IQK_ESHAPE: return "unsupported shape (widths must be positive multiples of 256)";
+    case IQK_EUNSUPPORTED: return "unsupported configuration";
+    case IQK_ECUDA: return "CUDA error";
+    case IQK_ETIMEOUT: return "bounded device wait expired";
+    case IQK_EWORKSPACE: return "workspace missing, misaligned or too small";
+    default: return "unknown status";
+  }
+}
+
+const char* iqk_last_cuda_error(void) { return g_cuda_err; }
+
+int iqk_version(void) { return 1; }
+
+int64_t iqk_row_bytes(int32_t fmt, int32_t cols) {
+  if (cols <= 0 || cols % 256) return -1;
+  if (fmt == IQK_IQ2_KS) return 2 + (int64_t)70 * cols / 256;
+  if (fmt == IQK_IQ2_K) return (int64_t)76 * cols / 256;
+  return -1;
+}
+
+int iqk_dequant(const iqk_weights* w, int32_t expert, const float* values, float* out, void* stream) {
+  WDev wd;
+  Values V;
+  int rc;
+  if ((rc = check_weights(w, &wd)) || (rc = check_values(values, &V))) return rc;
+  if (expert < 0 || expert >= wd.experts || !out || !aligned(out, 16)) return IQK_EINVAL;
+  const int sms = num_sms();
+  if (sms < 0) return cuda_fail(cudaGetLastError());
+  return from_launch(launch_dequant(wd, w->fmt, expert, V, out, false, (cudaStream_t)stream, sms));
+}
+
+int iqk_dequant_bf16(const iqk_weights* w, int32_t expert, const float* values, uint16_t* out, void* stream) {
+  WDev wd;
+  Values V;
+  int rc;
+  if ((rc = check_weights(w, &wd)) || (rc = check_values(values, &V))) return rc;
+  if (expert < 0 || expert >= wd.experts || !out || !aligned(out, 16)) return IQK_EINVAL;
+  const int sms = num_sms();
+  if (sms < 0) return cuda_fail(cudaGetLastError());
+  return from_launch(launch_dequant(wd, w->fmt, expert, V, out, true, (cudaStream_t)stream, sms));
+}
+
+size_t iqk_gemv_workspace_bytes(int32_t T, int32_t rows, int32_t cols) {
+  if (T < 1 || T > 64 || rows < 1 || cols <= 0 || cols % 256) return 0;
+  return gemv_ws(T, rows, cols).total;
+}
+
+int iqk_gemv(const iqk_weights* w, int32_t expert, const float* values, const uint16_t* x, int32_t T, float* y,
+             void* workspace, size_t ws_bytes, void* stream) {
+  WDev wd;
+  Values V;
+  int rc;
+  if ((rc = check_weights(w, &wd)) || (rc = check_values(values, &V))) return rc;
+  if (expert < 0 || expert >= wd.experts || !x || !y) return IQK_EINVAL;
+  if (T < 1 || T > 64) return IQK_EUNSUPPORTED;
+  if ((rc = check_ws(workspace, ws_bytes, gemv_ws(T, wd.rows, wd.cols).total))) return rc;
+  const int sms = num_sms();
+  if (sms < 0) return cuda_fail(cudaGetLastError());
+  return from_launch(launch_gemv(wd, w->fmt, expert, V, x, T, y, (char*)workspace, (cudaStream_t)stream, sms));
+}
+
+size_t iqk_moe_workspace_bytes(int32_t mode, int32_t T, int32_t topk, int32_t experts, int32_t hidden,
+                               int32_t inter) {
+  if (T < 1 || topk < 1 || topk > 16 || experts < 1 || hidden <= 0 || inter <= 0 || hidden % 256 || inter % 256)
+    return 0;
+  if (mode == 0) {
+    if (T > 64 || T * topk > kMaxPairs) return 0;
+    return decode_ws(T, topk, experts, hidden, inter).total;
+  }
+  if (mode == 1) {
+    if (T > 65536) return 0;
+    return prefill_ws(T, topk, experts, hidden, inter).total;
+  }
+  return 0;
+}
+
+int iqk_moe_decode(const iqk_weights* gate, const iqk_weights* up, const iqk_weights* down, const float* values,
+                   const uint16_t* x, int32_t T, const int32_t* ids, const float* p, int32_t topk, uint16_t* y,
+                   void* workspace, size_t ws_bytes, void* stream) {
+  WDev g, u, d;
+  Values V;
+  int rc;
+  if ((rc = check_moe(gate, up, down, &g, &u, &d)) || (rc = check_values(values, &V))) return rc;
+  if (!x || !ids || !p || !y) return IQK_EINVAL;
+  if (T == 0) return IQK_OK;
+  if (T < 0 || topk < 1 || topk > 16) return IQK_EINVAL;
+  if (T > 64 || T * topk > kMaxPairs) return IQK_EUNSUPPORTED;
+  if ((rc = check_ws(workspace, ws_bytes, decode_ws(T, topk, g.experts, g.cols, g.rows).total))) return rc;
+  const int sms = num_sms();
+  if (sms < 0) return cuda_fail(cudaGetLastError());
+  return from_launch(launch_moe_decode(g, gate->fmt, u, up->fmt, d, down->fmt, V, x, T, ids, p, topk, y,
+                                       (char*)workspace, (cudaStream_t)stream, sms));
+}
+
+int iqk_moe_prefill(const iqk_weights* gate, const iqk_weights* up, const iqk_weights* down, const float* values,
+                    const uint16_t* x, int32_t T, const int32_t* ids, const float* p, int32_t topk, uint16_t* y,
+                    void* workspace, size_t ws_bytes, void* stream) {
+  WDev g, u, d;
+  Values V;
+  int rc;
+  if ((rc = check_moe(gate, up, down, &g, &u, &d)) || (rc = check_values(values, &V))) return rc;
+  if (!x || !ids || !p || !y) return IQK_EINVAL;
+  if (T == 0) return IQK_OK;
+  if (T < 0 || topk < 1 || topk > 16) return IQK_EINVAL;
+  if (T > 65536) return IQK_EUNSUPPORTED;
+  if (!aligned(x, 16) || !aligned(y, 16)) return IQK_EINVAL;
+  if ((rc = check_ws(workspace, ws_bytes, prefill_ws(T, topk, g.experts, g.cols, g.rows).total))) return rc;
+  const int sms = num_sms();
+  if (sms < 0) return cuda_fail(cudaGetLastError());
+  return from_launch(launch_moe_prefill(g, gate->fmt, u, up->fmt, d, down->fmt, V, x, T, ids, p, topk, y,
+                                        (char*)workspace, (cudaStream_t)stream, sms));
+}
+
+int iqk_moe_status(const void* workspace, void* stream) {
+  if (!workspace) return IQK_EINVAL;
+  cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e);
+  int32_t s = 0;
+  e = cudaMemcpy(&s, workspace, 4, cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(e);
+  if (s & 2) return IQK_ETIMEOUT;
+  if (s & 1) return IQK_EINVAL;
+  return IQK_OK;
+}
+
+size_t iqk_route_workspace_bytes(int32_t T, int32_t topk, int32_t experts) {
+  if (T < 1 || topk < 1 || topk > 16 || experts < 1) return 0;
+  return align256(16) + align256(route_scratch_ints(T * topk, experts) * 4);
+}
+
+int iqk_moe_route(const int32_t* ids, int32_t T, int32_t topk, int32_t experts, int32_t* counts, int32_t* offsets,
+                  int32_t* perm, void* workspace, size_t ws_bytes, void* stream) {
+  if (!ids || !counts || !offsets || !perm) return IQK_EINVAL;
+  if (T < 1 || topk < 1 || topk > 16 || experts < 1) return IQK_EINVAL;
+  if (T > 65536 || experts > 50000) return IQK_EUNSUPPORTED;
+  int rc;
+  if ((rc = check_ws(workspace, ws_bytes, iqk_route_workspace_bytes(T, topk, experts)))) return rc;
+  char* ws = (char*)workspace;
+  return from_launch(launch_route(ids, T, topk, experts, counts, offsets, perm, reinterpret_cast<int32_t*>(ws),
+                                  reinterpret_cast<int32_t*>(ws + align256(16)), (cudaStream_t)stream));
+}
+
+int iqk_floor(const iqk_weights* w, const int32_t* expert_list, int32_t n_experts, uint32_t* out, void* stream) {
+  WDev wd;
+  int rc;
+  if ((rc = check_weights(w, &wd))) return rc;
+  if (!expert_list || !out || n_experts < 1) return IQK_EINVAL;
+  const int sms = num_sms();
+  if (sms < 0) return cuda_fail(cudaGetLastError());
+  return from_launch(launch_floor(wd, w->fmt, expert_list, n_experts, out, (cudaStream_t)stream, sms));
+}
+
+}  // extern "C"

@@ -1,0 +1,162 @@
+// Device-side building blocks shared by the IQ2_KS / IQ2_K kernels (sm_100a).
+//
+// Stream geometry follows the mlx-iqk 0.1.1 project page, section "Format"
+// (IQ2_KS: 2-bit codes, 32-weight sub-blocks with a 5-bit signed scale index
+// split over scl/sch, an alphabet bit, an fp16 row scale; IQ2_K: 16-weight
+// sub-blocks with a 4-bit offset-8 index and an alphabet bit, fp16 scale per
+// 256 weights). The bit packing inside scl/sch/sex is documented in iqk.h.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace iqk {
+
+enum : int { FMT_KS = 0, FMT_K = 1 };
+
+// Device view of one stacked weight tensor.
+struct WDev {
+  const uint32_t* qs;
+  const uint32_t* scl;
+  const uint8_t* sch;
+  const void* sex;
+  const uint16_t* dv;
+  int32_t experts, rows, cols;
+};
+
+struct Values {
+  float v[8];
+};
+
+// Per-row element counts of each plane.
+template <int FMT>
+struct Geo {
+  static __host__ __device__ __forceinline__ int64_t qs_w(int cols) { return cols / 16; }
+  static __host__ __device__ __forceinline__ int64_t scl_w(int cols) { return FMT == FMT_KS ? cols / 256 : cols / 128; }
+  static __host__ __device__ __forceinline__ int64_t sub_n(int cols) { return cols / 256; }  // sch / sex entries
+  static __host__ __device__ __forceinline__ int64_t dv_n(int cols) { return FMT == FMT_KS ? 1 : cols / 256; }
+};
+
+// ------------------------------------------------------------------ PTX helpers
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t s) {
+  uint32_t d;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(s));
+  return d;
+}
+
+// D = A(16x16 bf16, row) * B(16x8 bf16, col) + C, fp32 accumulate.
+__device__ __forceinline__ void mma_bf16(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                         uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
+}
+
+__device__ __forceinline__ void fence_mbar_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void fence_proxy_async() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
+               "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Bounded wait on an mbarrier phase. Returns false if the bound expired.
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity,
+                                                  uint32_t max_iters = (1u << 24)) {
+  for (uint32_t i = 0; i < max_iters; i++) {
+    if (mbar_try_wait(bar, parity)) return true;
+  }
+  return false;
+}
+
+// 2-D tiled TMA load (no multicast) into shared memory, completion on `bar`.
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int32_t x, int32_t y,
+                                            uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, "
+      "%3}], [%4];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
+      : "memory");
+}
+
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+__device__ __forceinline__ uint2 ld_nc_u2(const void* p) {
+  uint2 r;
+  asm volatile("ld.global.nc.v2.u32 {%0,%1}, [%2];" : "=r"(r.x), "=r"(r.y) : "l"(p));
+  return r;
+}
+
+// bf16 helpers (bit patterns)
+__device__ __forceinline__ float bf16_bits_to_f32(uint16_t b) { return __uint_as_float((uint32_t)b << 16); }
+__device__ __forceinline__ uint16_t f32_to_bf16_bits(float f) {
+  return __bfloat16_as_ushort(__float2bfloat16_rn(f));
+}
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
+// ------------------------------------------------------------- code lookup
+//
+// The tensor-core operand for one qs word and one "slot" i (0..3): the bytes
+// of u = (q >> 2i) & 0x03030303 hold the codes of weights i, i+4, i+8, i+12
+// of the word. With a 4-entry table laid out as bf16 entry c at bytes
+// (2c, 2c+1) of the pair {t0, t1}, the byte-permute selector of a code is
+// 0x22*c + 0x10 (nibbles 2c, 2c+1); one multiply-add builds the selectors of
+// four codes at once (the FMA pipe), and each permute yields two weights.
+struct Pair2 {
+  uint32_t lo, hi;  // bf16x2 (w_i, w_{i+4}) and (w_{i+8}, w_{i+12})
+};
+
+__device__ __forceinline__ Pair2 lookup_slot(uint32_t q, int i, uint32_t t0, uint32_t t1) {
+  uint32_t u = (q >> (2 * i)) & 0x03030303u;
+  uint32_t s = u * 0x22u + 0x10101010u;
+  Pair2 r;
+  r.lo = prmt(t0, t1, s);
+  r.hi = prmt(t0, t1, s >> 16);
+  return r;
+}
+
+// Position of k within its 16-group after the slot transpose used by the
+// activation operand: element k = 16w + i + 4j lives at 16w + 4i + j.
+__host__ __device__ __forceinline__ int perm16(int k) {
+  return (k & ~15) | ((k & 3) << 2) | ((k >> 2) & 3);
+}
+
+}  // namespace iqk

@@ -1,0 +1,89 @@
+// Internal interface between the C-ABI layer (iqk_api.cu) and the kernel
+// translation units. Not installed; not part of the public ABI.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "iqk_device.cuh"
+
+namespace iqk {
+
+// ---------------------------------------------------------------- dequant
+int launch_dequant(const WDev& w, int fmt, int expert, const Values& V, void* out, bool bf16,
+                   cudaStream_t st, int num_sms);
+
+// ------------------------------------------------------- decode (GEMV-type)
+// Unit geometry shared by the GEMV-shaped kernels: 16-row tiles, each unit a
+// run of `nb` 256-weight blocks of one tile ("k-chunk"), split over `nkc`
+// chunks per row.
+struct Chunking {
+  int nb;     // blocks per unit (1, 2 or 4)
+  int nkc;    // chunks per row = blocks_per_row / nb
+  int tiles;  // ceil(rows / 16)
+};
+Chunking chunking(int rows, int cols);
+
+constexpr int kTile = 16;
+constexpr int kDecodeWarps = 4;
+constexpr int kStages = 2;
+constexpr int kMaxPairs = 1024;  // decode: T * topk
+
+// Workspace carve-up for iqk_gemv.
+struct GemvWs {
+  size_t status, xperm, cnt, part, total;
+};
+GemvWs gemv_ws(int T, int rows, int cols);
+
+// Workspace carve-up for iqk_moe_decode.
+struct DecodeWs {
+  size_t status, xperm, hperm, cnt2, cnt3, part2, part3, total;
+  int dmax, nt, nc;
+  Chunking c2, c3;
+};
+DecodeWs decode_ws(int T, int topk, int experts, int hidden, int inter);
+
+// Host-side TMA descriptor for a qs plane ([experts*rows][cols/16] uint32),
+// box [16 rows][nb*16 words]. Returns 0 on success.
+int make_qs_map(CUtensorMap* map, const WDev& w, int nb);
+
+int launch_gemv(const WDev& w, int fmt, int expert, const Values& V, const uint16_t* x, int T,
+                float* y, char* ws, cudaStream_t st, int num_sms);
+
+int launch_moe_decode(const WDev& g, int fg, const WDev& u, int fu, const WDev& d, int fd,
+                      const Values& V, const uint16_t* x, int T, const int32_t* ids, const float* p,
+                      int topk, uint16_t* y, char* ws, cudaStream_t st, int num_sms);
+
+int launch_floor(const WDev& w, int fmt, const int32_t* experts, int n, uint32_t* out, cudaStream_t st,
+                 int num_sms);
+
+// ----------------------------------------------------------------- prefill
+struct PrefillWs {
+  size_t status, counts, offsets, perm, tiles, xs, hs, outp, total;
+  int npairs, max_tiles;
+};
+PrefillWs prefill_ws(int T, int topk, int experts, int hidden, int inter);
+
+// Grouping step. `cc` is scratch of route_scratch_ints(T*topk, experts) ints.
+int launch_route(const int32_t* ids, int T, int topk, int experts, int32_t* counts, int32_t* offsets,
+                 int32_t* perm, int32_t* status, int32_t* cc, cudaStream_t st);
+inline size_t route_scratch_ints(int npairs, int experts) {
+  return (size_t)((npairs + 1023) / 1024) * experts;
+}
+
+int launch_moe_prefill(const WDev& g, int fg, const WDev& u, int fu, const WDev& d, int fd,
+                       const Values& V, const uint16_t* x, int T, const int32_t* ids, const float* p,
+                       int topk, uint16_t* y, char* ws, cudaStream_t st, int num_sms);
+
+// Driver entry point for cuTensorMapEncodeTiled (resolved once).
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*,
+                                  CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
+                                  CUtensorMapFloatOOBfill);
+EncodeTiledFn encode_tiled_fn();
+
+inline size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+}  // namespace iqk

@@ -179,10 +179,14 @@ int iqk_moe_status(const void* workspace, void* stream);
  * counts[e] = number of (token, slot) pairs routed to e; offsets[e] =
  * exclusive prefix sum (offsets[E] = number of valid pairs); perm[i] = pair
  * index t*topk + j of the i-th pair in expert order, ties in pair order.
- * counts: device int32 [E]; offsets: device int32 [E+1]; perm: device int32 [T*topk].
+ * counts: device int32 [E]; offsets: device int32 [E+1]; perm: device int32 [T*topk]
+ * (entries past offsets[E] are left unwritten when ids are out of range).
+ * workspace: >= iqk_route_workspace_bytes(T, topk, E) bytes, 256-B aligned;
+ * its first word is the status word read by iqk_moe_status. E <= 50000.
  * Page: prefill "honouring the caller's sort flag so each expert's weights are
  * read once per sorted prefill" (section "Surface").
  */
+size_t iqk_route_workspace_bytes(int32_t T, int32_t topk, int32_t experts);
 int iqk_moe_route(const int32_t* ids, int32_t T, int32_t topk, int32_t experts, int32_t* counts,
                   int32_t* offsets, int32_t* perm, void* workspace, size_t ws_bytes,
                   void* stream);

@@ -183,11 +183,31 @@ class _Cache:
         return self.m[e]
 
 
+def silu_grad(g: np.ndarray) -> np.ndarray:
+    s = 1.0 / (1.0 + np.exp(-g))
+    return s * (1.0 + g * (1.0 - s))
+
+
+def bf16_spacing(v: np.ndarray) -> np.ndarray:
+    """Distance between consecutive bfloat16 numbers at |v| (normal range)."""
+    a = np.maximum(np.abs(v), 2.0 ** -126)
+    return 2.0 ** (np.floor(np.log2(a)) - 7)
+
+
 def moe(gate, up, down, values, x_bits, ids, p, tokens=None):
     """Routed-expert block for the listed tokens (all by default).
 
-    Returns dict with y_bits (bf16 [n, hidden]), y (float64 before the final
-    rounding), S (tolerance scale, float64) and h_bits (bf16 [n, topk, inter]).
+    Returns dict with
+      y_bits  bf16 [n, hidden], the rounded output;
+      y       float64 [n, hidden] before the final rounding;
+      S       sum_j p_j sum_k |Wd_jk h_jk|: the tolerance scale of the down GEMV;
+      S_prop  sum_j p_j sum_k |Wd_jk| (|dh/dg| S_g + |dh/du| S_u)_k: how far y
+              can move when g and u are each off by their own GEMV scale
+              S_g = sum |Wg x|, S_u = sum |Wu x| (first-order propagation
+              through h = silu(g) u);
+      S_round sum_j p_j sum_k |Wd_jk| * spacing_bf16(h_jk): y's reach when h
+              rounds to the neighbouring bfloat16;
+      h_bits  bf16 [n, topk, inter].
     """
     x_bits = np.atleast_2d(x_bits)
     ids = np.atleast_2d(ids)
@@ -198,19 +218,28 @@ def moe(gate, up, down, values, x_bits, ids, p, tokens=None):
     H, F = down.rows, down.cols
     y = np.zeros((len(toks), H))
     S = np.zeros((len(toks), H))
+    S_prop = np.zeros((len(toks), H))
+    S_round = np.zeros((len(toks), H))
     hb = np.zeros((len(toks), topk, F), np.uint16)
     for n, t in enumerate(toks):
         x = bf16_to_float(x_bits[t]).astype(np.float64)
+        ax = np.abs(x)
         for j in range(topk):
             e = int(ids[t, j])
-            g = Wg(e) @ x
-            u = Wu(e) @ x
+            wg, wu = Wg(e), Wu(e)
+            g = wg @ x
+            u = wu @ x
             hb[n, j] = bf16_round((silu(g) * u).astype(np.float32))
             h = bf16_to_float(hb[n, j]).astype(np.float64)
             wd = Wd(e)
-            y[n] += float(p[t, j]) * (wd @ h)
-            S[n] += float(p[t, j]) * (np.abs(wd) @ np.abs(h))
-    return dict(y_bits=bf16_round(y.astype(np.float32)), y=y, S=S, h_bits=hb)
+            pj = float(p[t, j])
+            awd = np.abs(wd)
+            y[n] += pj * (wd @ h)
+            S[n] += pj * (awd @ np.abs(h))
+            reach = np.abs(u * silu_grad(g)) * (np.abs(wg) @ ax) + np.abs(silu(g)) * (np.abs(wu) @ ax)
+            S_prop[n] += pj * (awd @ reach)
+            S_round[n] += pj * (awd @ bf16_spacing(h))
+    return dict(y_bits=bf16_round(y.astype(np.float32)), y=y, S=S, S_prop=S_prop, S_round=S_round, h_bits=hb)
 
 
 # ----------------------------------------------------------------- route prep

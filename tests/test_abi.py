@@ -1,0 +1,93 @@
+"""The C-ABI library loads, exports every declared entry point and rejects bad
+arguments on the host before touching a GPU (no compute calls here)."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+from gemm_iq2_ks_b200 import binding as B
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_symbols():
+    src = open(os.path.join(ROOT, "include", "iqk.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(iqk_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_header_declares_the_binding_exports():
+    assert set(declared_symbols()) == set(B.EXPORTS)
+
+
+def test_library_exports_every_declared_symbol():
+    L = B.lib()
+    for name in declared_symbols():
+        assert hasattr(L, name), name
+
+
+def test_row_bytes_and_version():
+    L = B.lib()
+    assert L.iqk_version() == 1
+    assert L.iqk_row_bytes(0, 4096) == 2 + 70 * 4096 // 256
+    assert L.iqk_row_bytes(1, 2048) == 76 * 2048 // 256
+    assert L.iqk_row_bytes(0, 100) == -1
+    assert L.iqk_row_bytes(7, 256) == -1
+
+
+def _w(fmt=0, experts=1, rows=16, cols=256, sch=True):
+    return B.IqkWeights(fmt, experts, rows, cols, 4096, 4096, 4096 if sch else None, 4096, 4096)
+
+
+def test_host_validation_rejects_before_any_launch():
+    L = B.lib()
+    v = np.zeros(8, np.float32)
+    P = v.ctypes.data
+    bad = [
+        (_w(cols=100), B.IQK_ESHAPE),
+        (_w(cols=0), B.IQK_ESHAPE),
+        (_w(rows=0), B.IQK_ESHAPE),
+        (_w(fmt=5), B.IQK_EINVAL),
+        (_w(fmt=1, sch=True), B.IQK_EINVAL),   # IQ2_K takes no sch plane
+        (_w(fmt=0, sch=False), B.IQK_EINVAL),  # IQ2_KS needs it
+    ]
+    for w, rc in bad:
+        assert L.iqk_dequant(ctypes.byref(w), 0, P, 4096, None) == rc
+    w = _w()
+    assert L.iqk_dequant(ctypes.byref(w), 1, P, 4096, None) == B.IQK_EINVAL  # expert out of range
+    assert L.iqk_dequant(ctypes.byref(w), 0, None, 4096, None) == B.IQK_EINVAL  # no table
+    assert L.iqk_dequant(None, 0, P, 4096, None) == B.IQK_EINVAL
+    # gemv: token count and workspace
+    assert L.iqk_gemv(ctypes.byref(w), 0, P, 4096, 65, 4096, 4096, 1 << 20, None) == B.IQK_EUNSUPPORTED
+    assert L.iqk_gemv(ctypes.byref(w), 0, P, 4096, 1, 4096, None, 0, None) == B.IQK_EWORKSPACE
+    assert L.iqk_gemv(ctypes.byref(w), 0, P, 4096, 1, 4096, 4097, 1 << 20, None) == B.IQK_EWORKSPACE
+
+
+def test_moe_shape_checks():
+    L = B.lib()
+    v = np.zeros(8, np.float32).ctypes.data
+    g = _w(experts=4, rows=512, cols=256)
+    u = _w(experts=4, rows=512, cols=256)
+    d = _w(experts=4, rows=256, cols=512)
+    d_bad = _w(experts=4, rows=256, cols=768)
+    e_bad = _w(experts=3, rows=256, cols=512)
+    args = lambda dd, T=1, k=6: (ctypes.byref(g), ctypes.byref(u), ctypes.byref(dd), v, 4096, T, 4096, 4096, k,
+                                 4096, None, 0, None)
+    assert L.iqk_moe_decode(*args(d_bad)) == B.IQK_EINVAL
+    assert L.iqk_moe_decode(*args(e_bad)) == B.IQK_EINVAL
+    assert L.iqk_moe_decode(*args(d, k=17)) == B.IQK_EINVAL
+    assert L.iqk_moe_decode(*args(d, T=65)) == B.IQK_EUNSUPPORTED
+    assert L.iqk_moe_decode(*args(d, T=0)) == B.IQK_OK  # empty call is a no-op
+    assert L.iqk_moe_decode(*args(d)) == B.IQK_EWORKSPACE
+    assert L.iqk_moe_prefill(*args(d, T=70000)) == B.IQK_EUNSUPPORTED
+    assert L.iqk_moe_workspace_bytes(0, 65, 6, 4, 256, 512) == 0
+    assert L.iqk_moe_workspace_bytes(0, 1, 6, 4, 256, 512) > 0
+
+
+def test_strerror_covers_every_status():
+    L = B.lib()
+    for rc in range(0, -7, -1):
+        assert L.iqk_strerror(rc) not in (b"", b"unknown status")
+    assert L.iqk_strerror(-99) == b"unknown status"

@@ -1,0 +1,239 @@
+"""GPU parity: dequantization, GEMV, routed decode, grouping and the floor arm,
+each through the C ABI against the CPU oracle on the same seeded inputs."""
+import numpy as np
+import pytest
+
+import iqk_synth as S
+from oracle import oracle as O
+from tests.encode import encode, idx_range, sub_size
+from tests.util import check_fp32, check_moe, from_dev_bf16, to_dev_bf16
+
+pytestmark = pytest.mark.gpu
+
+torch = pytest.importorskip("torch")
+
+
+@pytest.fixture(scope="module")
+def B():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from gemm_iq2_ks_b200 import binding
+    binding.lib()
+    return binding
+
+
+def bits_equal(a, b):
+    return np.array_equal(np.asarray(a, np.float32).view(np.uint32), np.asarray(b, np.float32).view(np.uint32))
+
+
+# ------------------------------------------------------------------ dequant
+
+@pytest.mark.parametrize("cfg", [0, 1])
+@pytest.mark.parametrize("table", ["int", "f16"])
+def test_dequant_bitexact_configs(B, cfg, table):
+    w, _, _ = S.matrix_case(cfg)
+    values = S.value_table(table, cfg)
+    dw = B.Weights.from_host(w)
+    got = B.iqk_dequant(dw, 0, values).cpu().numpy()
+    assert bits_equal(got, O.dequant_expert(w, 0, values))
+
+
+@pytest.mark.parametrize("fmt", ["iq2_ks", "iq2_k"])
+def test_dequant_edge_fields_multi_expert(B, fmt):
+    """Zero/subnormal/negative scales, every index, ragged row count, expert > 0."""
+    rng = np.random.default_rng(41)
+    rows, cols = 37, 768
+    experts = []
+    for e in range(3):
+        lo, hi = idx_range(fmt)
+        nsub = cols // sub_size(fmt)
+        codes = rng.integers(0, 4, size=(rows, cols))
+        idx = rng.integers(lo, hi + 1, size=(rows, nsub))
+        alpha = rng.integers(0, 2, size=(rows, nsub))
+        dshape = (rows,) if fmt == "iq2_ks" else (rows, cols // 256)
+        d = rng.uniform(1e-3, 1e-2, size=dshape).astype(np.float16)
+        m = rng.random(dshape)
+        d[m < 0.1] = (rng.integers(1, 1024, size=(m < 0.1).sum()) * 2.0 ** -24).astype(np.float16)
+        d[(m >= 0.1) & (m < 0.15)] = 0
+        d *= rng.choice([-1, 1], size=dshape).astype(np.float16)
+        experts.append(encode(fmt, codes, idx, alpha, d.view(np.uint16)))
+    st = S.Streams(fmt, 3, rows, cols, *[None if getattr(experts[0], k) is None else
+                                         np.concatenate([getattr(x, k) for x in experts])
+                                         for k in ("qs", "scl", "sch", "sex", "dv")])
+    values = S.value_table("f16", 9)
+    dw = B.Weights.from_host(st)
+    for e in range(3):
+        got = B.iqk_dequant(dw, e, values).cpu().numpy()
+        assert bits_equal(got, O.dequant_expert(st, e, values)), e
+
+
+@pytest.mark.parametrize("cfg", [0, 1])
+def test_dequant_bf16_is_rounded_fp32(B, cfg):
+    w, _, _ = S.matrix_case(cfg)
+    values = S.value_table("f16", cfg)
+    dw = B.Weights.from_host(w)
+    got = B.iqk_dequant_bf16(dw, 0, values).view(torch.int16).cpu().numpy().view(np.uint16)
+    assert np.array_equal(got, O.bf16_round(O.dequant_expert(w, 0, values)))
+
+
+# --------------------------------------------------------------------- gemv
+
+@pytest.mark.parametrize("cfg", [0, 1])
+@pytest.mark.parametrize("T", [1, 3, 8])
+def test_gemv_configs(B, cfg, T):
+    w, x, values = S.matrix_case(cfg)
+    rng = S.rng_for(100 + T)
+    x = np.concatenate([x, S.random_bf16(rng, (T - 1, w.cols))]) if T > 1 else x
+    dw = B.Weights.from_host(w)
+    y = B.iqk_gemv(dw, 0, values, to_dev_bf16(x)).cpu().numpy()
+    y_ref, Sabs = O.gemv(O.dequant_expert(w, 0, values), x)
+    check_fp32(y, y_ref, Sabs, f"gemv cfg{cfg} T={T}")
+
+
+@pytest.mark.parametrize("fmt", ["iq2_ks", "iq2_k"])
+@pytest.mark.parametrize("T", [9, 16, 33, 64])
+def test_gemv_ragged_and_many_tokens(B, fmt, T):
+    rng = S.rng_for(7 + T)
+    w = S.random_streams(rng, fmt, 2, 200, 1280)  # rows not a multiple of 16; 5 blocks
+    x = S.random_bf16(rng, (T, 1280))
+    values = S.value_table("f16", 4)
+    dw = B.Weights.from_host(w)
+    y = B.iqk_gemv(dw, 1, values, to_dev_bf16(x)).cpu().numpy()
+    y_ref, Sabs = O.gemv(O.dequant_expert(w, 1, values), x)
+    check_fp32(y, y_ref, Sabs, f"gemv {fmt} T={T}")
+
+
+# ------------------------------------------------------------- moe decode
+
+def _moe_case(seed, fg, fu, fd, E, H, F, T, topk):
+    rng = S.rng_for(seed)
+    gate = S.random_streams(rng, fg, E, F, H)
+    up = S.random_streams(rng, fu, E, F, H)
+    down = S.random_streams(rng, fd, E, H, F)
+    x = S.random_bf16(rng, (T, H))
+    ids, p = S.routing(rng, T, E, topk)
+    return gate, up, down, x, ids, p
+
+
+def _run_decode(B, gate, up, down, values, x, ids, p, prefill=False):
+    dg, du, dd = (B.Weights.from_host(w) for w in (gate, up, down))
+    fn = B.iqk_moe_prefill if prefill else B.iqk_moe_decode
+    y = fn(dg, du, dd, values, to_dev_bf16(x), torch.from_numpy(ids).cuda(), torch.from_numpy(p).cuda())
+    torch.cuda.synchronize()
+    return from_dev_bf16(y)
+
+
+@pytest.mark.parametrize("fmts", [("iq2_ks",) * 3, ("iq2_k",) * 3, ("iq2_ks", "iq2_k", "iq2_ks"),
+                                  ("iq2_k", "iq2_ks", "iq2_k")])
+@pytest.mark.parametrize("T", [1, 4, 16])
+def test_moe_decode_small(B, fmts, T):
+    gate, up, down, x, ids, p = _moe_case(50 + T, *fmts, E=12, H=512, F=768, T=T, topk=6)
+    values = S.value_table("int", 1)
+    y = _run_decode(B, gate, up, down, values, x, ids, p)
+    ref = O.moe(gate, up, down, values, x, ids, p)
+    check_moe(y, ref, f"decode {fmts} T={T}")
+
+
+def test_moe_decode_topk_edge(B):
+    """topk = 1 and topk = 16, T = 64 (the decode limits)."""
+    for T, k in [(3, 1), (64, 16)]:
+        gate, up, down, x, ids, p = _moe_case(60 + k, "iq2_ks", "iq2_ks", "iq2_k", E=40, H=256, F=256, T=T, topk=k)
+        values = S.value_table("f16", 2)
+        y = _run_decode(B, gate, up, down, values, x, ids, p)
+        ref = O.moe(gate, up, down, values, x, ids, p)
+        check_moe(y, ref, f"decode T={T} topk={k}")
+
+
+def test_moe_decode_bad_ids_skipped_and_flagged(B):
+    gate, up, down, x, ids, p = _moe_case(77, "iq2_ks", "iq2_ks", "iq2_ks", E=8, H=256, F=256, T=2, topk=3)
+    values = S.value_table("int", 0)
+    bad = ids.copy()
+    bad[0, 1] = 8
+    bad[1, 2] = -1
+    dg, du, dd = (B.Weights.from_host(w) for w in (gate, up, down))
+    ws = B.workspace(B.iqk_moe_workspace_bytes(0, 2, 3, 8, 256, 256))
+    y = B.iqk_moe_decode(dg, du, dd, values, to_dev_bf16(x), torch.from_numpy(bad).cuda(),
+                         torch.from_numpy(p).cuda(), ws=ws)
+    assert B.iqk_moe_status(ws) == B.IQK_EINVAL
+    pv = p.copy()
+    pv[0, 1] = 0.0
+    pv[1, 2] = 0.0
+    fixed = ids.copy()
+    fixed[0, 1] = 0
+    fixed[1, 2] = 0
+    ref = O.moe(gate, up, down, values, x, fixed, pv)
+    check_moe(from_dev_bf16(y), ref, "bad ids")
+    # a clean call resets the status word
+    B.iqk_moe_decode(dg, du, dd, values, to_dev_bf16(x), torch.from_numpy(ids).cuda(),
+                     torch.from_numpy(p).cuda(), ws=ws)
+    assert B.iqk_moe_status(ws) == B.IQK_OK
+
+
+# full-size geometry: 256 experts, gate/up [2048, 4096], down [4096, 2048]
+@pytest.fixture(scope="module")
+def full_ks(B):
+    rng = S.rng_for(2)
+    return S.moe_weights(rng, "iq2_ks", S.EXPERTS, S.HIDDEN, S.INTER)
+
+
+@pytest.fixture(scope="module")
+def full_k(B):
+    rng = S.rng_for(3)
+    return S.moe_weights(rng, "iq2_k", S.EXPERTS, S.HIDDEN, S.INTER)
+
+
+def test_moe_decode_full_config2(B, full_ks):
+    gate, up, down = full_ks
+    rng = S.rng_for(20)
+    x = S.random_bf16(rng, (1, S.HIDDEN))
+    ids, p = S.routing(rng, 1, S.EXPERTS, S.TOPK)
+    values = S.value_table("int", 2)
+    y = _run_decode(B, gate, up, down, values, x, ids, p)
+    ref = O.moe(gate, up, down, values, x, ids, p)
+    check_moe(y, ref, "config 2")
+
+
+@pytest.mark.parametrize("T", [1, 4, 16])
+def test_moe_decode_full_config3(B, full_k, T):
+    gate, up, down = full_k
+    rng = S.rng_for(30 + T)
+    x = S.random_bf16(rng, (T, S.HIDDEN))
+    ids, p = S.routing(rng, T, S.EXPERTS, S.TOPK)
+    values = S.value_table("f16", 3)
+    y = _run_decode(B, gate, up, down, values, x, ids, p)
+    ref = O.moe(gate, up, down, values, x, ids, p)
+    check_moe(y, ref, f"config 3 T={T}")
+
+
+# ------------------------------------------------------------------- route
+
+@pytest.mark.parametrize("T,E,k", [(1, 8, 6), (100, 16, 6), (2048, 256, 6), (3000, 1000, 4)])
+def test_route_bitexact(B, T, E, k):
+    rng = S.rng_for(T + E)
+    ids, _ = S.routing(rng, T, E, k)
+    counts, offsets, perm, _ = B.iqk_moe_route(torch.from_numpy(ids).cuda(), E)
+    c_ref, o_ref, p_ref = O.route_prep(ids, E)
+    assert np.array_equal(counts.cpu().numpy(), c_ref)
+    assert np.array_equal(offsets.cpu().numpy(), o_ref)
+    assert np.array_equal(perm.cpu().numpy(), p_ref)
+
+
+def test_route_bad_ids(B):
+    ids = np.array([[0, 5, 9], [2, 2, -3]], np.int32)
+    counts, offsets, perm, ws = B.iqk_moe_route(torch.from_numpy(ids).cuda(), 8)
+    assert B.iqk_moe_status(ws) == B.IQK_EINVAL
+    assert offsets.cpu().numpy()[-1] == 4
+    assert list(perm.cpu().numpy()[:4]) == [0, 3, 4, 1]
+
+
+# ------------------------------------------------------------------- floor
+
+@pytest.mark.parametrize("fmt,rows,cols", [("iq2_ks", 2048, 4096), ("iq2_k", 4096, 2048), ("iq2_ks", 37, 512)])
+def test_floor_xor_bitexact(B, fmt, rows, cols):
+    rng = S.rng_for(rows)
+    w = S.random_streams(rng, fmt, 4, rows, cols)
+    dw = B.Weights.from_host(w)
+    elist = torch.tensor([3, 1], dtype=torch.int32, device="cuda")
+    out = B.iqk_floor(dw, elist).cpu().numpy().view(np.uint32)
+    assert np.array_equal(out[0], O.floor_xor(w, 3))
+    assert np.array_equal(out[1], O.floor_xor(w, 1))

@@ -289,6 +289,21 @@ def test_constant_scale_reduces_to_table_lookup_and_matvec():
 
 # ---------------------------------------------------------------------- moe
 
+def test_silu_grad_matches_central_difference():
+    g = np.linspace(-30, 30, 2001)
+    h = 1e-6
+    num = (O.silu(g + h) - O.silu(g - h)) / (2 * h)
+    assert np.allclose(O.silu_grad(g), num, rtol=1e-7, atol=1e-9)
+
+
+def test_bf16_spacing_is_the_gap_to_the_next_bfloat16():
+    torch = pytest.importorskip("torch")
+    v = np.array([1.0, 1.5, 3.0, 1e-3, 7e4, -2.5], np.float64)
+    t = torch.tensor(v, dtype=torch.bfloat16)
+    nxt = torch.nextafter(t.abs(), torch.tensor(float("inf"), dtype=torch.bfloat16))
+    assert np.allclose(O.bf16_spacing(v), (nxt - t.abs()).double().numpy(), rtol=0, atol=0)
+
+
 def test_silu_matches_scipy():
     special = pytest.importorskip("scipy.special")
     g = np.linspace(-40, 40, 10001)
