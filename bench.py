@@ -1,0 +1,510 @@
+"""Benchmark: routed-expert decode (and prefill) on B200 through the C ABI.
+
+Headline (N=1 and every rank at N>1): IQ2_KS routed-expert decode, one token
+per call, 256 experts, top-6, gate/up [2048 x 4096], down [4096 x 2048]
+(seeded synthetic streams, bf16 N(0,1) activations, softmax routing weights).
+A step is one decode call; consecutive calls take their experts from a chain
+of random permutations, so no expert repeats within 42 calls and the 41 MB a
+call reads are never resident in the 126 MB L2. Steps are captured once into
+CUDA graphs and replayed; device time comes from CUDA events on the launching
+stream, max over ranks.
+
+Printed: one JSON line (rank 0).
+"""
+from __future__ import annotations
+
+import argparse
+import faulthandler
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import iqk_synth as S  # noqa: E402
+
+METRIC = "MoE decode µs/token & weight GB/s vs HBM floor; prefill bf16 TFLOP/s"
+RING = 420  # calls per captured graph (10 permutation cycles of 42 calls)
+
+
+def env_int(k, d):
+    try:
+        return int(os.environ.get(k, d))
+    except ValueError:
+        return d
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return dict(hbm_gbs=float(d["hbm_gbs"]), bf16=float(d["bf16_tflops"]),
+                    bf16_sustained=float(d.get("bf16_tflops_sustained", d["bf16_tflops"])), source="measured")
+    return dict(hbm_gbs=6650.0, bf16=1590.0, bf16_sustained=1400.0, source="fallback")
+
+
+# ---------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons with nvidia-smi (100 ms period)
+    while the timed region runs; only this GPU's lines (by PCI bus id) count."""
+
+    REASONS = {
+        0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x10: "sync_boost",
+        0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+        0x100: "display_clock_setting",
+    }
+
+    def __init__(self, props):
+        # nvidia-smi prints e.g. 00000000:1B:00.0; match on bus:device.function
+        try:
+            self.bus = f"{int(props.pci_bus_id):02x}:{int(props.pci_device_id):02x}.0"
+        except Exception:
+            self.bus = ""
+        self.samples, self.max_mhz, self.reasons = [], None, set()
+        self.proc = None
+
+    def __enter__(self):
+        import subprocess
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "--query-gpu=pci.bus_id,clocks.sm,clocks.max.sm,clocks_event_reasons.active",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is None:
+            return
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except Exception:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        for line in out.splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 4 or (self.bus and not f[0].lower().endswith(self.bus)):
+                continue
+            try:
+                self.samples.append(float(f[1]))
+                self.max_mhz = float(f[2])
+                r = int(f[3], 16)
+            except ValueError:
+                continue
+            for bit, name in self.REASONS.items():
+                if r & bit:
+                    self.reasons.add(name)
+
+    def summary(self):
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+# ---------------------------------------------------------------- helpers
+
+def cuda_time(torch, stream, fn):
+    """Device seconds of fn's work: fn runs with `stream` current (graph
+    replays launch on the current stream) between two events on it."""
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        a.record(stream)
+        fn()
+        b.record(stream)
+    b.synchronize()
+    return a.elapsed_time(b) * 1e-3  # seconds
+
+
+def log(msg):
+    print(f"[bench {time.strftime('%H:%M:%S')}] {msg}", file=sys.stderr, flush=True)
+
+
+def capture(torch, stream, fn):
+    """Capture fn's launches into a CUDA graph. Every C-ABI path captured here
+    has run once eagerly first, so no attribute/occupancy query happens
+    inside the capture."""
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(stream):
+        with torch.cuda.graph(g, stream=stream):
+            fn()
+    return g
+
+
+def run_steps(graphs, K):
+    """Replay graphs so that exactly K steps run (full rings, then a remainder)."""
+    full, rem_graphs = graphs
+    for _ in range(K // RING):
+        full.replay()
+    r = K % RING
+    if r:
+        rem_graphs[r].replay()
+
+
+class DecodeBench:
+    """One routed-expert decode workload (format, token count) resident on the GPU."""
+
+    def __init__(self, torch, B, weights, values, T, seed, device, stream, remainders=()):
+        self.torch, self.B, self.T, self.stream = torch, B, T, stream
+        gate, up, down = weights
+        E = gate.experts
+        self.dw = [B.Weights.from_host(w, device) for w in weights]
+        self.host_w = weights
+        rng = S.rng_for(seed)
+        ids = np.empty((RING, T, S.TOPK), np.int32)
+        p = np.empty((RING, T, S.TOPK), np.float32)
+        if T == 1:
+            ids, p = S.routing_ring(rng, RING, E, S.TOPK)
+        else:
+            for c in range(RING):
+                ids[c], p[c] = S.routing(rng, T, E, S.TOPK)
+        x = S.random_bf16(rng, (RING, T, S.HIDDEN))
+        self.ids_h, self.p_h, self.x_h = ids, p, x
+        self.ids = torch.from_numpy(ids).to(device)
+        self.p = torch.from_numpy(p).to(device)
+        self.x = torch.from_numpy(x.view(np.int16)).to(device).view(torch.bfloat16)
+        self.y = torch.empty((RING, T, S.HIDDEN), dtype=torch.bfloat16, device=device)
+        ws_bytes = B.iqk_moe_workspace_bytes(0, T, S.TOPK, E, S.HIDDEN, S.INTER)
+        self.ws = B.workspace(ws_bytes, device)
+        self.distinct = np.array([len(np.unique(ids[c])) for c in range(RING)])
+        self.bytes_per_expert = sum(w.nbytes() // w.experts for w in weights)
+        self.values = values
+        self.remainders = remainders
+
+    def call(self, c):
+        B = self.B
+        g, u, d = self.dw
+        B.iqk_moe_decode(g, u, d, self.values, self.x[c], self.ids[c], self.p[c], y=self.y[c], ws=self.ws,
+                         stream=self.stream)
+
+    def graphs(self):
+        torch = self.torch
+        with torch.cuda.stream(self.stream):
+            self.call(0)
+        torch.cuda.synchronize()
+        full = capture(torch, self.stream, lambda: [self.call(c) for c in range(RING)])
+        rem = {r: capture(torch, self.stream, lambda r=r: [self.call(c) for c in range(r)]) for r in self.remainders}
+        return full, rem
+
+    def weight_bytes(self, calls):
+        return float(sum(self.distinct[c % RING] for c in range(calls))) * self.bytes_per_expert
+
+
+def e2e_graph(torch, bench, stream, n):
+    """n steps, each: pinned-host x/ids/p -> device, decode, y -> pinned host."""
+    T = bench.T
+    hx = torch.empty((n, T, S.HIDDEN), dtype=torch.bfloat16, pin_memory=True)
+    hx.copy_(bench.x[:n].cpu())
+    hids = bench.ids[:n].cpu().pin_memory()
+    hp = bench.p[:n].cpu().pin_memory()
+    hy = torch.empty((n, T, S.HIDDEN), dtype=torch.bfloat16, pin_memory=True)
+    dx = torch.empty((T, S.HIDDEN), dtype=torch.bfloat16, device=bench.x.device)
+    dids = torch.empty((T, S.TOPK), dtype=torch.int32, device=bench.x.device)
+    dp = torch.empty((T, S.TOPK), dtype=torch.float32, device=bench.x.device)
+    dy = torch.empty((T, S.HIDDEN), dtype=torch.bfloat16, device=bench.x.device)
+    g, u, d = bench.dw
+
+    with torch.cuda.stream(stream):
+        bench.B.iqk_moe_decode(g, u, d, bench.values, bench.x[0], bench.ids[0], bench.p[0], y=dy, ws=bench.ws,
+                               stream=stream)
+    torch.cuda.synchronize()
+
+    def body():
+        for c in range(n):
+            dx.copy_(hx[c], non_blocking=True)
+            dids.copy_(hids[c], non_blocking=True)
+            dp.copy_(hp[c], non_blocking=True)
+            bench.B.iqk_moe_decode(g, u, d, bench.values, dx, dids, dp, y=dy, ws=bench.ws, stream=stream)
+            hy[c].copy_(dy, non_blocking=True)
+
+    graph = capture(torch, stream, body)
+    h2d = T * S.HIDDEN * 2 + T * S.TOPK * 4 * 2
+    d2h = T * S.HIDDEN * 2
+    return graph, h2d, d2h, hy
+
+
+def floor_graph(torch, bench, stream, n):
+    """The deleted-decode address floor over the same experts, n calls."""
+    B = bench.B
+    g, u, d = bench.dw
+    lists = [torch.from_numpy(np.unique(bench.ids_h[c]).astype(np.int32)).to(bench.x.device) for c in range(n)]
+    outs = [(torch.empty((len(l), g.rows), dtype=torch.int32, device=bench.x.device),
+             torch.empty((len(l), d.rows), dtype=torch.int32, device=bench.x.device)) for l in lists]
+
+    with torch.cuda.stream(stream):
+        B.iqk_floor(g, lists[0], out=outs[0][0], stream=stream)
+        B.iqk_floor(d, lists[0], out=outs[0][1], stream=stream)
+    torch.cuda.synchronize()
+
+    def body():
+        for c in range(n):
+            B.iqk_floor(g, lists[c], out=outs[c][0], stream=stream)
+            B.iqk_floor(u, lists[c], out=outs[c][0], stream=stream)
+            B.iqk_floor(d, lists[c], out=outs[c][1], stream=stream)
+
+    return capture(torch, stream, body)
+
+
+# ------------------------------------------------------------ cpu oracle
+
+def oracle_decode_seconds(weights, values, budget_s, seed=99):
+    """Time the CPU oracle (as it stands) on whole single-token decode calls of
+    the same workload until ``budget_s`` of CPU work has run."""
+    from oracle import oracle as O
+    try:
+        from threadpoolctl import threadpool_limits
+        limiter = threadpool_limits(limits=1)
+    except Exception:
+        limiter = None
+    gate, up, down = weights
+    rng = S.rng_for(seed)
+    tokens, t0 = 0, time.perf_counter()
+    while True:
+        x = S.random_bf16(rng, (1, S.HIDDEN))
+        ids, p = S.routing(rng, 1, S.EXPERTS, S.TOPK)
+        O.moe(gate, up, down, values, x, ids, p)
+        tokens += 1
+        el = time.perf_counter() - t0
+        if el >= budget_s:
+            break
+    if limiter is not None:
+        limiter.unregister() if hasattr(limiter, "unregister") else None
+    return el / tokens, tokens
+
+
+def oracle_pair_sample_seconds(weights, values, rows_per_matrix, seed):
+    """One bounded sample of the decode work: dequantize and multiply
+    ``rows_per_matrix`` rows of the gate, up and down matrices of one routed
+    expert (the oracle's own functions). Returns (seconds, weights processed)."""
+    from oracle import oracle as O
+    gate, up, down = weights
+    rng = S.rng_for(seed)
+    e = int(rng.integers(0, S.EXPERTS))
+    t0 = time.perf_counter()
+    n = 0
+    for w in (gate, up, down):
+        r0 = int(rng.integers(0, w.rows - rows_per_matrix + 1))
+        sl = slice(r0, r0 + rows_per_matrix)
+        dq = O.dequant(w.fmt, rows_per_matrix, w.cols, w.qs[e, sl], w.scl[e, sl],
+                       None if w.sch is None else w.sch[e, sl], w.sex[e, sl], w.dv[e, sl], values)
+        x = S.random_bf16(rng, (1, w.cols))
+        O.gemv(dq, x)
+        n += rows_per_matrix * w.cols
+    return time.perf_counter() - t0, n
+
+
+def decode_weights_per_token():
+    return S.TOPK * (2 * S.INTER * S.HIDDEN + S.HIDDEN * S.INTER)
+
+
+def config_block(extra=None):
+    c = {"workload": "routed-expert decode, IQ2_KS, 1 token/call, 256 experts top-6, gate/up 2048x4096, "
+                     "down 4096x2048 (config 2)",
+         "global_batch": 1, "experts": S.EXPERTS, "topk": S.TOPK, "hidden": S.HIDDEN, "inter": S.INTER,
+         "format": "iq2_ks", "parallelism": "replicas",
+         "l2": "inputs larger than L2: consecutive calls' experts come from a chain of random "
+               "permutations (no expert reused within 42 calls; 1.77 GB resident, 41 MB per call)"}
+    if extra:
+        c.update(extra)
+    return c
+
+
+# ------------------------------------------------------------------ main
+
+def run_reference(args):
+    """The CPU oracle as the reference arm (rank 0 only)."""
+    rank = env_int("RANK", 0)
+    if rank != 0:
+        return 0
+    rng = S.rng_for(2)
+    weights = S.moe_weights(rng, "iq2_ks", S.EXPERTS, S.HIDDEN, S.INTER)
+    values = S.value_table("int", 2)
+    # each step: a bounded sample of one token's work (rows of one expert's three matrices)
+    rows = 64
+    per_token = decode_weights_per_token()
+    for w in range(args.warmup):
+        oracle_pair_sample_seconds(weights, values, rows, 1000 + w)
+    tot_s, tot_n = 0.0, 0
+    for k in range(args.steps):
+        s, n = oracle_pair_sample_seconds(weights, values, rows, 2000 + k)
+        tot_s += s
+        tot_n += n
+    us_per_token = tot_s / tot_n * per_token * 1e6
+    sample = (f"each step dequantizes and multiplies {rows} rows of each of the gate, up and down matrices of one "
+              f"routed expert ({tot_n // max(args.steps, 1)} weights); us/token = time per weight x "
+              f"{per_token} weights per token")
+    line = {"impl": "reference", "metric": METRIC, "value": us_per_token, "unit": "us/token",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": tot_s / max(args.steps, 1) * 1e3, "higher_is_better": False, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": config_block(),
+            "cpu_baseline": {"value": us_per_token, "unit": "us/token", "cores": 1, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": us_per_token, "unit": "us/token", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    faulthandler.enable()
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=250 * RING)
+    ap.add_argument("--warmup", type=int, default=RING)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work for cpu_baseline")
+    ap.add_argument("--no-details", action="store_true")
+    ap.add_argument("--profile", choices=["decode"], default=None,
+                    help="plain launches without graphs or reporting (for ncu captures)")
+    ap.add_argument("--experts", type=int, default=S.EXPERTS,
+                    help="experts resident in --profile mode (fewer keeps ncu captures small)")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        return run_reference(args)
+
+    import torch
+    world = env_int("WORLD_SIZE", 1)
+    rank = env_int("RANK", 0)
+    local = env_int("LOCAL_RANK", 0)
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=device)
+
+    from gemm_iq2_ks_b200 import binding as B
+    B.lib()
+    peaks = measured_peaks()
+    stream = torch.cuda.Stream(device)
+
+    if args.profile == "decode":
+        rng = S.rng_for(2)
+        w_ks = S.moe_weights(rng, "iq2_ks", args.experts, S.HIDDEN, S.INTER)
+        dec = DecodeBench(torch, B, w_ks, S.value_table("int", 2), 1, 20, device, stream)
+        with torch.cuda.stream(stream):
+            for c in range(args.warmup + args.steps):
+                dec.call(c % RING)
+        torch.cuda.synchronize()
+        return 0
+
+    # ---------------- headline: config 2 decode
+    log("generating config 2 weights")
+    rng = S.rng_for(2 + 1000 * rank)
+    w_ks = S.moe_weights(rng, "iq2_ks", S.EXPERTS, S.HIDDEN, S.INTER)
+    values = S.value_table("int", 2)
+    K, W = args.steps, args.warmup
+    rems = sorted({K % RING, W % RING} - {0})
+    dec = DecodeBench(torch, B, w_ks, values, 1, 20 + rank, device, stream, remainders=rems)
+    log("capturing decode graphs")
+    graphs = dec.graphs()
+    torch.cuda.synchronize()
+    log("warmup")
+    with torch.cuda.stream(stream):
+        run_steps(graphs, W)
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(torch.cuda.get_device_properties(device)) as clk:
+        t = cuda_time(torch, stream, lambda: run_steps(graphs, K))
+    torch.cuda.synchronize()
+    if dist:
+        tt = torch.tensor([t], device=device)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        dist.barrier()
+        t = float(tt.item())
+    tokens_all = K * 1 * world
+    us_per_token = t / tokens_all * 1e6 if world > 1 else t / K * 1e6
+    bytes_per_call = dec.weight_bytes(K) / K
+    gbs = bytes_per_call * K / t / 1e9
+
+    log(f"decode timed: {t / K * 1e6:.2f} us/call")
+    # e2e through the C ABI with host buffers (copies inside the timed region)
+    ng = min(RING, K)
+    eg, h2d, d2h, _ = e2e_graph(torch, dec, stream, ng)
+    with torch.cuda.stream(stream):
+        eg.replay()
+    torch.cuda.synchronize()
+    reps = max(1, K // ng)
+    te = cuda_time(torch, stream, lambda: [eg.replay() for _ in range(reps)])
+    e2e_us = te / (reps * ng) * 1e6
+
+    log(f"e2e: {e2e_us:.2f} us/token")
+    # floor arm on the same experts (identical loads, decode removed)
+    fg = floor_graph(torch, dec, stream, ng)
+    with torch.cuda.stream(stream):
+        fg.replay()
+    torch.cuda.synchronize()
+    tf = cuda_time(torch, stream, lambda: [fg.replay() for _ in range(reps)])
+    floor_us = tf / (reps * ng) * 1e6
+
+    log(f"floor: {floor_us:.2f} us/call")
+    details = {}
+    if not args.no_details and rank == 0:
+        # config 3 (IQ2_K): T = 1, 4, 16
+        rng3 = S.rng_for(3)
+        w_k = S.moe_weights(rng3, "iq2_k", S.EXPERTS, S.HIDDEN, S.INTER)
+        for T in (1, 4, 16):
+            db = DecodeBench(torch, B, w_k, S.value_table("f16", 3), T, 30 + T, device, stream)
+            gr = db.graphs()
+            with torch.cuda.stream(stream):
+                run_steps(gr, RING)
+            torch.cuda.synchronize()
+            tt3 = cuda_time(torch, stream, lambda: run_steps(gr, 2 * RING))
+            per_call = tt3 / (2 * RING)
+            by = db.weight_bytes(2 * RING) / (2 * RING)
+            details[f"config3_T{T}"] = {"us_per_call": per_call * 1e6, "us_per_token": per_call / T * 1e6,
+                                        "weight_gbs": by / per_call / 1e9,
+                                        "hbm_frac": by / per_call / 1e9 / peaks["hbm_gbs"],
+                                        "mean_distinct_experts": float(db.distinct.mean())}
+            del db, gr
+        del w_k
+        torch.cuda.empty_cache()
+
+    launches = 3 * K
+    line = {
+        "metric": METRIC, "value": us_per_token, "unit": "us/token", "n_gpus": world, "steps": K, "warmup": W,
+        "ms_per_step": t / K * 1e3, "higher_is_better": False, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16", "data": "synthetic", "config": config_block({"format": "iq2_ks", "global_batch": world}),
+        "weight_gbs": gbs, "hbm_frac": gbs / peaks["hbm_gbs"],
+        "floor": {"us_per_token": floor_us, "decode_over_floor": us_per_token / floor_us if world == 1 else
+                  (t / K * 1e6) / floor_us},
+        "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": gbs / peaks["hbm_gbs"], "traffic": None,
+                     "kernel": "one decode call (prep + gate/up+SwiGLU + down+combine, PDL-chained)",
+                     "peak_source": peaks["source"] + " hbm_gbs (copy)"},
+        "e2e": {"value": e2e_us, "unit": "us/token", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": launches,
+        "clocks": clk.summary(),
+        "details": details,
+    }
+    if rank == 0 and world >= 1:
+        log("cpu baseline (oracle)")
+        sec, ntok = oracle_decode_seconds(w_ks, values, args.cpu_budget)
+        line["cpu_baseline"] = {"value": sec * 1e6, "unit": "us/token", "cores": 1, "kind": "oracle",
+                                "sample": f"{ntok} whole single-token decode calls of config 2 "
+                                          f"(fresh routing each), one thread"}
+    if dist:
+        dist.barrier()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    del graphs
+    if dist:
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -55,7 +55,10 @@ def _stamp() -> str:
 
 def up_to_date() -> bool:
     stamp = os.path.join(OUT_DIR, "stamp")
-    return os.path.exists(LIB) and os.path.exists(stamp) and open(stamp).read() == _stamp()
+    if not (os.path.exists(LIB) and os.path.exists(stamp)):
+        return False
+    with open(stamp) as f:
+        return f.read() == _stamp()
 
 
 def build(force: bool = False, verbose: bool = False) -> str:

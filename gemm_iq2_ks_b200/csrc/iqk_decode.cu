@@ -830,11 +830,39 @@ static size_t ring_bytes(int mats, int nb) {
 
 static int nt_for(int cols_needed) { return cols_needed <= 8 ? 1 : cols_needed <= 16 ? 2 : cols_needed <= 32 ? 4 : 8; }
 
+// Per (kernel, dynamic smem) caches so that a call made during stream
+// capture issues no attribute or occupancy queries after the first call.
+struct KernelCache {
+  const void* fn;
+  size_t smem_set;
+  size_t occ_smem;
+  int occ;
+};
+static KernelCache g_kcache[256];
+static int g_kcache_n = 0;
+
+static KernelCache* kcache(const void* fn) {
+  for (int i = 0; i < g_kcache_n; i++)
+    if (g_kcache[i].fn == fn) return &g_kcache[i];
+  if (g_kcache_n == 256) return nullptr;
+  g_kcache[g_kcache_n] = KernelCache{fn, 0, (size_t)-1, 0};
+  return &g_kcache[g_kcache_n++];
+}
+
 template <typename K>
 static int occupancy_grid(K kernel, size_t smem, int units_max, int num_sms) {
+  KernelCache* kc = kcache(reinterpret_cast<const void*>(kernel));
   int per_sm = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kDecodeWarps * 32, smem) != cudaSuccess)
-    return -1;
+  if (kc && kc->occ_smem == smem) {
+    per_sm = kc->occ;
+  } else {
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kDecodeWarps * 32, smem) != cudaSuccess)
+      return -1;
+    if (kc) {
+      kc->occ_smem = smem;
+      kc->occ = per_sm;
+    }
+  }
   if (per_sm < 1) return -1;
   per_sm = std::min(per_sm, 2);
   int want = (units_max + kDecodeWarps - 1) / kDecodeWarps;
@@ -843,7 +871,11 @@ static int occupancy_grid(K kernel, size_t smem, int units_max, int num_sms) {
 
 template <typename K>
 static int set_smem(K kernel, size_t smem) {
-  return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) == cudaSuccess ? 0 : -4;
+  KernelCache* kc = kcache(reinterpret_cast<const void*>(kernel));
+  if (kc && kc->smem_set >= smem) return 0;
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess) return -4;
+  if (kc) kc->smem_set = smem;
+  return 0;
 }
 
 static cudaLaunchAttribute pdl_attr() {

@@ -169,7 +169,10 @@ def gemv(w: np.ndarray, x_bits) -> tuple[np.ndarray, np.ndarray]:
 # ------------------------------------------------------------------------ moe
 
 def silu(g: np.ndarray) -> np.ndarray:
-    return g / (1.0 + np.exp(-g))
+    """g / (1 + exp(-g)); exp(-g) may overflow to inf for very negative g,
+    where the quotient's limit -0/0 is the right value."""
+    with np.errstate(over="ignore"):
+        return g / (1.0 + np.exp(-g))
 
 
 class _Cache:
@@ -184,7 +187,8 @@ class _Cache:
 
 
 def silu_grad(g: np.ndarray) -> np.ndarray:
-    s = 1.0 / (1.0 + np.exp(-g))
+    with np.errstate(over="ignore"):
+        s = 1.0 / (1.0 + np.exp(-g))
     return s * (1.0 + g * (1.0 - s))
 
 
