@@ -51,8 +51,9 @@ int check_weights(const iqk_weights* w, WDev* out) {
   if (w->cols <= 0 || w->cols % 256) return IQK_ESHAPE;
   if (!w->qs || !w->scl || !w->sex || !w->dv) return IQK_EINVAL;
   if ((w->fmt == IQK_IQ2_KS) != (w->sch != nullptr)) return IQK_EINVAL;
-  if (!aligned(w->qs, 16) || !aligned(w->scl, 4) || !aligned(w->dv, 2)) return IQK_EINVAL;
-  if (w->fmt == IQK_IQ2_K && !aligned(w->sex, 2)) return IQK_EINVAL;
+  // planes are staged by TMA / bulk copies: every base 16-byte aligned
+  if (!aligned(w->qs, 16) || !aligned(w->scl, 16) || !aligned(w->sex, 16) || !aligned(w->dv, 16)) return IQK_EINVAL;
+  if (w->sch && !aligned(w->sch, 16)) return IQK_EINVAL;
   if ((int64_t)w->experts * w->rows >= (int64_t)1 << 31) return IQK_ESHAPE;
   out->qs = w->qs;
   out->scl = w->scl;

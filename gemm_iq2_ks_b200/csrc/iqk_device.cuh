@@ -53,13 +53,17 @@ __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t s) {
 }
 
 // D = A(16x16 bf16, row) * B(16x8 bf16, col) + C, fp32 accumulate.
-__device__ __forceinline__ void mma_bf16(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
-                                         uint32_t a3, uint32_t b0, uint32_t b1) {
+__device__ __forceinline__ void mma_bf16_4(float& d0, float& d1, float& d2, float& d3, uint32_t a0, uint32_t a1,
+                                           uint32_t a2, uint32_t a3, uint32_t b0, uint32_t b1) {
   asm volatile(
       "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
       "{%8,%9}, {%0,%1,%2,%3};"
-      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "+f"(d0), "+f"(d1), "+f"(d2), "+f"(d3)
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ void mma_bf16(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                         uint32_t b0, uint32_t b1) {
+  mma_bf16_4(d[0], d[1], d[2], d[3], a0, a1, a2, a3, b0, b1);
 }
 
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
@@ -150,6 +154,32 @@ __device__ __forceinline__ Pair2 lookup_slot(uint32_t q, int i, uint32_t t0, uin
   Pair2 r;
   r.lo = prmt(t0, t1, s);
   r.hi = prmt(t0, t1, s >> 16);
+  return r;
+}
+
+// Same, with the high selector's 16-bit shift done as a multiply-high by
+// `k65536` (= 65536, held in a register the compiler cannot fold), which runs
+// on the FMA pipe instead of the integer-logic pipe the permutes use.
+__device__ __forceinline__ Pair2 lookup_slot_mh(uint32_t q, int i, uint32_t t0, uint32_t t1, uint32_t k65536) {
+  uint32_t u = (q >> (2 * i)) & 0x03030303u;
+  uint32_t s = u * 0x22u + 0x10101010u;
+  uint32_t sh;
+  asm("mul.hi.u32 %0, %1, %2;" : "=r"(sh) : "r"(s), "r"(k65536));
+  Pair2 r;
+  r.lo = prmt(t0, t1, s);
+  r.hi = prmt(t0, t1, sh);
+  return r;
+}
+
+__device__ __forceinline__ uint32_t opaque_u32(uint32_t v) {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %1;" : "=r"(r) : "r"(v));
+  return r;
+}
+
+__device__ __forceinline__ uint4 ld_nc_u4(const void* p) {
+  uint4 r;
+  asm volatile("ld.global.nc.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w) : "l"(p));
   return r;
 }
 

@@ -28,7 +28,7 @@ Chunking chunking(int rows, int cols);
 
 constexpr int kTile = 16;
 constexpr int kDecodeWarps = 4;
-constexpr int kStages = 2;
+constexpr int kStages = 4;
 constexpr int kMaxPairs = 1024;  // decode: T * topk
 
 // Workspace carve-up for iqk_gemv.

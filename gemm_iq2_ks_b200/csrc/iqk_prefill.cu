@@ -128,7 +128,8 @@ __device__ __forceinline__ bool pf_wait(uint64_t* bar, uint32_t par, volatile ui
 template <int MODE, int F0, int F1>
 __global__ void __launch_bounds__(PF_THREADS, 1) k_pf_gemm(const __grid_constant__ CUtensorMap q0,
                                                            const __grid_constant__ CUtensorMap q1,
-                                                           const __grid_constant__ CUtensorMap bmap, PfArgs A) {
+                                                           const __grid_constant__ CUtensorMap bmap,
+                                                           const __grid_constant__ PfArgs A) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
   uint8_t* bbuf = smem;                                   // [SB][128 rows][128 B], 1024-aligned

@@ -47,6 +47,8 @@
  *     ids) is checked on the device: bad ids are skipped and recorded in the
  *     workspace status word (iqk_moe_status).
  *   - bf16 and fp16 values are passed as their 16-bit patterns (uint16_t).
+ *   - Every stream plane's base address must be 16-byte aligned (the planes
+ *     are staged into shared memory by TMA and bulk copies); IQK_EINVAL if not.
  */
 #ifndef IQK_H_
 #define IQK_H_
