@@ -6,60 +6,76 @@
 // values[4*alphabet+code] (section "Format"); pricing against "identical
 // loads, decode removed" (section "Pricing").
 //
-// Work is cut into units of 16 weight rows x one k-chunk (nb 256-weight
-// blocks). Each warp owns a two-stage ring in shared memory: one elected lane
-// stages a unit's qs tile with a 2-D TMA load (no multicast), the warp decodes
-// it against a per-CTA table of bf16(scale_index * value) entries with
-// byte-permutes and reduces with m16n8k16 tensor-core MMAs (tokens or pairs
-// as the MMA's N). Partial sums of a tile's k-chunks meet in the workspace;
-// the last unit to finish a tile (device-scope counter) sums them in chunk
-// order, so results do not depend on arrival order.
+// Work is cut into items of 16 weight rows x `bpi` 256-weight blocks (a
+// slice of the reduction width). Each warp owns a ring of item stages in
+// shared memory: one elected lane loads an item's qs tile with a 2-D TMA
+// (no multicast) while the lanes copy the item's scale slice with cp.async
+// onto the same mbarrier; the warp decodes the tile against a per-CTA table
+// of bf16(scale_index * value) entries with byte-permutes and reduces with
+// m16n8k16 tensor-core MMAs (tokens or pairs as the MMA's N). The slices of
+// a tile meet in the workspace; the last item to finish a tile (device-scope
+// counter) sums them in slice order, so results do not depend on arrival
+// order.
 #include <algorithm>
 
 #include "iqk_device.cuh"
 #include "iqk_internal.h"
 
+// Selector arithmetic of the code lookup: 0 all shifts on the integer-logic
+// pipe; 1 the high-half selector by multiply-high; 2 as 1, plus slot 2's
+// pre-shift by multiply-high (integer-logic and FMA pipes about even).
+#ifndef IQK_LOOKUP
+#define IQK_LOOKUP 2
+#endif
+
 namespace iqk {
+
+// Blocks per item: four when the row's block count allows (the scale slices
+// then start on the boundaries cp.async needs), else two or one.
+int item_blocks(int cols) {
+  const int nbk = cols / 256;
+  return nbk % 4 == 0 ? 4 : nbk % 2 == 0 ? 2 : 1;
+}
 
 Chunking chunking(int rows, int cols) {
   Chunking c;
   const int nbk = cols / 256;
-  c.nb = (nbk % 2 == 0) ? 2 : 1;
+  c.nb = item_blocks(cols);
   c.nkc = nbk / c.nb;
   c.tiles = (rows + kTile - 1) / kTile;
   return c;
 }
 
-// ---------------------------------------------------------- unit scales
-// A unit's scale planes (16 rows, full reduction width) sit in a per-warp
-// shared-memory slot with the global layout of those rows:
-//   IQ2_KS: scl [16][nbk] u32 | sch [16][nbk] u8 | sex [16][nbk] u8 | dv [16] u16
-//   IQ2_K:  scl [16][2 nbk] u32 | sex [16][nbk] u16 | dv [16][nbk] u16
-// (nbk = 256-weight blocks per row). Every part starts on a 16-byte boundary.
+// ---------------------------------------------------------- item scales
+// An item's scale slice (16 rows x bpi blocks) sits in a per-stage slot:
+//   IQ2_KS: scl [16][bpi] u32 | sch [16][bpi] u8 | sex [16][bpi] u8
+//   IQ2_K:  scl [16][2 bpi] u32 | sex [16][bpi] u16 | dv [16][bpi] u16
+// Every part starts on a 16-byte boundary (bpi = 1, 2 or 4). The IQ2_KS row
+// scale is read straight from global memory at the start of the item.
 template <int FMT>
 struct Slot {
-  static __host__ __device__ __forceinline__ uint32_t scl_off(int) { return 0; }
-  static __host__ __device__ __forceinline__ uint32_t b_off(int nbk) { return FMT == FMT_KS ? 64u * nbk : 128u * nbk; }
-  static __host__ __device__ __forceinline__ uint32_t c_off(int nbk) { return FMT == FMT_KS ? 80u * nbk : 160u * nbk; }
-  static __host__ __device__ __forceinline__ uint32_t bytes(int nbk) { return FMT == FMT_KS ? 96u * nbk + 32u : 192u * nbk; }
+  static __host__ __device__ __forceinline__ uint32_t b_off(int bpi) { return FMT == FMT_KS ? 64u * bpi : 128u * bpi; }
+  static __host__ __device__ __forceinline__ uint32_t c_off(int bpi) { return FMT == FMT_KS ? 80u * bpi : 160u * bpi; }
+  static __host__ __device__ __forceinline__ uint32_t bytes(int bpi) { return FMT == FMT_KS ? 96u * bpi : 192u * bpi; }
 };
 
+// Bytes between consecutive slots: the larger format's slot, rounded up to
+// 128 so that every ring stage and slot keeps a 128-byte aligned base.
 template <int F0, int F1>
-__host__ __device__ inline uint32_t slot_bytes2(int nbk) {
-  const uint32_t a = Slot<F0>::bytes(nbk), b = Slot<F1>::bytes(nbk);
-  return a > b ? a : b;
+__host__ __device__ inline uint32_t slot_bytes2(int bpi) {
+  const uint32_t a = Slot<F0>::bytes(bpi), b = Slot<F1>::bytes(bpi);
+  return ((a > b ? a : b) + 127u) & ~127u;
 }
 
-// Table indices of the sub-blocks covering words 4t..4t+3 of block kb of row r.
+// Table indices of the sub-blocks covering words 4t..4t+3 of slot block lb of row r.
 // IQ2_KS: (low4 | high<<4) + 32*alphabet, words (4t, 4t+1) in sub-block 2t.
 // IQ2_K:  nibble + 16*alphabet, word 4t+m is sub-block 4t+m.
 template <int FMT>
-__device__ __forceinline__ void combos_smem(const uint8_t* slot, int nbk, int r, int kb, int t, uint32_t (&c)[4]) {
+__device__ __forceinline__ void combos_smem(const uint8_t* slot, int bpi, int r, int lb, int t, uint32_t (&c)[4]) {
   if constexpr (FMT == FMT_KS) {
-    const uint32_t s = reinterpret_cast<const uint32_t*>(slot)[r * nbk + kb];
-    const uint32_t h = slot[Slot<FMT>::b_off(nbk) + r * nbk + kb];
-    const uint32_t a = slot[Slot<FMT>::c_off(nbk) + r * nbk + kb];
-    const uint32_t sb = (s >> (8 * t)) & 0xFFu;
+    const uint32_t sb = slot[(r * bpi + lb) * 4 + t];
+    const uint32_t h = slot[Slot<FMT>::b_off(bpi) + r * bpi + lb];
+    const uint32_t a = slot[Slot<FMT>::c_off(bpi) + r * bpi + lb];
     const uint32_t hb = (h >> (2 * t)) & 3u;
     const uint32_t ab = (a >> (2 * t)) & 3u;
     const uint32_t c0 = (sb & 15u) | ((hb & 1u) << 4) | ((ab & 1u) << 5);
@@ -69,20 +85,17 @@ __device__ __forceinline__ void combos_smem(const uint8_t* slot, int nbk, int r,
     c[2] = c1;
     c[3] = c1;
   } else {
-    const uint32_t sw = reinterpret_cast<const uint32_t*>(slot)[r * 2 * nbk + 2 * kb + (t >> 1)] >> (16 * (t & 1));
-    const uint32_t x = (reinterpret_cast<const uint16_t*>(slot + Slot<FMT>::b_off(nbk))[r * nbk + kb] >> (4 * t)) & 15u;
+    const uint32_t sw = reinterpret_cast<const uint16_t*>(slot)[(r * 2 * bpi + 2 * lb) * 2 + t];
+    const uint32_t x = (reinterpret_cast<const uint16_t*>(slot + Slot<FMT>::b_off(bpi))[r * bpi + lb] >> (4 * t)) & 15u;
 #pragma unroll
     for (int m = 0; m < 4; m++) c[m] = ((sw >> (4 * m)) & 15u) | (((x >> m) & 1u) << 4);
   }
 }
 
-// Row scale d: IQ2_KS per row, IQ2_K per (row, block).
-template <int FMT>
-__device__ __forceinline__ float d_smem(const uint8_t* slot, int nbk, int r, int kb) {
-  // IQ2_KS: dv follows the 16 * nbk sex bytes; IQ2_K: dv is the third plane
-  const uint16_t* dv =
-      reinterpret_cast<const uint16_t*>(slot + Slot<FMT>::c_off(nbk) + (FMT == FMT_KS ? 16u * nbk : 0u));
-  return __half2float(__ushort_as_half(FMT == FMT_KS ? dv[r] : dv[r * nbk + kb]));
+// IQ2_K scale d of (row r, slot block lb).
+__device__ __forceinline__ float d_smem_k(const uint8_t* slot, int bpi, int r, int lb) {
+  const uint16_t* dv = reinterpret_cast<const uint16_t*>(slot + Slot<FMT_K>::c_off(bpi));
+  return __half2float(__ushort_as_half(dv[r * bpi + lb]));
 }
 
 // Entry c of the table: bf16 of scale_index * values[4*alphabet + code] for
@@ -108,11 +121,36 @@ __device__ __forceinline__ void build_lut(uint2* lut, const Values& V) {
   }
 }
 
+// 16-byte activation fragment: from shared memory (BSM) or the read-only path.
+template <bool BSM>
+__device__ __forceinline__ uint4 ld_act(const uint16_t* p) {
+  if constexpr (BSM) {
+    uint4 r;
+    asm("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w) : "r"(smem_u32(p)));
+    return r;
+  } else {
+    return ld_nc_u4(p);
+  }
+}
+
+__device__ __forceinline__ Pair2 lookup(uint32_t q, int i, uint32_t t0, uint32_t t1, uint32_t k65536) {
+#if IQK_LOOKUP == 0
+  (void)k65536;
+  return lookup_slot(q, i, t0, t1);
+#elif IQK_LOOKUP == 1
+  return lookup_slot_mh(q, i, t0, t1, k65536);
+#else
+  // 2^28 = 65536 << 12, kept opaque through k65536
+  if (i == 2) return lookup_slot_mh2(q, t0, t1, k65536, k65536 << 12);
+  return lookup_slot_mh(q, i, t0, t1, k65536);
+#endif
+}
+
 // One 256-weight block of a 16-row tile: part[m] += W(16 x 64 of word m) * B.
 // Each of the block's four qs words feeds its own accumulator set, so
 // consecutive MMAs do not wait on each other; half a block's activation
 // fragments are requested ahead of their MMAs.
-template <int FMT, int NT>
+template <int FMT, int NT, bool BSM>
 __device__ __forceinline__ void block_mma(const uint32_t* __restrict__ sq, int ldw, int bcol, const uint16_t* const (&src)[NT],
                                           const uint32_t (&cg)[4], const uint32_t (&ch)[4],
                                           const uint2* __restrict__ lut, float (&part)[4][NT][4], int g, int t,
@@ -122,7 +160,7 @@ __device__ __forceinline__ void block_mma(const uint32_t* __restrict__ sq, int l
 #pragma unroll
   for (int n = 0; n < NT; n++)
 #pragma unroll
-    for (int f = 0; f < 4; f++) bf[n][f] = src[n] ? ld_nc_u4(src[n] + 8 * f) : make_uint4(0u, 0u, 0u, 0u);
+    for (int f = 0; f < 4; f++) bf[n][f] = ld_act<BSM>(src[n] + 8 * f);
   const uint4 qg = *reinterpret_cast<const uint4*>(sq + g * ldw + bcol + 4 * t);
   const uint4 qh = *reinterpret_cast<const uint4*>(sq + (g + 8) * ldw + bcol + 4 * t);
 #pragma unroll
@@ -131,7 +169,7 @@ __device__ __forceinline__ void block_mma(const uint32_t* __restrict__ sq, int l
 #pragma unroll
       for (int n = 0; n < NT; n++)
 #pragma unroll
-        for (int f = 0; f < 4; f++) bf[n][f] = src[n] ? ld_nc_u4(src[n] + 32 + 8 * f) : make_uint4(0u, 0u, 0u, 0u);
+        for (int f = 0; f < 4; f++) bf[n][f] = ld_act<BSM>(src[n] + 32 + 8 * f);
     }
     const uint32_t wg = m == 0 ? qg.x : m == 1 ? qg.y : m == 2 ? qg.z : qg.w;
     const uint32_t wh = m == 0 ? qh.x : m == 1 ? qh.y : m == 2 ? qh.z : qh.w;
@@ -139,14 +177,76 @@ __device__ __forceinline__ void block_mma(const uint32_t* __restrict__ sq, int l
     const uint2 th = lut[ch[m]];
 #pragma unroll
     for (int i = 0; i < 4; i++) {
-      const Pair2 pg = lookup_slot_mh(wg, i, tg.x, tg.y, k65536);
-      const Pair2 ph = lookup_slot_mh(wh, i, th.x, th.y, k65536);
+      const Pair2 pg = lookup(wg, i, tg.x, tg.y, k65536);
+      const Pair2 ph = lookup(wh, i, th.x, th.y, k65536);
 #pragma unroll
       for (int n = 0; n < NT; n++) {
         const uint4 b4 = bf[n][2 * (m & 1) + (i >> 1)];
         const uint32_t b0 = (i & 1) ? b4.z : b4.x, b1 = (i & 1) ? b4.w : b4.y;
         mma_bf16_4(part[m][n][0], part[m][n][1], part[m][n][2], part[m][n][3], pg.lo, ph.lo, pg.hi, ph.hi, b0, b1);
       }
+    }
+  }
+}
+
+// One item (16 rows x bpi blocks) of a matrix in format F0 (fmt0) or F1:
+// acc[n] = d * sum over the item's blocks of W * B, rows g and g + 8.
+template <int F0, int F1, int NT, bool BSM>
+__device__ __forceinline__ void item_mma(const uint32_t* sq, const uint8_t* slot, int bpi, int ldw,
+                                         const uint16_t* const (&bsrc)[NT], bool fmt0, bool kfmt, const uint2* lut0,
+                                         const uint2* lut1, float dg, float dh, int g, int t, uint32_t k65536,
+                                         float (&acc)[NT][4]) {
+  constexpr int BLKE = BSM ? 320 : 256;  // elements between consecutive 256-weight blocks
+  float part[4][NT][4];
+#pragma unroll
+  for (int m = 0; m < 4; m++)
+#pragma unroll
+    for (int n = 0; n < NT; n++)
+#pragma unroll
+      for (int q = 0; q < 4; q++) part[m][n][q] = 0.f;
+  for (int b = 0; b < bpi; b++) {
+    const uint16_t* src[NT];
+#pragma unroll
+    for (int n = 0; n < NT; n++) {
+      src[n] = bsrc[n] + BLKE * b;
+      if (!BSM && b + 1 < bpi) prefetch_l1(src[n] + BLKE);
+    }
+    uint32_t cg[4], ch[4];
+    if (fmt0) {
+      combos_smem<F0>(slot, bpi, g, b, t, cg);
+      combos_smem<F0>(slot, bpi, g + 8, b, t, ch);
+    } else {
+      combos_smem<F1>(slot, bpi, g, b, t, cg);
+      combos_smem<F1>(slot, bpi, g + 8, b, t, ch);
+    }
+    if (kfmt) {
+#pragma unroll
+      for (int m = 0; m < 4; m++)
+#pragma unroll
+        for (int n = 0; n < NT; n++)
+#pragma unroll
+          for (int q = 0; q < 4; q++) part[m][n][q] = 0.f;
+    }
+    block_mma<F0, NT, BSM>(sq, ldw, b * 16, src, cg, ch, fmt0 ? lut0 : lut1, part, g, t, k65536);
+    if (kfmt) {  // IQ2_K: d changes every block
+      const float kdg = d_smem_k(slot, bpi, g, b);
+      const float kdh = d_smem_k(slot, bpi, g + 8, b);
+#pragma unroll
+      for (int n = 0; n < NT; n++) {
+        acc[n][0] = fmaf(kdg, (part[0][n][0] + part[1][n][0]) + (part[2][n][0] + part[3][n][0]), acc[n][0]);
+        acc[n][1] = fmaf(kdg, (part[0][n][1] + part[1][n][1]) + (part[2][n][1] + part[3][n][1]), acc[n][1]);
+        acc[n][2] = fmaf(kdh, (part[0][n][2] + part[1][n][2]) + (part[2][n][2] + part[3][n][2]), acc[n][2]);
+        acc[n][3] = fmaf(kdh, (part[0][n][3] + part[1][n][3]) + (part[2][n][3] + part[3][n][3]), acc[n][3]);
+      }
+    }
+  }
+  if (!kfmt) {
+#pragma unroll
+    for (int n = 0; n < NT; n++) {
+      acc[n][0] = dg * ((part[0][n][0] + part[1][n][0]) + (part[2][n][0] + part[3][n][0]));
+      acc[n][1] = dg * ((part[0][n][1] + part[1][n][1]) + (part[2][n][1] + part[3][n][1]));
+      acc[n][2] = dh * ((part[0][n][2] + part[1][n][2]) + (part[2][n][2] + part[3][n][2]));
+      acc[n][3] = dh * ((part[0][n][3] + part[1][n][3]) + (part[2][n][3] + part[3][n][3]));
     }
   }
 }
@@ -265,18 +365,17 @@ __global__ void __launch_bounds__(256) k_prep(const uint16_t* __restrict__ x, in
 }
 
 // ------------------------------------------------------------ stream kernel
-// One kernel for the GEMV-shaped jobs and the floor arm. A unit is 16 rows of
-// one matrix over the full reduction width; its columns are the tokens (GEMV)
-// or the (token, slot) pairs routed to one distinct expert. Each warp streams
-// its units through a ring of kStages chunks (CH 256-weight blocks of the
-// unit's qs, by 2-D TMA); a unit's scale planes arrive by 1-D bulk copy into
-// one of kStages per-warp slots together with its first chunk, so loads run
-// kStages chunks ahead of the decode.
-//   GEMV:   y[t][row] = acc (fp32).
-//   GATEUP: gate and up units of a tile write partials; the tile's second
-//           unit forms h = bf16(silu(g) * u) in the slot-transposed layout.
-//   DOWN:   p-weighted partials per (tile, pair); the tile's last unit sums
-//           each token's slots in slot order into y (bf16).
+// One kernel for the GEMV-shaped jobs and the floor arm. An item is 16 rows
+// of one matrix over a slice of `bpi` blocks of the reduction width; its
+// columns are the tokens (GEMV) or the (token, slot) pairs routed to one
+// distinct expert. Each warp streams its items through a ring of kStages
+// stages, one item per stage, so loads run up to kStages items ahead of the
+// decode.
+//   GEMV:   slices of a tile meet in the workspace; y[t][row] = sum (fp32).
+//   GATEUP: gate and up slices of a tile write partials; the tile's last
+//           item forms h = bf16(silu(g) * u) in the slot-transposed layout.
+//   DOWN:   partials per (tile, pair, slice); the tile's last item sums each
+//           token's slots in slot order, weighted by p, into y (bf16).
 //   FLOOR:  identical loads; the decode is replaced by an XOR of every loaded
 //           byte into out[expert][row].
 enum : int { MODE_GEMV = 0, MODE_GATEUP = 1, MODE_DOWN = 2, MODE_FLOOR = 3 };
@@ -286,119 +385,146 @@ struct UnitArgs {
   Values V;
   const int32_t* ids;
   const float* p;
-  const uint16_t* act;  // slot-transposed activation rows
+  const uint16_t* act;   // slot-transposed activation rows (read-only path)
+  const uint16_t* xraw;  // BSM: the activation rows as given, transposed on the way into shared memory
   int T, topk, expert;
   const int32_t* elist;  // FLOOR: experts to stream
   int nexp;
   float* yf;        // GEMV output [T][rows]
   uint16_t* out16;  // GATEUP: h [pairs][inter]; DOWN: y [T][hidden]
-  uint32_t* outx;   // FLOOR: [nexp][rows]
+  uint32_t* outx;   // FLOOR: [nexp][rows], zeroed before the launch
   int32_t* cnt;
   float* part;
   int32_t* status;
-  int ch;  // blocks per chunk
+  int bpi;       // 256-weight blocks per item
+  int splits;    // items per tile and matrix (blocks per row / bpi)
+  int async_sc;  // scale slices by cp.async (bpi == 4)
+  int act_rows;  // BSM: activation rows copied into shared memory
+  FastDiv div_s, div_tiles;
 };
 
-struct Ring {
-  uint32_t* qs;    // [kStages][16][ldw]
-  uint8_t* slots;  // [kStages][slot bytes]
-  uint64_t* bar;   // [kStages]
-};
-
-__device__ __forceinline__ void bulk_copy(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
-  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-                   smem_u32(dst)),
-               "l"(src), "r"(bytes), "r"(smem_u32(bar))
-               : "memory");
+__device__ __forceinline__ void cp_async4(void* dst, const void* src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async8(void* dst, const void* src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
+// The mbarrier's current phase also waits for this thread's earlier cp.async copies.
+__device__ __forceinline__ void cp_async_arrive(uint64_t* bar) {
+  asm volatile("cp.async.mbarrier.arrive.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 
-// Stage the scale planes of rows [row0, row0 + 16) of `w` into `slot`.
-// A full tile whose four source ranges all start on 16-byte boundaries is
-// bulk-copied (the returned byte count is what the caller expects on the
-// barrier; the copies are issued when `issue` is set). Any other tile (past
-// the last row, or a shape whose rows do not fall on 16-byte boundaries) is
-// filled by the lanes with plain loads, zeros past the last row; that path
-// returns 0 and ends with __syncwarp.
+// Stage the scale slice of rows [R0, R0 + valid) and blocks [s*bpi, (s+1)*bpi)
+// of `w` into `slot`. With `async` (bpi == 4, so every row piece is 4-, 8- or
+// 16-byte aligned) the lanes issue cp.async copies tracked by `bar`;
+// otherwise they copy with plain loads, zero past the last row, and the call
+// ends with __syncwarp.
 template <int FMT>
-__device__ __forceinline__ uint32_t stage_scales(uint8_t* slot, const WDev& w, int64_t row0, int valid_rows,
-                                                 uint64_t* bar, int lane, bool issue) {
+__device__ __forceinline__ void stage_scales(uint8_t* slot, const WDev& w, int64_t R0, int valid, int s, int bpi,
+                                             bool async, uint64_t* bar, int lane) {
   const int nbk = w.cols / 256;
-  const uint32_t b_scl = FMT == FMT_KS ? 64u * nbk : 128u * nbk;  // 16 rows of scl
-  const uint32_t b_b = FMT == FMT_KS ? 16u * nbk : 32u * nbk;     // 16 rows of sch (KS) / sex (K)
-  const uint32_t b_c = FMT == FMT_KS ? 16u * nbk : 32u * nbk;     // 16 rows of sex (KS) / dv (K)
-  const uint8_t* src_scl = reinterpret_cast<const uint8_t*>(w.scl) + row0 * (b_scl / 16);
-  const uint8_t* src_b = FMT == FMT_KS ? w.sch + row0 * nbk
-                                       : reinterpret_cast<const uint8_t*>(reinterpret_cast<const uint16_t*>(w.sex) + row0 * nbk);
-  const uint8_t* src_c = FMT == FMT_KS ? reinterpret_cast<const uint8_t*>(w.sex) + row0 * nbk
-                                       : reinterpret_cast<const uint8_t*>(w.dv + row0 * nbk);
-  const uint8_t* src_d = reinterpret_cast<const uint8_t*>(w.dv + row0);  // IQ2_KS row scales
-  const uintptr_t mis = (reinterpret_cast<uintptr_t>(src_scl) | reinterpret_cast<uintptr_t>(src_b) |
-                         reinterpret_cast<uintptr_t>(src_c) | (FMT == FMT_KS ? reinterpret_cast<uintptr_t>(src_d) : 0)) &
-                        15u;
-  if (valid_rows == kTile && mis == 0) {
-    if (issue) {
-      bulk_copy(slot, src_scl, b_scl, bar);
-      bulk_copy(slot + Slot<FMT>::b_off(nbk), src_b, b_b, bar);
-      bulk_copy(slot + Slot<FMT>::c_off(nbk), src_c, b_c, bar);
-      if (FMT == FMT_KS) bulk_copy(slot + Slot<FMT>::c_off(nbk) + b_c, src_d, 32u, bar);
+  if (async) {
+    if (FMT == FMT_KS) {
+      const int r = lane & 15;
+      if (r < valid) {
+        const int64_t o = (R0 + r) * nbk + 4 * s;
+        if (lane < 16) {
+          cp_async16(slot + 16 * r, w.scl + o);
+        } else {
+          cp_async4(slot + 256 + 4 * r, w.sch + o);
+          cp_async4(slot + 320 + 4 * r, reinterpret_cast<const uint8_t*>(w.sex) + o);
+        }
+      }
+    } else {
+      const int r = lane >> 1, h = lane & 1;
+      if (r < valid) cp_async16(slot + 32 * r + 16 * h, w.scl + (R0 + r) * 2 * nbk + 8 * s + 4 * h);
+      const int r2 = lane & 15;
+      if (r2 < valid) {
+        const int64_t o = (R0 + r2) * nbk + 4 * s;
+        if (lane < 16) cp_async8(slot + 512 + 8 * r2, reinterpret_cast<const uint16_t*>(w.sex) + o);
+        else cp_async8(slot + 640 + 8 * r2, w.dv + o);
+      }
     }
-    return b_scl + b_b + b_c + (FMT == FMT_KS ? 32u : 0u);
+    cp_async_arrive(bar);
+    return;
   }
-  if (issue) return 0;
-  const uint32_t per_scl = b_scl / 16, per_b = b_b / 16, per_c = b_c / 16;  // bytes per row
-  for (uint32_t i = lane; i < b_scl / 4; i += 32) {
-    const bool ok = (int)(i / (per_scl / 4)) < valid_rows;
-    reinterpret_cast<uint32_t*>(slot)[i] = ok ? __ldg(reinterpret_cast<const uint32_t*>(src_scl) + i) : 0u;
-  }
-  uint8_t* sb = slot + Slot<FMT>::b_off(nbk);
-  for (uint32_t i = lane; i < b_b; i += 32) sb[i] = (int)(i / per_b) < valid_rows ? __ldg(src_b + i) : (uint8_t)0;
-  uint8_t* sc = slot + Slot<FMT>::c_off(nbk);
-  for (uint32_t i = lane; i < b_c; i += 32) sc[i] = (int)(i / per_c) < valid_rows ? __ldg(src_c + i) : (uint8_t)0;
   if (FMT == FMT_KS) {
-    uint16_t* sd = reinterpret_cast<uint16_t*>(sc + b_c);
-    for (int i = lane; i < kTile; i += 32) sd[i] = i < valid_rows ? __ldg(w.dv + row0 + i) : (uint16_t)0;
+    uint32_t* d32 = reinterpret_cast<uint32_t*>(slot);
+    for (int i = lane; i < 16 * bpi; i += 32) {
+      const int r = i / bpi, b = i - r * bpi;
+      d32[i] = r < valid ? __ldg(w.scl + (R0 + r) * nbk + s * bpi + b) : 0u;
+    }
+    uint8_t* sb = slot + Slot<FMT>::b_off(bpi);
+    uint8_t* sc = slot + Slot<FMT>::c_off(bpi);
+    for (int i = lane; i < 16 * bpi; i += 32) {
+      const int r = i / bpi, b = i - r * bpi;
+      const int64_t o = (R0 + r) * nbk + s * bpi + b;
+      sb[i] = r < valid ? __ldg(w.sch + o) : (uint8_t)0;
+      sc[i] = r < valid ? __ldg(reinterpret_cast<const uint8_t*>(w.sex) + o) : (uint8_t)0;
+    }
+  } else {
+    uint32_t* d32 = reinterpret_cast<uint32_t*>(slot);
+    for (int i = lane; i < 32 * bpi; i += 32) {
+      const int r = i / (2 * bpi), b = i - r * 2 * bpi;
+      d32[i] = r < valid ? __ldg(w.scl + (R0 + r) * 2 * nbk + 2 * s * bpi + b) : 0u;
+    }
+    uint16_t* sb = reinterpret_cast<uint16_t*>(slot + Slot<FMT>::b_off(bpi));
+    uint16_t* sc = reinterpret_cast<uint16_t*>(slot + Slot<FMT>::c_off(bpi));
+    for (int i = lane; i < 16 * bpi; i += 32) {
+      const int r = i / bpi, b = i - r * bpi;
+      const int64_t o = (R0 + r) * nbk + s * bpi + b;
+      sb[i] = r < valid ? __ldg(reinterpret_cast<const uint16_t*>(w.sex) + o) : (uint16_t)0;
+      sc[i] = r < valid ? __ldg(w.dv + o) : (uint16_t)0;
+    }
   }
   __syncwarp();
-  return 0;
 }
 
 // Timeout flag of the floor arm, which has no workspace; read with
 // cudaMemcpyFromSymbol when diagnosing.
 __device__ int32_t g_floor_status;
 
-template <int MODE, int F0, int F1, int NT>
-__global__ void __launch_bounds__(kDecodeWarps * 32, NT >= 8 ? 2 : (NT >= 4 ? 3 : 4)) k_stream(const __grid_constant__ CUtensorMap m0,
-                                                                 const __grid_constant__ CUtensorMap m1,
-                                                                 const __grid_constant__ UnitArgs A) {
+template <int MODE, int F0, int F1, int NT, bool BSM>
+__global__ void __launch_bounds__(kDecodeWarps * 32, kDecodeMinBlocks(NT)) k_stream(const __grid_constant__ CUtensorMap m0,
+                                                                         const __grid_constant__ CUtensorMap m1,
+                                                                         const __grid_constant__ UnitArgs A) {
   extern __shared__ __align__(128) uint8_t smem[];
   const int wid = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
-  const int K = A.w0.cols, nbk = K / 256;
-  const int CH = A.ch, ldw = CH * 16, nch = nbk / CH;
+  const int K = A.w0.cols;
+  const int bpi = A.bpi, S = A.splits;
+  const int ldw = 16 * bpi;
   const int stage_words = kTile * ldw;
-  const uint32_t slot_b = slot_bytes2<F0, F1>(nbk);
+  const uint32_t slot_b = slot_bytes2<F0, F1>(bpi);
   const uint32_t k65536 = opaque_u32(65536u);
   constexpr int NC = 8 * NT;
   const int npairs = A.T * A.topk;
   const size_t warp_bytes = (size_t)kStages * (stage_words * 4 + slot_b);
-  Ring ring;
-  ring.qs = reinterpret_cast<uint32_t*>(smem + wid * warp_bytes);
-  ring.slots = smem + wid * warp_bytes + (size_t)kStages * stage_words * 4;
+  uint32_t* ring_qs = reinterpret_cast<uint32_t*>(smem + wid * warp_bytes);
+  uint8_t* ring_slots = smem + wid * warp_bytes + (size_t)kStages * stage_words * 4;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kDecodeWarps * warp_bytes);
-  ring.bar = bars + wid * kStages;
+  uint64_t* bar = bars + wid * kStages;
   uint2* lut0 = reinterpret_cast<uint2*>(bars + kDecodeWarps * kStages);
   uint2* lut1 = lut0 + 64;
+  uint16_t* act_s = reinterpret_cast<uint16_t*>(lut1 + 64);  // BSM activation rows
+  // BSM rows keep each lane's 64-element segment in 80 elements (160 bytes),
+  // so the four segments a warp reads at once start in different bank groups
+  const int KP = BSM ? K / 64 * 80 : K;  // activation row stride (elements)
+  uint8_t* route_p = reinterpret_cast<uint8_t*>(act_s) + (BSM ? (size_t)A.act_rows * KP * 2 : 0);
   if (MODE != MODE_FLOOR) {
     build_lut<F0>(lut0, A.V);
     if (MODE == MODE_GATEUP) build_lut<F1>(lut1, A.V);
   }
   if (lane == 0) {
-    for (int s = 0; s < kStages; s++) mbar_init(&ring.bar[s], 1);
+    for (int s = 0; s < kStages; s++) mbar_init(&bar[s], 1);
     fence_mbar_init();
   }
   RouteView rt{};
   int D = 1;
   if (MODE == MODE_GATEUP || MODE == MODE_DOWN) {
-    rt = carve_route(reinterpret_cast<uint8_t*>(lut1 + 64), npairs);
+    rt = carve_route(route_p, npairs);
     build_route(A.ids, npairs, A.w0.experts, rt);  // ends with __syncthreads
     D = rt.scalars[0];
   } else {
@@ -408,73 +534,99 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, NT >= 8 ? 2 : (NT >= 4 ? 3 
   constexpr int NMAT = MODE == MODE_GATEUP ? 2 : 1;
   const int rows = A.w0.rows;
   const int tiles = (rows + kTile - 1) / kTile;
-  const int nunits = D * NMAT * tiles;
+  const int nitems = D * NMAT * tiles * S;
   const int W = gridDim.x * kDecodeWarps;
   const int gw = blockIdx.x * kDecodeWarps + wid;
-  // unit id -> (u, mat, tile): gate and up of one tile are adjacent
-  auto unit_of = [&](int id, int& u, int& mat, int& tile) {
-    mat = id % NMAT;
-    const int r = id / NMAT;
-    tile = r % tiles;
-    u = r / tiles;
+  // item id -> (u, tile, mat, s): the slices of a tile, then gate / up, are adjacent
+  auto item_of = [&](int id, int& u, int& mat, int& tile, int& s) {
+    int r = (int)A.div_s.div((uint32_t)id);
+    s = id - r * S;
+    mat = r % NMAT;
+    r /= NMAT;
+    u = (int)A.div_tiles.div((uint32_t)r);
+    tile = r - u * tiles;
   };
   auto expert_of = [&](int u) -> int {
     if (MODE == MODE_GEMV) return A.expert;
     if (MODE == MODE_FLOOR) return A.elist[u];
     return rt.uexp[u];
   };
-  // issue cursor: unit iteration `iu`, chunk `ic`; chunks are numbered
-  // q = iu * nch + ic. The unit's coordinates are decoded once per unit.
-  int iu = 0, ic = 0;
-  int cu_mat = 0;
-  int64_t cu_row0 = 0;
-  auto issue_next = [&]() {
-    const int id = gw + iu * W;
-    if (id >= nunits) return;
-    const int q = iu * nch + ic;
-    const int s = q % kStages;
-    uint32_t bytes = (uint32_t)stage_words * 4;
-    if (ic == 0) {
-      int u, mat, tile;
-      unit_of(id, u, mat, tile);
-      const int e = expert_of(u);
-      cu_mat = mat;
-      cu_row0 = (int64_t)e * rows + (int64_t)tile * kTile;
-      const int valid = min(kTile, rows - tile * kTile);
-      const WDev& w = mat ? A.w1 : A.w0;
-      // bulk-copyable tile: returns the bytes to expect; otherwise the lanes fill the slot now
-      uint8_t* slot = ring.slots + (size_t)(iu % kStages) * slot_b;
-      bytes += (mat == 0) ? stage_scales<F0>(slot, w, cu_row0, valid, &ring.bar[s], lane, false)
-                          : stage_scales<F1>(slot, w, cu_row0, valid, &ring.bar[s], lane, false);
-      if (lane == 0) {
-        mbar_arrive_expect_tx(&ring.bar[s], bytes);
-        if (mat == 0) stage_scales<F0>(slot, w, cu_row0, valid, &ring.bar[s], lane, true);
-        else stage_scales<F1>(slot, w, cu_row0, valid, &ring.bar[s], lane, true);
-      }
-    } else if (lane == 0) {
-      mbar_arrive_expect_tx(&ring.bar[s], bytes);
-    }
-    if (lane == 0)
-      tma_load_2d(ring.qs + (size_t)s * stage_words, cu_mat ? &m1 : &m0, ic * ldw, (int)cu_row0, &ring.bar[s]);
-    if (++ic == nch) {
-      ic = 0;
-      iu++;
+  auto issue = [&](int it) {
+    const int id = gw + it * W;
+    if (id >= nitems) return;
+    const int st = it % kStages;
+    int u, mat, tile, s;
+    item_of(id, u, mat, tile, s);
+    const int64_t R0 = (int64_t)expert_of(u) * rows + (int64_t)tile * kTile;
+    const int valid = min(kTile, rows - tile * kTile);
+    uint8_t* slot = ring_slots + (size_t)st * slot_b;
+    if (mat == 0) stage_scales<F0>(slot, A.w0, R0, valid, s, bpi, A.async_sc, &bar[st], lane);
+    else stage_scales<F1>(slot, A.w1, R0, valid, s, bpi, A.async_sc, &bar[st], lane);
+    __syncwarp();
+    if (lane == 0) {
+      mbar_arrive_expect_tx(&bar[st], (uint32_t)stage_words * 4);
+      tma_load_2d(ring_qs + (size_t)st * stage_words, mat ? &m1 : &m0, s * ldw, (int)R0, &bar[st]);
     }
   };
-  for (int s = 0; s < kStages; s++) issue_next();
+  for (int s = 0; s < kStages; s++) issue(s);
   if (MODE == MODE_GATEUP) griddep_launch();
-  griddep_wait();
+  // Results of the preceding kernel in the stream (the prep kernel's counters,
+  // transposed activations and status word; the gate/up kernel's h) are read
+  // only after griddepcontrol.wait. The raw activation rows are inputs of the
+  // call, complete before the prep kernel started, so a BSM launch copies them
+  // first and defers the wait to its first epilogue.
+  bool waited = false;
+  if constexpr (BSM) {  // the call's activation rows, slot-transposed and padded, once per CTA
+    if (MODE == MODE_DOWN) {  // h comes from the gate/up kernel, already slot-transposed
+      griddep_wait();
+      waited = true;
+    }
+    const int gpr = K / 16;  // 16-element groups per row
+    const int groups = A.act_rows * gpr;
+    for (int gi = threadIdx.x; gi < groups; gi += blockDim.x) {
+      const int r = gi / gpr, c0 = (gi - r * gpr) * 16;
+      uint32_t o[8];
+      if (MODE == MODE_DOWN) {
+        const uint4* src = reinterpret_cast<const uint4*>(A.act + (size_t)gi * 16);
+        const uint4 a = ld_nc_u4(src), b = ld_nc_u4(src + 1);
+        o[0] = a.x; o[1] = a.y; o[2] = a.z; o[3] = a.w; o[4] = b.x; o[5] = b.y; o[6] = b.z; o[7] = b.w;
+      } else {
+        const uint4* src = reinterpret_cast<const uint4*>(A.xraw + (size_t)gi * 16);
+        const uint4 a = ld_nc_u4(src), b = ld_nc_u4(src + 1);
+        const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+#pragma unroll
+        for (int i2 = 0; i2 < 4; i2++) {
+          const int wa = i2 >> 1;
+          const uint32_t sel = (i2 & 1) ? 0x7632u : 0x5410u;
+          o[2 * i2] = prmt(w[wa], w[wa + 2], sel);
+          o[2 * i2 + 1] = prmt(w[wa + 4], w[wa + 6], sel);
+        }
+      }
+      uint4* dst = reinterpret_cast<uint4*>(act_s + (size_t)r * KP + (c0 >> 6) * 80 + (c0 & 63));
+      dst[0] = make_uint4(o[0], o[1], o[2], o[3]);
+      dst[1] = make_uint4(o[4], o[5], o[6], o[7]);
+    }
+    __syncthreads();
+  } else {
+    griddep_wait();
+    waited = true;
+  }
   if (MODE == MODE_DOWN && D == 0) {  // every id out of range: the block output is zero
     for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < A.T * rows; i += gridDim.x * blockDim.x) A.out16[i] = 0;
     return;
   }
+  const uint16_t* act_base = BSM ? act_s : A.act;
+  constexpr int SEG = BSM ? 80 : 64;    // elements between the segments of lanes t and t + 1
+  constexpr int BLKE = BSM ? 320 : 256;  // elements between consecutive 256-weight blocks
 
   for (int it = 0;; it++) {
     const int id = gw + it * W;
-    if (id >= nunits) break;
-    int u, mat, tile;
-    unit_of(id, u, mat, tile);
+    if (id >= nitems) break;
+    int u, mat, tile, s;
+    item_of(id, u, mat, tile, s);
     const int e = expert_of(u);
+    const int64_t R0 = (int64_t)e * rows + (int64_t)tile * kTile;
+    const int valid = min(kTile, rows - tile * kTile);
     int p0 = 0, ncols = A.T;
     if (MODE == MODE_GATEUP || MODE == MODE_DOWN) {
       p0 = rt.ustart[u];
@@ -483,146 +635,142 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, NT >= 8 ? 2 : (NT >= 4 ? 3 
     const uint16_t* bsrc[NT];
 #pragma unroll
     for (int n = 0; n < NT; n++) {
-      const int col = 8 * n + g;
-      const uint16_t* b = nullptr;
-      if (MODE != MODE_FLOOR && col < ncols) {
-        if (MODE == MODE_GEMV) b = A.act + (size_t)col * K;
-        else if (MODE == MODE_GATEUP) b = A.act + (size_t)(rt.sorted[p0 + col] / A.topk) * K;
-        else b = A.act + (size_t)rt.sorted[p0 + col] * K;
-      }
-      bsrc[n] = b;
+      // columns past the last token or pair repeat column 0; their sums are never stored
+      const int col = 8 * n + g < ncols ? 8 * n + g : 0;
+      int arow = 0;
+      if (MODE == MODE_GEMV) arow = col;
+      else if (MODE == MODE_GATEUP) arow = rt.sorted[p0 + col] / A.topk;
+      else if (MODE == MODE_DOWN) arow = rt.sorted[p0 + col];
+      bsrc[n] = act_base + (size_t)arow * KP + (size_t)s * bpi * BLKE + SEG * t;
+      if (!BSM && MODE != MODE_FLOOR) prefetch_l1(bsrc[n]);
     }
-    const uint8_t* slot = ring.slots + (size_t)(it % kStages) * slot_b;
     const bool fmt0 = (MODE != MODE_GATEUP) || mat == 0;
-    float part[4][NT][4];
-#pragma unroll
-    for (int m = 0; m < 4; m++)
-#pragma unroll
-      for (int n = 0; n < NT; n++)
-#pragma unroll
-        for (int q = 0; q < 4; q++) part[m][n][q] = 0.f;
+    const bool kfmt = fmt0 ? (F0 == FMT_K) : (F1 == FMT_K);
+    // IQ2_KS row scales of rows g and g + 8, applied after the slice's MMAs
+    float dg = 0.f, dh = 0.f;
+    if (MODE != MODE_FLOOR && !kfmt) {
+      const uint16_t* dv = fmt0 ? A.w0.dv : A.w1.dv;
+      if (g < valid) dg = __half2float(__ushort_as_half(__ldg(dv + R0 + g)));
+      if (g + 8 < valid) dh = __half2float(__ushort_as_half(__ldg(dv + R0 + g + 8)));
+    }
+    const int st = it % kStages;
+    if (!mbar_wait_bounded(&bar[st], (uint32_t)((it / kStages) & 1))) {
+      if (!waited) griddep_wait();
+      if (lane == 0) atomicOr(A.status ? A.status : &g_floor_status, 2);
+      // let this warp's copies still in flight land before the CTA exits
+      for (int k = 1; k < kStages; k++)
+        (void)mbar_wait_bounded(&bar[(it + k) % kStages], (uint32_t)(((it + k) / kStages) & 1));
+      return;
+    }
+    const uint32_t* sq = ring_qs + (size_t)st * stage_words;
+    const uint8_t* slot = ring_slots + (size_t)st * slot_b;
     float acc[NT][4];
 #pragma unroll
     for (int n = 0; n < NT; n++)
 #pragma unroll
       for (int q = 0; q < 4; q++) acc[n][q] = 0.f;
     uint32_t xg = 0, xh = 0;  // FLOOR checksums of rows g and g + 8
-    for (int j = 0; j < nch; j++) {
-      const int q = it * nch + j;
-      const int s = q % kStages;
-      if (!mbar_wait_bounded(&ring.bar[s], (uint32_t)((q / kStages) & 1))) {
-        if (lane == 0) atomicOr(A.status ? A.status : &g_floor_status, 2);
-        for (int k = 1; k < kStages; k++) (void)mbar_wait_bounded(&ring.bar[(q + k) % kStages], (uint32_t)(((q + k) / kStages) & 1));
-        return;
-      }
-      const uint32_t* sq = ring.qs + (size_t)s * stage_words;
-      if (MODE == MODE_FLOOR) {
-        for (int b = 0; b < CH; b++) {
-          const uint4 a4 = *reinterpret_cast<const uint4*>(sq + g * ldw + b * 16 + 4 * t);
-          const uint4 b4 = *reinterpret_cast<const uint4*>(sq + (g + 8) * ldw + b * 16 + 4 * t);
-          xg ^= a4.x ^ a4.y ^ a4.z ^ a4.w;
-          xh ^= b4.x ^ b4.y ^ b4.z ^ b4.w;
-        }
-      } else {
-        for (int b = 0; b < CH; b++) {
-          const int kb = j * CH + b;
-          const uint16_t* src[NT];
-#pragma unroll
-          for (int n = 0; n < NT; n++) src[n] = bsrc[n] ? bsrc[n] + 256 * kb + 64 * t : nullptr;
-          uint32_t cg[4], ch[4];
-          if (fmt0) {
-            combos_smem<F0>(slot, nbk, g, kb, t, cg);
-            combos_smem<F0>(slot, nbk, g + 8, kb, t, ch);
-          } else {
-            combos_smem<F1>(slot, nbk, g, kb, t, cg);
-            combos_smem<F1>(slot, nbk, g + 8, kb, t, ch);
-          }
-          const bool kfmt = fmt0 ? (F0 == FMT_K) : (F1 == FMT_K);
-          if (kfmt) {
-#pragma unroll
-            for (int m = 0; m < 4; m++)
-#pragma unroll
-              for (int n = 0; n < NT; n++)
-#pragma unroll
-                for (int qq = 0; qq < 4; qq++) part[m][n][qq] = 0.f;
-          }
-          block_mma<F0, NT>(sq, ldw, b * 16, src, cg, ch, fmt0 ? lut0 : lut1, part, g, t, k65536);
-          if (kfmt) {  // IQ2_K: d changes every block
-            const float dg = fmt0 ? d_smem<F0>(slot, nbk, g, kb) : d_smem<F1>(slot, nbk, g, kb);
-            const float dh = fmt0 ? d_smem<F0>(slot, nbk, g + 8, kb) : d_smem<F1>(slot, nbk, g + 8, kb);
-#pragma unroll
-            for (int n = 0; n < NT; n++) {
-              acc[n][0] = fmaf(dg, (part[0][n][0] + part[1][n][0]) + (part[2][n][0] + part[3][n][0]), acc[n][0]);
-              acc[n][1] = fmaf(dg, (part[0][n][1] + part[1][n][1]) + (part[2][n][1] + part[3][n][1]), acc[n][1]);
-              acc[n][2] = fmaf(dh, (part[0][n][2] + part[1][n][2]) + (part[2][n][2] + part[3][n][2]), acc[n][2]);
-              acc[n][3] = fmaf(dh, (part[0][n][3] + part[1][n][3]) + (part[2][n][3] + part[3][n][3]), acc[n][3]);
-            }
-          }
-        }
-      }
-      __syncwarp();
-      issue_next();
-    }
-    const int rg = tile * kTile + g, rh = rg + 8;
     if (MODE == MODE_FLOOR) {
-      // fold the slot's scale bytes for rows g and g + 8 (byte i of a row's
-      // stream lands in byte i & 3 of the word)
+      for (int b = 0; b < bpi; b++) {
+        const uint4 a4 = *reinterpret_cast<const uint4*>(sq + g * ldw + b * 16 + 4 * t);
+        const uint4 b4 = *reinterpret_cast<const uint4*>(sq + (g + 8) * ldw + b * 16 + 4 * t);
+        xg ^= a4.x ^ a4.y ^ a4.z ^ a4.w;
+        xh ^= b4.x ^ b4.y ^ b4.z ^ b4.w;
+      }
+      // the slice's scale bytes; byte j of a row's plane lands in byte j & 3
       const bool ks = F0 == FMT_KS;
       const uint32_t* s32 = reinterpret_cast<const uint32_t*>(slot);
-      const int nw = ks ? nbk : 2 * nbk;
+      const int nw = ks ? bpi : 2 * bpi;  // scl words per row (slices start on word boundaries)
       for (int i = t; i < nw; i += 4) {
         xg ^= s32[g * nw + i];
         xh ^= s32[(g + 8) * nw + i];
       }
-      const uint8_t* sb = slot + Slot<F0>::b_off(nbk);
-      const uint8_t* sc = slot + Slot<F0>::c_off(nbk);
-      const int nbb = ks ? nbk : 2 * nbk;  // bytes per row of the second / third plane
-      for (int i = t; i < nbb; i += 4) {
-        xg ^= (uint32_t)sb[g * nbb + i] << (8 * (i & 3));
-        xh ^= (uint32_t)sb[(g + 8) * nbb + i] << (8 * (i & 3));
-        xg ^= (uint32_t)sc[g * nbb + i] << (8 * (i & 3));
-        xh ^= (uint32_t)sc[(g + 8) * nbb + i] << (8 * (i & 3));
+      if (ks) {
+        const uint8_t* sb = slot + Slot<FMT_KS>::b_off(bpi);
+        const uint8_t* sc = slot + Slot<FMT_KS>::c_off(bpi);
+        for (int i = t; i < bpi; i += 4) {
+          const int sh = 8 * ((s * bpi + i) & 3);
+          xg ^= ((uint32_t)sb[g * bpi + i] ^ (uint32_t)sc[g * bpi + i]) << sh;
+          xh ^= ((uint32_t)sb[(g + 8) * bpi + i] ^ (uint32_t)sc[(g + 8) * bpi + i]) << sh;
+        }
+        if (s == 0 && t == 0) {  // the row scale belongs to the first slice
+          if (g < valid) xg ^= __ldg(A.w0.dv + R0 + g);
+          if (g + 8 < valid) xh ^= __ldg(A.w0.dv + R0 + g + 8);
+        }
+      } else {
+        const uint16_t* sb = reinterpret_cast<const uint16_t*>(slot + Slot<FMT_K>::b_off(bpi));
+        const uint16_t* sc = reinterpret_cast<const uint16_t*>(slot + Slot<FMT_K>::c_off(bpi));
+        for (int i = t; i < bpi; i += 4) {
+          const int sh = 16 * ((s * bpi + i) & 1);
+          xg ^= ((uint32_t)sb[g * bpi + i] ^ (uint32_t)sc[g * bpi + i]) << sh;
+          xh ^= ((uint32_t)sb[(g + 8) * bpi + i] ^ (uint32_t)sc[(g + 8) * bpi + i]) << sh;
+        }
       }
-      if (ks && t == 0) {
-        const uint16_t* sd = reinterpret_cast<const uint16_t*>(sc + 16u * nbk);
-        xg ^= sd[g];
-        xh ^= sd[g + 8];
-      }
+    } else {
+      item_mma<F0, F1, NT, BSM>(sq, slot, bpi, ldw, bsrc, fmt0, kfmt, lut0, lut1, dg, dh, g, t, k65536, acc);
+    }
+    __syncwarp();
+    issue(it + kStages);  // refill the stage just consumed
+    if (!waited) {
+      griddep_wait();
+      waited = true;
+    }
+
+    const int rg = tile * kTile + g, rh = rg + 8;
+    if (MODE == MODE_FLOOR) {
       xg ^= __shfl_xor_sync(0xffffffffu, xg, 1);
       xg ^= __shfl_xor_sync(0xffffffffu, xg, 2);
       xh ^= __shfl_xor_sync(0xffffffffu, xh, 1);
       xh ^= __shfl_xor_sync(0xffffffffu, xh, 2);
       if (t == 0) {
-        if (rg < rows) A.outx[(size_t)u * rows + rg] = xg;
-        if (rh < rows) A.outx[(size_t)u * rows + rh] = xh;
+        if (rg < rows) atomicXor(A.outx + (size_t)u * rows + rg, xg);
+        if (rh < rows) atomicXor(A.outx + (size_t)u * rows + rh, xh);
       }
       continue;
     }
-    const bool kfmt = fmt0 ? (F0 == FMT_K) : (F1 == FMT_K);
-    if (!kfmt) {
-      const float dg = fmt0 ? d_smem<F0>(slot, nbk, g, 0) : d_smem<F1>(slot, nbk, g, 0);
-      const float dh = fmt0 ? d_smem<F0>(slot, nbk, g + 8, 0) : d_smem<F1>(slot, nbk, g + 8, 0);
-#pragma unroll
-      for (int n = 0; n < NT; n++) {
-        acc[n][0] = dg * ((part[0][n][0] + part[1][n][0]) + (part[2][n][0] + part[3][n][0]));
-        acc[n][1] = dg * ((part[0][n][1] + part[1][n][1]) + (part[2][n][1] + part[3][n][1]));
-        acc[n][2] = dh * ((part[0][n][2] + part[1][n][2]) + (part[2][n][2] + part[3][n][2]));
-        acc[n][3] = dh * ((part[0][n][3] + part[1][n][3]) + (part[2][n][3] + part[3][n][3]));
-      }
-    }
 
     if (MODE == MODE_GEMV) {
+      if (S == 1) {
+#pragma unroll
+        for (int n = 0; n < NT; n++)
+#pragma unroll
+          for (int q = 0; q < 4; q++) {
+            const int col = 8 * n + 2 * t + (q & 1);
+            const int row = tile * kTile + g + 8 * (q >> 1);
+            if (col < A.T && row < rows) A.yf[(size_t)col * rows + row] = acc[n][q];
+          }
+        continue;
+      }
+      float* slotp = A.part + ((size_t)tile * S + s) * NC * kTile;
+#pragma unroll
+      for (int n = 0; n < NT; n++)
+#pragma unroll
+        for (int q = 0; q < 4; q++) slotp[(8 * n + 2 * t + (q & 1)) * kTile + g + 8 * (q >> 1)] = acc[n][q];
+      __syncwarp();
+      int prev = 0;
+      if (lane == 0) {
+        __threadfence();
+        prev = atomicAdd(A.cnt + tile, 1);
+      }
+      prev = __shfl_sync(0xffffffffu, prev, 0);
+      if (prev != S - 1) continue;
+      __threadfence();
+      const float* base = A.part + (size_t)tile * S * NC * kTile;
 #pragma unroll
       for (int n = 0; n < NT; n++)
 #pragma unroll
         for (int q = 0; q < 4; q++) {
           const int col = 8 * n + 2 * t + (q & 1);
-          const int row = tile * kTile + g + 8 * (q >> 1);
-          if (col < A.T && row < rows) A.yf[(size_t)col * rows + row] = acc[n][q];
+          const int r = g + 8 * (q >> 1);
+          const int row = tile * kTile + r;
+          if (col >= A.T || row >= rows) continue;
+          float sum = 0.f;
+          for (int ss = 0; ss < S; ss++) sum += __ldcg(base + ((size_t)ss * NC + col) * kTile + r);
+          A.yf[(size_t)col * rows + row] = sum;
         }
     } else if (MODE == MODE_GATEUP) {
       const size_t ut = (size_t)u * tiles + tile;
-      float* slotp = A.part + (ut * 2 + mat) * NC * kTile;
+      float* slotp = A.part + ((ut * 2 + mat) * S + s) * NC * kTile;
 #pragma unroll
       for (int n = 0; n < NT; n++)
 #pragma unroll
@@ -634,9 +782,10 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, NT >= 8 ? 2 : (NT >= 4 ? 3 
         prev = atomicAdd(A.cnt + ut, 1);
       }
       prev = __shfl_sync(0xffffffffu, prev, 0);
-      if (prev != 1) continue;
+      if (prev != 2 * S - 1) continue;
       __threadfence();
-      const float* other = A.part + (ut * 2 + (mat ^ 1)) * NC * kTile;
+      const float* gb = A.part + (ut * 2) * S * NC * kTile;
+      const float* ub = gb + (size_t)S * NC * kTile;
 #pragma unroll
       for (int n = 0; n < NT; n++)
 #pragma unroll
@@ -645,14 +794,16 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, NT >= 8 ? 2 : (NT >= 4 ? 3 
           const int r = g + 8 * (q >> 1);
           const int f = tile * kTile + r;
           if (col >= ncols || f >= rows) continue;
-          const float o = __ldcg(other + col * kTile + r);
-          const float gv = mat == 0 ? acc[n][q] : o;
-          const float uv = mat == 0 ? o : acc[n][q];
+          float gv = 0.f, uv = 0.f;
+          for (int ss = 0; ss < S; ss++) {
+            gv += __ldcg(gb + ((size_t)ss * NC + col) * kTile + r);
+            uv += __ldcg(ub + ((size_t)ss * NC + col) * kTile + r);
+          }
           const float h = gv / (1.0f + __expf(-gv)) * uv;
           A.out16[(size_t)rt.sorted[p0 + col] * rows + perm16(f)] = f32_to_bf16_bits(h);
         }
     } else {
-      float* slab = A.part + (size_t)tile * npairs * kTile;
+      float* slab = A.part + (size_t)tile * npairs * S * kTile;
 #pragma unroll
       for (int n = 0; n < NT; n++)
 #pragma unroll
@@ -660,7 +811,7 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, NT >= 8 ? 2 : (NT >= 4 ? 3 
           const int col = 8 * n + 2 * t + (q & 1);
           if (col >= ncols) continue;
           const int pair = rt.sorted[p0 + col];
-          slab[(size_t)pair * kTile + g + 8 * (q >> 1)] = __ldg(A.p + pair) * acc[n][q];
+          slab[((size_t)pair * S + s) * kTile + g + 8 * (q >> 1)] = acc[n][q];
         }
       __syncwarp();
       int prev = 0;
@@ -669,7 +820,7 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, NT >= 8 ? 2 : (NT >= 4 ? 3 
         prev = atomicAdd(A.cnt + tile, 1);
       }
       prev = __shfl_sync(0xffffffffu, prev, 0);
-      if (prev != D - 1) continue;
+      if (prev != D * S - 1) continue;
       __threadfence();
       for (int o = lane; o < A.T * kTile; o += 32) {
         const int tok = o / kTile, r = o % kTile;
@@ -679,12 +830,262 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, NT >= 8 ? 2 : (NT >= 4 ? 3 
         for (int jj = 0; jj < A.topk; jj++) {
           const int pair = tok * A.topk + jj;
           if (rt.ids[pair] < 0) continue;
-          sum += __ldcg(slab + (size_t)pair * kTile + r);
+          float v = 0.f;
+          for (int ss = 0; ss < S; ss++) v += __ldcg(slab + ((size_t)pair * S + ss) * kTile + r);
+          sum += __ldg(A.p + pair) * v;
         }
         A.out16[(size_t)tok * rows + row] = f32_to_bf16_bits(sum);
       }
     }
   }
+  if (!waited) griddep_wait();  // this grid completes only after the one it depends on
+}
+
+// ------------------------------------------------------------- tile kernel
+// Gate/up and down with the slices of an output tile reduced inside one CTA
+// (one or two MMA column groups). A CTA takes tile groups in turn, group
+// blockIdx.x + r * gridDim.x in round r:
+//   GATEUP: group = (distinct expert u, 16-row tile of the intermediate
+//           dimension); its items are the gate and up slices, 2 * S of them;
+//   DOWN:   group = 16-row tile of the hidden dimension; its items are the
+//           (distinct expert, slice) pairs, D * S of them.
+// Warp w takes items w, w + kDecodeWarps, ... of each group and adds them into
+// its own shared-memory slot; after a CTA barrier the threads sum the slots in
+// warp order (the same order every call) and write h = bf16(silu(g) * u) or
+// y = bf16(sum over slots of p * down). No device-scope counters are needed.
+template <int MODE, int F0, int F1, int NT, bool BSM>
+__global__ void __launch_bounds__(kDecodeWarps * 32, kDecodeMinBlocks(NT)) k_tiles(const __grid_constant__ CUtensorMap m0,
+                                                                             const __grid_constant__ CUtensorMap m1,
+                                                                             const __grid_constant__ UnitArgs A) {
+  static_assert(MODE == MODE_GATEUP || MODE == MODE_DOWN, "tile kernel: gate/up or down");
+  extern __shared__ __align__(128) uint8_t smem[];
+  const int wid = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+  const int K = A.w0.cols;
+  const int bpi = A.bpi, S = A.splits;
+  const int ldw = 16 * bpi;
+  const int stage_words = kTile * ldw;
+  const uint32_t slot_b = slot_bytes2<F0, F1>(bpi);
+  const uint32_t k65536 = opaque_u32(65536u);
+  constexpr int NC = 8 * NT;
+  const int npairs = A.T * A.topk;
+  const size_t warp_bytes = (size_t)kStages * (stage_words * 4 + slot_b);
+  uint32_t* ring_qs = reinterpret_cast<uint32_t*>(smem + wid * warp_bytes);
+  uint8_t* ring_slots = smem + wid * warp_bytes + (size_t)kStages * stage_words * 4;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kDecodeWarps * warp_bytes);
+  uint64_t* bar = bars + wid * kStages;
+  uint2* lut0 = reinterpret_cast<uint2*>(bars + kDecodeWarps * kStages);
+  uint2* lut1 = lut0 + 64;
+  const int KP = BSM ? K / 64 * 80 : K;  // activation row stride (elements), see k_stream
+  uint16_t* act_s = reinterpret_cast<uint16_t*>(lut1 + 64);
+  float* red = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(act_s) + (BSM ? (size_t)A.act_rows * KP * 2 : 0));
+  const int slot_f = MODE == MODE_GATEUP ? 2 * NC * kTile : A.T * kTile;  // floats per warp slot
+  uint8_t* route_p = reinterpret_cast<uint8_t*>(red + (size_t)kDecodeWarps * slot_f);
+  build_lut<F0>(lut0, A.V);
+  if (MODE == MODE_GATEUP) build_lut<F1>(lut1, A.V);
+  if (lane == 0) {
+    for (int s = 0; s < kStages; s++) mbar_init(&bar[s], 1);
+    fence_mbar_init();
+  }
+  const RouteView rt = carve_route(route_p, npairs);
+  build_route(A.ids, npairs, A.w0.experts, rt);  // ends with __syncthreads
+  const int D = rt.scalars[0];
+  const int rows = A.w0.rows;
+  const int tiles = (rows + kTile - 1) / kTile;
+  const int n_it = MODE == MODE_GATEUP ? 2 * S : D * S;          // items per group
+  const int ngroups = MODE == MODE_GATEUP ? D * tiles : tiles;
+  const int rounds = (int)blockIdx.x < ngroups ? (ngroups - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
+  const int cnt_w = wid < n_it ? (n_it - 1 - wid) / kDecodeWarps + 1 : 0;  // this warp's items per group
+  const int nq = rounds * cnt_w;
+  // q-th item of this warp -> (u, mat, tile, s)
+  auto item_at = [&](int q, int& u, int& mat, int& tile, int& s) {
+    const int r = q / cnt_w;
+    const int j = wid + (q - r * cnt_w) * kDecodeWarps;
+    const int tg = (int)blockIdx.x + r * (int)gridDim.x;
+    const int js = (int)A.div_s.div((uint32_t)j);
+    s = j - js * S;
+    if (MODE == MODE_GATEUP) {
+      mat = js;
+      u = (int)A.div_tiles.div((uint32_t)tg);
+      tile = tg - u * tiles;
+    } else {
+      mat = 0;
+      u = js;
+      tile = tg;
+    }
+  };
+  int issued = 0;
+  auto issue = [&](int q) {
+    if (q >= nq) return;
+    const int st = q % kStages;
+    int u, mat, tile, s;
+    item_at(q, u, mat, tile, s);
+    const int64_t R0 = (int64_t)rt.uexp[u] * rows + (int64_t)tile * kTile;
+    const int valid = min(kTile, rows - tile * kTile);
+    uint8_t* slot = ring_slots + (size_t)st * slot_b;
+    if (mat == 0) stage_scales<F0>(slot, A.w0, R0, valid, s, bpi, A.async_sc, &bar[st], lane);
+    else stage_scales<F1>(slot, A.w1, R0, valid, s, bpi, A.async_sc, &bar[st], lane);
+    __syncwarp();
+    if (lane == 0) {
+      mbar_arrive_expect_tx(&bar[st], (uint32_t)stage_words * 4);
+      tma_load_2d(ring_qs + (size_t)st * stage_words, mat ? &m1 : &m0, s * ldw, (int)R0, &bar[st]);
+    }
+    issued = q + 1;
+  };
+  for (int q = 0; q < kStages; q++) issue(q);
+  if (MODE == MODE_GATEUP) griddep_launch();
+  // The raw activation rows are inputs of the call and can be read before the
+  // dependency wait; h (DOWN) is the preceding kernel's result.
+  bool waited = false;
+  if (MODE == MODE_DOWN || !BSM) {
+    griddep_wait();
+    waited = true;
+  }
+  if constexpr (BSM) {  // activation rows, slot-transposed and padded, once per CTA
+    const int gpr = K / 16;
+    const int groups = A.act_rows * gpr;
+    for (int gi = threadIdx.x; gi < groups; gi += blockDim.x) {
+      const int r = gi / gpr, c0 = (gi - r * gpr) * 16;
+      uint32_t o[8];
+      if (MODE == MODE_DOWN) {
+        const uint4* src = reinterpret_cast<const uint4*>(A.act + (size_t)gi * 16);
+        const uint4 a = ld_nc_u4(src), b = ld_nc_u4(src + 1);
+        o[0] = a.x; o[1] = a.y; o[2] = a.z; o[3] = a.w; o[4] = b.x; o[5] = b.y; o[6] = b.z; o[7] = b.w;
+      } else {
+        const uint4* src = reinterpret_cast<const uint4*>(A.xraw + (size_t)gi * 16);
+        const uint4 a = ld_nc_u4(src), b = ld_nc_u4(src + 1);
+        const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+#pragma unroll
+        for (int i2 = 0; i2 < 4; i2++) {
+          const int wa = i2 >> 1;
+          const uint32_t sel = (i2 & 1) ? 0x7632u : 0x5410u;
+          o[2 * i2] = prmt(w[wa], w[wa + 2], sel);
+          o[2 * i2 + 1] = prmt(w[wa + 4], w[wa + 6], sel);
+        }
+      }
+      uint4* dst = reinterpret_cast<uint4*>(act_s + (size_t)r * KP + (c0 >> 6) * 80 + (c0 & 63));
+      dst[0] = make_uint4(o[0], o[1], o[2], o[3]);
+      dst[1] = make_uint4(o[4], o[5], o[6], o[7]);
+    }
+    __syncthreads();
+  }
+  if (MODE == MODE_DOWN && D == 0) {  // every id out of range: the block output is zero
+    for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < A.T * rows; i += gridDim.x * blockDim.x) A.out16[i] = 0;
+    return;
+  }
+  const uint16_t* act_base = BSM ? act_s : A.act;
+  constexpr int SEG = BSM ? 80 : 64;
+  constexpr int BLKE = BSM ? 320 : 256;
+  float* my = red + (size_t)wid * slot_f;
+  bool failed = false;
+  int consumed = 0;
+  int q = 0;
+  for (int r = 0; r < rounds; r++) {
+    for (int i = lane; i < slot_f; i += 32) my[i] = 0.f;
+    __syncwarp();
+    for (int k = 0; k < cnt_w; k++, q++) {
+      int u, mat, tile, s;
+      item_at(q, u, mat, tile, s);
+      const int64_t R0 = (int64_t)rt.uexp[u] * rows + (int64_t)tile * kTile;
+      const int valid = min(kTile, rows - tile * kTile);
+      const int p0 = rt.ustart[u];
+      const int ncols = rt.ustart[u + 1] - p0;
+      const uint16_t* bsrc[NT];
+#pragma unroll
+      for (int n = 0; n < NT; n++) {
+        // columns past the last pair repeat column 0; their sums are never used
+        const int col = 8 * n + g < ncols ? 8 * n + g : 0;
+        const int pair = rt.sorted[p0 + col];
+        const int arow = MODE == MODE_GATEUP ? pair / A.topk : pair;
+        bsrc[n] = act_base + (size_t)arow * KP + (size_t)s * bpi * BLKE + SEG * t;
+        if (!BSM) prefetch_l1(bsrc[n]);
+      }
+      const bool fmt0 = (MODE != MODE_GATEUP) || mat == 0;
+      const bool kfmt = fmt0 ? (F0 == FMT_K) : (F1 == FMT_K);
+      float dg = 0.f, dh = 0.f;
+      if (!kfmt) {
+        const uint16_t* dv = fmt0 ? A.w0.dv : A.w1.dv;
+        if (g < valid) dg = __half2float(__ushort_as_half(__ldg(dv + R0 + g)));
+        if (g + 8 < valid) dh = __half2float(__ushort_as_half(__ldg(dv + R0 + g + 8)));
+      }
+      float acc[NT][4];
+#pragma unroll
+      for (int n = 0; n < NT; n++)
+#pragma unroll
+        for (int qq = 0; qq < 4; qq++) acc[n][qq] = 0.f;
+      const int st = q % kStages;
+      if (!failed && !mbar_wait_bounded(&bar[st], (uint32_t)((q / kStages) & 1))) {
+        failed = true;  // keep taking part in the CTA barriers; stop loading
+        if (!waited) {
+          griddep_wait();
+          waited = true;
+        }
+        if (lane == 0) atomicOr(A.status, 2);
+      }
+      if (!failed) {
+        consumed = q + 1;
+        const uint32_t* sq = ring_qs + (size_t)st * stage_words;
+        const uint8_t* slot = ring_slots + (size_t)st * slot_b;
+        item_mma<F0, F1, NT, BSM>(sq, slot, bpi, ldw, bsrc, fmt0, kfmt, lut0, lut1, dg, dh, g, t, k65536, acc);
+        __syncwarp();
+        issue(q + kStages);  // refill the stage just consumed
+      }
+      // add into this warp's slot: (mat, column, row) for gate/up, (token, row) for down
+      if (MODE == MODE_GATEUP) {
+#pragma unroll
+        for (int n = 0; n < NT; n++)
+#pragma unroll
+          for (int qq = 0; qq < 4; qq++)
+            my[(mat * NC + 8 * n + 2 * t + (qq & 1)) * kTile + g + 8 * (qq >> 1)] += acc[n][qq];
+      } else {
+        // one column (pair) at a time: a token may list one expert twice
+        for (int c = 0; c < ncols; c++) {
+#pragma unroll
+          for (int n = 0; n < NT; n++)
+#pragma unroll
+            for (int qq = 0; qq < 4; qq++) {
+              if (8 * n + 2 * t + (qq & 1) != c) continue;
+              const int pair = rt.sorted[p0 + c];
+              my[(pair / A.topk) * kTile + g + 8 * (qq >> 1)] += __ldg(A.p + pair) * acc[n][qq];
+            }
+          __syncwarp();
+        }
+      }
+      __syncwarp();
+    }
+    __syncthreads();  // every warp's slot of this group is complete
+    const int tg = (int)blockIdx.x + r * (int)gridDim.x;
+    if (MODE == MODE_GATEUP) {
+      const int u = (int)A.div_tiles.div((uint32_t)tg);
+      const int tile = tg - u * tiles;
+      const int p0 = rt.ustart[u];
+      const int ncols = rt.ustart[u + 1] - p0;
+      for (int o = threadIdx.x; o < ncols * kTile; o += blockDim.x) {
+        const int col = o / kTile, row = o - col * kTile;
+        const int f = tile * kTile + row;
+        if (f >= rows) continue;
+        float gv = 0.f, uv = 0.f;
+        for (int w = 0; w < kDecodeWarps; w++) {
+          gv += red[(size_t)w * slot_f + col * kTile + row];
+          uv += red[(size_t)w * slot_f + (NC + col) * kTile + row];
+        }
+        const float h = gv / (1.0f + __expf(-gv)) * uv;
+        A.out16[(size_t)rt.sorted[p0 + col] * rows + perm16(f)] = f32_to_bf16_bits(h);
+      }
+    } else {
+      for (int o = threadIdx.x; o < A.T * kTile; o += blockDim.x) {
+        const int tok = o / kTile, row = o - tok * kTile;
+        const int f = tg * kTile + row;
+        if (f >= rows) continue;
+        float y = 0.f;
+        for (int w = 0; w < kDecodeWarps; w++) y += red[(size_t)w * slot_f + tok * kTile + row];
+        A.out16[(size_t)tok * rows + f] = f32_to_bf16_bits(y);
+      }
+    }
+    __syncthreads();  // slots free for the next group
+  }
+  // let copies still in flight land before the CTA exits (only after a timeout)
+  for (int qd = consumed; qd < issued; qd++) (void)mbar_wait_bounded(&bar[qd % kStages], (uint32_t)((qd / kStages) & 1));
+  if (!waited) griddep_wait();  // this grid completes only after the one it depends on
 }
 
 // ================================================================== host
@@ -714,16 +1115,24 @@ int make_qs_map(CUtensorMap* map, const WDev& w, int nb) {
   return r == CUDA_SUCCESS ? 0 : -4;
 }
 
-static int chunk_blocks(int cols) {
-  const int nbk = cols / 256;
-  return nbk % 2 == 0 ? 2 : 1;
-}
+// Activation rows staged in shared memory (padded by 5/4) when they fit this budget.
+constexpr size_t kActSmemMax = 40 * 1024;
 
 template <int F0, int F1>
-static size_t stream_smem(int cols, int npairs, bool route) {
-  const int nbk = cols / 256, ch = chunk_blocks(cols);
-  const size_t warp = (size_t)kStages * ((size_t)kTile * ch * 16 * 4 + slot_bytes2<F0, F1>(nbk));
-  return kDecodeWarps * warp + (size_t)kDecodeWarps * kStages * 8 + 2 * 64 * 8 + (route ? route_smem_bytes(npairs) : 0);
+static size_t stream_smem(int cols, int npairs, bool route, int act_rows) {
+  const int bpi = item_blocks(cols);
+  const size_t warp = (size_t)kStages * ((size_t)kTile * bpi * 16 * 4 + slot_bytes2<F0, F1>(bpi));
+  return kDecodeWarps * warp + (size_t)kDecodeWarps * kStages * 8 + 2 * 64 * 8 +
+         (size_t)act_rows * (cols / 64 * 80) * 2 + (route ? route_smem_bytes(npairs) : 0);
+}
+
+template <int MODE, int F0, int F1, int NT>
+static size_t tiles_smem(int cols, int T, int npairs, int act_rows) {
+  const int bpi = item_blocks(cols);
+  const size_t warp = (size_t)kStages * ((size_t)kTile * bpi * 16 * 4 + slot_bytes2<F0, F1>(bpi));
+  const size_t red = (size_t)kDecodeWarps * (MODE == MODE_GATEUP ? 2 * 8 * NT * kTile : T * kTile) * 4;
+  return kDecodeWarps * warp + (size_t)kDecodeWarps * kStages * 8 + 2 * 64 * 8 + (size_t)act_rows * (cols / 64 * 80) * 2 +
+         red + route_smem_bytes(npairs);
 }
 
 static int nt_for(int cols_needed) { return cols_needed <= 8 ? 1 : cols_needed <= 16 ? 2 : cols_needed <= 32 ? 4 : 8; }
@@ -748,7 +1157,7 @@ static KernelCache* kcache(const void* fn) {
 }
 
 template <typename K>
-static int occupancy_grid(K kernel, size_t smem, int units_max, int num_sms) {
+static int occupancy_grid(K kernel, size_t smem, int items, int num_sms) {
   KernelCache* kc = kcache(reinterpret_cast<const void*>(kernel));
   int per_sm = 0;
   if (kc && kc->occ_smem == smem) {
@@ -762,8 +1171,7 @@ static int occupancy_grid(K kernel, size_t smem, int units_max, int num_sms) {
     }
   }
   if (per_sm < 1) return -1;
-  per_sm = std::min(per_sm, 4);
-  int want = (units_max + kDecodeWarps - 1) / kDecodeWarps;
+  const int want = (items + kDecodeWarps - 1) / kDecodeWarps;
   return std::max(1, std::min(want, per_sm * num_sms));
 }
 
@@ -785,24 +1193,34 @@ static cudaLaunchAttribute pdl_attr() {
 
 GemvWs gemv_ws(int T, int rows, int cols) {
   GemvWs ws;
+  const int tiles = (rows + kTile - 1) / kTile;
+  const int S = (cols / 256) / item_blocks(cols);
+  const int nc = 8 * nt_for(T);
   size_t o = 0;
   ws.status = o;
   o = align256(o + 16);
   ws.xperm = o;
   o = align256(o + (size_t)T * cols * 2);
   ws.cnt = o;
+  o = align256(o + (size_t)tiles * 4);
   ws.part = o;
+  o = align256(o + (S > 1 ? (size_t)tiles * S * nc * kTile * 4 : 0));
   ws.total = o;
   return ws;
 }
 
-template <int MODE, int F0, int F1, int NT>
-static int launch_stream(const CUtensorMap& m0, const CUtensorMap& m1, const UnitArgs& a, int units_max,
-                         cudaStream_t st, int num_sms, bool pdl) {
-  auto kern = k_stream<MODE, F0, F1, NT>;
-  const size_t smem = stream_smem<F0, F1>(a.w0.cols, a.T * a.topk, MODE == MODE_GATEUP || MODE == MODE_DOWN);
+template <int MODE, int F0, int F1, int NT, bool BSM>
+static int launch_stream(const CUtensorMap& m0, const CUtensorMap& m1, const UnitArgs& a, int items, cudaStream_t st,
+                         int num_sms, bool pdl) {
+  auto kern = k_stream<MODE, F0, F1, NT, BSM>;
+  // the item-index dividers follow this launch's own geometry
+  UnitArgs args = a;
+  args.div_s = FastDiv::of((uint32_t)a.splits);
+  args.div_tiles = FastDiv::of((uint32_t)((a.w0.rows + kTile - 1) / kTile));
+  const size_t smem = stream_smem<F0, F1>(a.w0.cols, a.T * a.topk, MODE == MODE_GATEUP || MODE == MODE_DOWN,
+                                          BSM ? a.act_rows : 0);
   if (set_smem(kern, smem)) return -4;
-  const int grid = occupancy_grid(kern, smem, units_max, num_sms);
+  const int grid = occupancy_grid(kern, smem, items, num_sms);
   if (grid < 0) return -4;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
@@ -812,33 +1230,97 @@ static int launch_stream(const CUtensorMap& m0, const CUtensorMap& m1, const Uni
   cudaLaunchAttribute at[1] = {pdl_attr()};
   cfg.attrs = at;
   cfg.numAttrs = pdl ? 1 : 0;
-  return cudaLaunchKernelEx(&cfg, kern, m0, m1, a) == cudaSuccess ? 0 : -4;
+  return cudaLaunchKernelEx(&cfg, kern, m0, m1, args) == cudaSuccess ? 0 : -4;
+}
+
+template <int MODE, int F0, int F1, int NT, bool BSM>
+static int launch_tiles(const CUtensorMap& m0, const CUtensorMap& m1, const UnitArgs& a, int groups, cudaStream_t st,
+                        int num_sms, bool pdl) {
+  auto kern = k_tiles<MODE, F0, F1, NT, BSM>;
+  UnitArgs args = a;
+  args.div_s = FastDiv::of((uint32_t)a.splits);
+  args.div_tiles = FastDiv::of((uint32_t)((a.w0.rows + kTile - 1) / kTile));
+  const size_t smem = tiles_smem<MODE, F0, F1, NT>(a.w0.cols, a.T, a.T * a.topk, BSM ? a.act_rows : 0);
+  if (set_smem(kern, smem)) return -4;
+  KernelCache* kc = kcache(reinterpret_cast<const void*>(kern));
+  int per_sm = 0;
+  if (kc && kc->occ_smem == smem) {
+    per_sm = kc->occ;
+  } else {
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kDecodeWarps * 32, smem) != cudaSuccess) return -4;
+    if (kc) {
+      kc->occ_smem = smem;
+      kc->occ = per_sm;
+    }
+  }
+  if (per_sm < 1) return -4;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(std::max(1, std::min(groups, per_sm * num_sms)));
+  cfg.blockDim = dim3(kDecodeWarps * 32);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute at[1] = {pdl_attr()};
+  cfg.attrs = at;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kern, m0, m1, args) == cudaSuccess ? 0 : -4;
+}
+
+// Activation rows a stream launch can keep in shared memory (0: read them
+// through the read-only path instead).
+static int act_rows_smem(int NT, int rows_needed, int cols) {
+  if (NT != 1) return 0;
+  return (size_t)rows_needed * (cols / 64 * 80) * 2 <= kActSmemMax ? rows_needed : 0;
+}
+
+static void split_args(UnitArgs& a, int cols) {
+  a.bpi = item_blocks(cols);
+  a.splits = (cols / 256) / a.bpi;
+  a.async_sc = a.bpi == 4;
+}
+
+template <int MODE, int F0, int F1, int NT>
+static int launch_stream_any(const CUtensorMap& m0, const CUtensorMap& m1, UnitArgs a, int items, cudaStream_t st,
+                             int num_sms, bool pdl, int act_rows) {
+  if constexpr (NT == 1) {
+    if (act_rows > 0) {
+      a.act_rows = act_rows;
+      return launch_stream<MODE, F0, F1, NT, true>(m0, m1, a, items, st, num_sms, pdl);
+    }
+  }
+  a.act_rows = 0;
+  return launch_stream<MODE, F0, F1, NT, false>(m0, m1, a, items, st, num_sms, pdl);
 }
 
 template <int FMT, int NT>
 static int gemv_impl(const WDev& w, int expert, const Values& V, const uint16_t* x, int T, float* y, char* ws,
                      cudaStream_t st, int num_sms) {
-  const int ch = chunk_blocks(w.cols);
   const GemvWs L = gemv_ws(T, w.rows, w.cols);
+  UnitArgs a = {};
+  split_args(a, w.cols);
   CUtensorMap map;
-  if (make_qs_map(&map, w, ch)) return -4;
+  if (make_qs_map(&map, w, a.bpi)) return -4;
   uint16_t* xp = reinterpret_cast<uint16_t*>(ws + L.xperm);
   int32_t* status = reinterpret_cast<int32_t*>(ws + L.status);
+  int32_t* cnt = reinterpret_cast<int32_t*>(ws + L.cnt);
+  const int tiles = (w.rows + kTile - 1) / kTile;
   const int pblocks = std::max(1, std::min(num_sms, (int)(((int64_t)T * (w.cols / 16) + 63) / 64)));
-  k_prep<<<pblocks, 256, 0, st>>>(x, T, w.cols, xp, nullptr, 0, nullptr, 0, 1, status);
+  const int nzero = (int)((L.part - L.cnt) / 4);  // the tile counters
+  k_prep<<<pblocks, 256, 0, st>>>(x, T, w.cols, xp, cnt, nzero, nullptr, 0, 1, status);
   if (cudaGetLastError() != cudaSuccess) return -4;
-  UnitArgs a = {};
   a.w0 = w;
   a.w1 = w;
   a.V = V;
   a.act = xp;
+  a.xraw = x;
   a.T = T;
   a.topk = 1;
   a.expert = expert;
   a.yf = y;
+  a.cnt = cnt;
+  a.part = reinterpret_cast<float*>(ws + L.part);
   a.status = status;
-  a.ch = ch;
-  return launch_stream<MODE_GEMV, FMT, FMT, NT>(map, map, a, (w.rows + kTile - 1) / kTile, st, num_sms, true);
+  return launch_stream_any<MODE_GEMV, FMT, FMT, NT>(map, map, a, tiles * a.splits, st, num_sms, true,
+                                                    act_rows_smem(NT, T, w.cols));
 }
 
 int launch_gemv(const WDev& w, int fmt, int expert, const Values& V, const uint16_t* x, int T, float* y, char* ws,
@@ -872,9 +1354,9 @@ DecodeWs decode_ws(int T, int topk, int experts, int hidden, int inter) {
   ws.cnt3 = o;
   o = align256(o + (size_t)ws.c3.tiles * 4);
   ws.part2 = o;
-  o = align256(o + (size_t)ws.dmax * ws.c2.tiles * 2 * ws.nc * kTile * 4);
+  o = align256(o + (size_t)ws.dmax * ws.c2.tiles * 2 * ws.c2.nkc * ws.nc * kTile * 4);
   ws.part3 = o;
-  o = align256(o + (size_t)ws.c3.tiles * npairs * kTile * 4);
+  o = align256(o + (size_t)ws.c3.tiles * npairs * ws.c3.nkc * kTile * 4);
   ws.total = o;
   return ws;
 }
@@ -885,9 +1367,10 @@ static int decode_impl(const WDev& g, const WDev& u, const WDev& d, const Values
                        int num_sms) {
   const DecodeWs L = decode_ws(T, topk, g.experts, g.cols, g.rows);
   const int npairs = T * topk;
-  const int ch2 = chunk_blocks(g.cols), ch3 = chunk_blocks(d.cols);
+  UnitArgs a = {};
+  split_args(a, g.cols);
   CUtensorMap mg, mu, md;
-  if (make_qs_map(&mg, g, ch2) || make_qs_map(&mu, u, ch2) || make_qs_map(&md, d, ch3)) return -4;
+  if (make_qs_map(&mg, g, a.bpi) || make_qs_map(&mu, u, a.bpi) || make_qs_map(&md, d, item_blocks(d.cols))) return -4;
   int32_t* status = reinterpret_cast<int32_t*>(ws + L.status);
   uint16_t* xp = reinterpret_cast<uint16_t*>(ws + L.xperm);
   uint16_t* hp = reinterpret_cast<uint16_t*>(ws + L.hperm);
@@ -897,31 +1380,45 @@ static int decode_impl(const WDev& g, const WDev& u, const WDev& d, const Values
   const int pblocks = std::max(1, std::min(num_sms, (int)(((int64_t)T * (g.cols / 16) + 63) / 64)));
   k_prep<<<pblocks, 256, 0, st>>>(x, T, g.cols, xp, cnt2, nzero, ids, npairs, g.experts, status);
   if (cudaGetLastError() != cudaSuccess) return -4;
-  UnitArgs a = {};
   a.w0 = g;
   a.w1 = u;
   a.V = V;
   a.ids = ids;
   a.p = p;
   a.act = xp;
+  a.xraw = x;
   a.T = T;
   a.topk = topk;
   a.out16 = hp;
   a.cnt = cnt2;
   a.part = reinterpret_cast<float*>(ws + L.part2);
   a.status = status;
-  a.ch = ch2;
-  int rc = launch_stream<MODE_GATEUP, FG, FU, NT>(mg, mu, a, L.dmax * 2 * L.c2.tiles, st, num_sms, true);
+  int rc;
+  if constexpr (NT <= 2) {
+    const int ar = act_rows_smem(NT, T, g.cols);
+    a.act_rows = ar;
+    rc = ar ? launch_tiles<MODE_GATEUP, FG, FU, NT, true>(mg, mu, a, L.dmax * L.c2.tiles, st, num_sms, true)
+            : launch_tiles<MODE_GATEUP, FG, FU, NT, false>(mg, mu, a, L.dmax * L.c2.tiles, st, num_sms, true);
+  } else {
+    rc = launch_stream_any<MODE_GATEUP, FG, FU, NT>(mg, mu, a, L.dmax * 2 * L.c2.tiles * a.splits, st, num_sms, true,
+                                                    0);
+  }
   if (rc) return rc;
   UnitArgs b = a;
+  split_args(b, d.cols);
   b.w0 = d;
   b.w1 = d;
   b.act = hp;
   b.out16 = y;
   b.cnt = cnt3;
   b.part = reinterpret_cast<float*>(ws + L.part3);
-  b.ch = ch3;
-  return launch_stream<MODE_DOWN, FD, FD, NT>(md, md, b, L.dmax * L.c3.tiles, st, num_sms, true);
+  if constexpr (NT <= 2) {
+    const int ar = act_rows_smem(NT, npairs, d.cols);
+    b.act_rows = ar;
+    return ar ? launch_tiles<MODE_DOWN, FD, FD, NT, true>(md, md, b, L.c3.tiles, st, num_sms, true)
+              : launch_tiles<MODE_DOWN, FD, FD, NT, false>(md, md, b, L.c3.tiles, st, num_sms, true);
+  }
+  return launch_stream_any<MODE_DOWN, FD, FD, NT>(md, md, b, L.dmax * L.c3.tiles * b.splits, st, num_sms, true, 0);
 }
 
 int launch_moe_decode(const WDev& g, int fg, const WDev& u, int fu, const WDev& d, int fd, const Values& V,
@@ -942,10 +1439,11 @@ int launch_moe_decode(const WDev& g, int fg, const WDev& u, int fu, const WDev& 
 
 int launch_floor(const WDev& w, int fmt, const int32_t* experts, int n, uint32_t* out, cudaStream_t st,
                  int num_sms) {
-  const int ch = chunk_blocks(w.cols);
-  CUtensorMap map;
-  if (make_qs_map(&map, w, ch)) return -4;
   UnitArgs a = {};
+  split_args(a, w.cols);
+  CUtensorMap map;
+  if (make_qs_map(&map, w, a.bpi)) return -4;
+  if (cudaMemsetAsync(out, 0, (size_t)n * w.rows * 4, st) != cudaSuccess) return -4;
   a.w0 = w;
   a.w1 = w;
   a.elist = experts;
@@ -953,11 +1451,10 @@ int launch_floor(const WDev& w, int fmt, const int32_t* experts, int n, uint32_t
   a.outx = out;
   a.T = 1;
   a.topk = 1;
-  a.ch = ch;
   a.status = nullptr;  // the floor reports a timeout through g_floor_status
-  const int units = n * ((w.rows + kTile - 1) / kTile);
-  if (fmt == FMT_KS) return launch_stream<MODE_FLOOR, FMT_KS, FMT_KS, 1>(map, map, a, units, st, num_sms, false);
-  return launch_stream<MODE_FLOOR, FMT_K, FMT_K, 1>(map, map, a, units, st, num_sms, false);
+  const int items = n * ((w.rows + kTile - 1) / kTile) * a.splits;
+  if (fmt == FMT_KS) return launch_stream<MODE_FLOOR, FMT_KS, FMT_KS, 1, false>(map, map, a, items, st, num_sms, false);
+  return launch_stream<MODE_FLOOR, FMT_K, FMT_K, 1, false>(map, map, a, items, st, num_sms, false);
 }
 
 }  // namespace iqk

@@ -171,6 +171,22 @@ __device__ __forceinline__ Pair2 lookup_slot_mh(uint32_t q, int i, uint32_t t0, 
   return r;
 }
 
+// Same, with the 2i-bit pre-shift of slot i also done as a multiply-high by
+// `k_shift` (= 2^(32 - 2i), opaque): balances the integer-logic and FMA pipes.
+__device__ __forceinline__ Pair2 lookup_slot_mh2(uint32_t q, uint32_t t0, uint32_t t1, uint32_t k65536,
+                                                 uint32_t k_shift) {
+  uint32_t qs;
+  asm("mul.hi.u32 %0, %1, %2;" : "=r"(qs) : "r"(q), "r"(k_shift));
+  uint32_t u = qs & 0x03030303u;
+  uint32_t s = u * 0x22u + 0x10101010u;
+  uint32_t sh;
+  asm("mul.hi.u32 %0, %1, %2;" : "=r"(sh) : "r"(s), "r"(k65536));
+  Pair2 r;
+  r.lo = prmt(t0, t1, s);
+  r.hi = prmt(t0, t1, sh);
+  return r;
+}
+
 __device__ __forceinline__ uint32_t opaque_u32(uint32_t v) {
   uint32_t r;
   asm volatile("mov.u32 %0, %1;" : "=r"(r) : "r"(v));
@@ -181,6 +197,10 @@ __device__ __forceinline__ uint4 ld_nc_u4(const void* p) {
   uint4 r;
   asm volatile("ld.global.nc.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w) : "l"(p));
   return r;
+}
+
+__device__ __forceinline__ void prefetch_l1(const void* p) {
+  asm volatile("prefetch.global.L1 [%0];" ::"l"(p));
 }
 
 // Position of k within its 16-group after the slot transpose used by the

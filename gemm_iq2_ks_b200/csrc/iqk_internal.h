@@ -16,20 +16,49 @@ int launch_dequant(const WDev& w, int fmt, int expert, const Values& V, void* ou
                    cudaStream_t st, int num_sms);
 
 // ------------------------------------------------------- decode (GEMV-type)
-// Unit geometry shared by the GEMV-shaped kernels: 16-row tiles, each unit a
-// run of `nb` 256-weight blocks of one tile ("k-chunk"), split over `nkc`
-// chunks per row.
+// Item geometry shared by the GEMV-shaped kernels: 16-row tiles, each item a
+// run of `nb` 256-weight blocks of one tile (a slice of the reduction width),
+// `nkc` slices per row.
 struct Chunking {
-  int nb;     // blocks per unit (1, 2 or 4)
-  int nkc;    // chunks per row = blocks_per_row / nb
+  int nb;     // blocks per item (1, 2 or 4)
+  int nkc;    // slices per row = blocks_per_row / nb
   int tiles;  // ceil(rows / 16)
 };
 Chunking chunking(int rows, int cols);
+int item_blocks(int cols);
 
 constexpr int kTile = 16;
-constexpr int kDecodeWarps = 4;
-constexpr int kStages = 4;
+#ifndef IQK_DECODE_WARPS
+#define IQK_DECODE_WARPS 8
+#endif
+#ifndef IQK_DECODE_STAGES
+#define IQK_DECODE_STAGES 2
+#endif
+constexpr int kDecodeWarps = IQK_DECODE_WARPS;  // warps per decode CTA, each with its own ring
+constexpr int kStages = IQK_DECODE_STAGES;      // ring stages per warp, one item each
+// Resident CTAs per SM the decode kernels are compiled for (16 warps per SM
+// with one or two MMA column groups, 8 with more).
+constexpr int kDecodeMinBlocks(int nt) {
+  return nt >= 4 ? (8 / kDecodeWarps > 0 ? 8 / kDecodeWarps : 1) : (16 / kDecodeWarps > 0 ? 16 / kDecodeWarps : 1);
+}
 constexpr int kMaxPairs = 1024;  // decode: T * topk
+
+// n / d for 0 <= n < 2^31 as (umulhi(n, m) + n) >> s, with m and s fixed on
+// the host (division by an invariant integer, Granlund and Montgomery 1994).
+struct FastDiv {
+  uint32_t m, s;
+  static FastDiv of(uint32_t d) {
+    FastDiv f{0u, 0u};
+    if (d > 1) {
+      uint32_t l = 0;
+      while ((1ull << l) < d) l++;
+      f.m = (uint32_t)((((1ull << 32) * ((1ull << l) - d)) / d) + 1);
+      f.s = l;
+    }
+    return f;
+  }
+  __device__ __forceinline__ uint32_t div(uint32_t n) const { return (__umulhi(n, m) + n) >> s; }
+};
 
 // Workspace carve-up for iqk_gemv.
 struct GemvWs {
