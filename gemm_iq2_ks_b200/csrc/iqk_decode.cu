@@ -30,12 +30,16 @@
 
 namespace iqk {
 
-// Blocks per item: four when the row's block count allows (the scale slices
-// then start on the boundaries cp.async needs), else two or one.
+// Blocks per item: four for rows of at least 16 blocks, two for shorter rows
+// with a multiple of four blocks (more items to spread over the warps), else
+// two or one. With a multiple of four blocks per row every scale slice lies
+// on the boundaries cp.async needs.
 int item_blocks(int cols) {
   const int nbk = cols / 256;
-  return nbk % 4 == 0 ? 4 : nbk % 2 == 0 ? 2 : 1;
+  if (nbk % 4 == 0) return nbk >= 16 ? 4 : 2;
+  return nbk % 2 == 0 ? 2 : 1;
 }
+static bool async_scales(int cols) { return (cols / 256) % 4 == 0; }
 
 Chunking chunking(int rows, int cols) {
   Chunking c;
@@ -48,15 +52,17 @@ Chunking chunking(int rows, int cols) {
 
 // ---------------------------------------------------------- item scales
 // An item's scale slice (16 rows x bpi blocks) sits in a per-stage slot:
-//   IQ2_KS: scl [16][bpi] u32 | sch [16][bpi] u8 | sex [16][bpi] u8
+//   IQ2_KS: scl [16][bpi] u32 | sch [16][4] u8 | sex [16][4] u8
 //   IQ2_K:  scl [16][2 bpi] u32 | sex [16][bpi] u16 | dv [16][bpi] u16
-// Every part starts on a 16-byte boundary (bpi = 1, 2 or 4). The IQ2_KS row
-// scale is read straight from global memory at the start of the item.
+// Every part starts on a 16-byte boundary (bpi = 1, 2 or 4). An IQ2_KS row of
+// sch / sex holds the aligned 4-byte window around the slice's bpi bytes
+// (cp.async copies 4 bytes at least); the slice starts `o` bytes into it. The
+// IQ2_KS row scale is read straight from global memory at the start of the item.
 template <int FMT>
 struct Slot {
   static __host__ __device__ __forceinline__ uint32_t b_off(int bpi) { return FMT == FMT_KS ? 64u * bpi : 128u * bpi; }
-  static __host__ __device__ __forceinline__ uint32_t c_off(int bpi) { return FMT == FMT_KS ? 80u * bpi : 160u * bpi; }
-  static __host__ __device__ __forceinline__ uint32_t bytes(int bpi) { return FMT == FMT_KS ? 96u * bpi : 192u * bpi; }
+  static __host__ __device__ __forceinline__ uint32_t c_off(int bpi) { return FMT == FMT_KS ? 64u * bpi + 64u : 160u * bpi; }
+  static __host__ __device__ __forceinline__ uint32_t bytes(int bpi) { return FMT == FMT_KS ? 64u * bpi + 128u : 192u * bpi; }
 };
 
 // Bytes between consecutive slots: the larger format's slot, rounded up to
@@ -71,11 +77,11 @@ __host__ __device__ inline uint32_t slot_bytes2(int bpi) {
 // IQ2_KS: (low4 | high<<4) + 32*alphabet, words (4t, 4t+1) in sub-block 2t.
 // IQ2_K:  nibble + 16*alphabet, word 4t+m is sub-block 4t+m.
 template <int FMT>
-__device__ __forceinline__ void combos_smem(const uint8_t* slot, int bpi, int r, int lb, int t, uint32_t (&c)[4]) {
+__device__ __forceinline__ void combos_smem(const uint8_t* slot, int bpi, int o, int r, int lb, int t, uint32_t (&c)[4]) {
   if constexpr (FMT == FMT_KS) {
     const uint32_t sb = slot[(r * bpi + lb) * 4 + t];
-    const uint32_t h = slot[Slot<FMT>::b_off(bpi) + r * bpi + lb];
-    const uint32_t a = slot[Slot<FMT>::c_off(bpi) + r * bpi + lb];
+    const uint32_t h = slot[Slot<FMT>::b_off(bpi) + r * 4 + o + lb];
+    const uint32_t a = slot[Slot<FMT>::c_off(bpi) + r * 4 + o + lb];
     const uint32_t hb = (h >> (2 * t)) & 3u;
     const uint32_t ab = (a >> (2 * t)) & 3u;
     const uint32_t c0 = (sb & 15u) | ((hb & 1u) << 4) | ((ab & 1u) << 5);
@@ -192,7 +198,7 @@ __device__ __forceinline__ void block_mma(const uint32_t* __restrict__ sq, int l
 // One item (16 rows x bpi blocks) of a matrix in format F0 (fmt0) or F1:
 // acc[n] = d * sum over the item's blocks of W * B, rows g and g + 8.
 template <int F0, int F1, int NT, bool BSM>
-__device__ __forceinline__ void item_mma(const uint32_t* sq, const uint8_t* slot, int bpi, int ldw,
+__device__ __forceinline__ void item_mma(const uint32_t* sq, const uint8_t* slot, int bpi, int o, int ldw,
                                          const uint16_t* const (&bsrc)[NT], bool fmt0, bool kfmt, const uint2* lut0,
                                          const uint2* lut1, float dg, float dh, int g, int t, uint32_t k65536,
                                          float (&acc)[NT][4]) {
@@ -213,11 +219,11 @@ __device__ __forceinline__ void item_mma(const uint32_t* sq, const uint8_t* slot
     }
     uint32_t cg[4], ch[4];
     if (fmt0) {
-      combos_smem<F0>(slot, bpi, g, b, t, cg);
-      combos_smem<F0>(slot, bpi, g + 8, b, t, ch);
+      combos_smem<F0>(slot, bpi, o, g, b, t, cg);
+      combos_smem<F0>(slot, bpi, o, g + 8, b, t, ch);
     } else {
-      combos_smem<F1>(slot, bpi, g, b, t, cg);
-      combos_smem<F1>(slot, bpi, g + 8, b, t, ch);
+      combos_smem<F1>(slot, bpi, o, g, b, t, cg);
+      combos_smem<F1>(slot, bpi, o, g + 8, b, t, ch);
     }
     if (kfmt) {
 #pragma unroll
@@ -398,7 +404,7 @@ struct UnitArgs {
   int32_t* status;
   int bpi;       // 256-weight blocks per item
   int splits;    // items per tile and matrix (blocks per row / bpi)
-  int async_sc;  // scale slices by cp.async (bpi == 4)
+  int async_sc;  // scale slices by cp.async (blocks per row a multiple of four)
   int act_rows;  // BSM: activation rows copied into shared memory
   FastDiv div_s, div_tiles;
 };
@@ -418,34 +424,35 @@ __device__ __forceinline__ void cp_async_arrive(uint64_t* bar) {
 }
 
 // Stage the scale slice of rows [R0, R0 + valid) and blocks [s*bpi, (s+1)*bpi)
-// of `w` into `slot`. With `async` (bpi == 4, so every row piece is 4-, 8- or
-// 16-byte aligned) the lanes issue cp.async copies tracked by `bar`;
-// otherwise they copy with plain loads, zero past the last row, and the call
+// of `w` into `slot`. With `async` (blocks per row a multiple of four and bpi
+// 2 or 4, so every row piece is 4-, 8- or 16-byte aligned) the lanes issue
+// cp.async copies tracked by `bar`; otherwise they copy with plain loads
+// (IQ2_KS sch / sex at window offset 0), zero past the last row, and the call
 // ends with __syncwarp.
 template <int FMT>
 __device__ __forceinline__ void stage_scales(uint8_t* slot, const WDev& w, int64_t R0, int valid, int s, int bpi,
                                              bool async, uint64_t* bar, int lane) {
   const int nbk = w.cols / 256;
   if (async) {
-    if (FMT == FMT_KS) {
-      const int r = lane & 15;
-      if (r < valid) {
-        const int64_t o = (R0 + r) * nbk + 4 * s;
+    const int r = lane & 15;
+    if (r < valid) {
+      const int64_t o = (R0 + r) * nbk + (int64_t)s * bpi;  // first block of the slice in the row's planes
+      if (FMT == FMT_KS) {
         if (lane < 16) {
-          cp_async16(slot + 16 * r, w.scl + o);
+          if (bpi == 4) cp_async16(slot + 16 * r, w.scl + o);
+          else cp_async8(slot + 8 * r, w.scl + o);
         } else {
-          cp_async4(slot + 256 + 4 * r, w.sch + o);
-          cp_async4(slot + 320 + 4 * r, reinterpret_cast<const uint8_t*>(w.sex) + o);
+          const int64_t win = o & ~(int64_t)3;
+          cp_async4(slot + Slot<FMT>::b_off(bpi) + 4 * r, w.sch + win);
+          cp_async4(slot + Slot<FMT>::c_off(bpi) + 4 * r, reinterpret_cast<const uint8_t*>(w.sex) + win);
         }
-      }
-    } else {
-      const int r = lane >> 1, h = lane & 1;
-      if (r < valid) cp_async16(slot + 32 * r + 16 * h, w.scl + (R0 + r) * 2 * nbk + 8 * s + 4 * h);
-      const int r2 = lane & 15;
-      if (r2 < valid) {
-        const int64_t o = (R0 + r2) * nbk + 4 * s;
-        if (lane < 16) cp_async8(slot + 512 + 8 * r2, reinterpret_cast<const uint16_t*>(w.sex) + o);
-        else cp_async8(slot + 640 + 8 * r2, w.dv + o);
+      } else {
+        if (bpi == 4) cp_async16(slot + 32 * r + 16 * (lane >> 4), w.scl + 2 * o + 4 * (lane >> 4));
+        else if (lane < 16) cp_async16(slot + 16 * r, w.scl + 2 * o);
+        const uint16_t* src = lane < 16 ? reinterpret_cast<const uint16_t*>(w.sex) + o : w.dv + o;
+        uint8_t* dst = slot + (lane < 16 ? Slot<FMT>::b_off(bpi) : Slot<FMT>::c_off(bpi)) + 2 * bpi * r;
+        if (bpi == 4) cp_async8(dst, src);
+        else cp_async4(dst, src);
       }
     }
     cp_async_arrive(bar);
@@ -462,8 +469,8 @@ __device__ __forceinline__ void stage_scales(uint8_t* slot, const WDev& w, int64
     for (int i = lane; i < 16 * bpi; i += 32) {
       const int r = i / bpi, b = i - r * bpi;
       const int64_t o = (R0 + r) * nbk + s * bpi + b;
-      sb[i] = r < valid ? __ldg(w.sch + o) : (uint8_t)0;
-      sc[i] = r < valid ? __ldg(reinterpret_cast<const uint8_t*>(w.sex) + o) : (uint8_t)0;
+      sb[4 * r + b] = r < valid ? __ldg(w.sch + o) : (uint8_t)0;
+      sc[4 * r + b] = r < valid ? __ldg(reinterpret_cast<const uint8_t*>(w.sex) + o) : (uint8_t)0;
     }
   } else {
     uint32_t* d32 = reinterpret_cast<uint32_t*>(slot);
@@ -688,10 +695,11 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, kDecodeMinBlocks(NT)) k_str
       if (ks) {
         const uint8_t* sb = slot + Slot<FMT_KS>::b_off(bpi);
         const uint8_t* sc = slot + Slot<FMT_KS>::c_off(bpi);
+        const int o = A.async_sc ? (s * bpi) & 3 : 0;
         for (int i = t; i < bpi; i += 4) {
           const int sh = 8 * ((s * bpi + i) & 3);
-          xg ^= ((uint32_t)sb[g * bpi + i] ^ (uint32_t)sc[g * bpi + i]) << sh;
-          xh ^= ((uint32_t)sb[(g + 8) * bpi + i] ^ (uint32_t)sc[(g + 8) * bpi + i]) << sh;
+          xg ^= ((uint32_t)sb[g * 4 + o + i] ^ (uint32_t)sc[g * 4 + o + i]) << sh;
+          xh ^= ((uint32_t)sb[(g + 8) * 4 + o + i] ^ (uint32_t)sc[(g + 8) * 4 + o + i]) << sh;
         }
         if (s == 0 && t == 0) {  // the row scale belongs to the first slice
           if (g < valid) xg ^= __ldg(A.w0.dv + R0 + g);
@@ -707,7 +715,8 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, kDecodeMinBlocks(NT)) k_str
         }
       }
     } else {
-      item_mma<F0, F1, NT, BSM>(sq, slot, bpi, ldw, bsrc, fmt0, kfmt, lut0, lut1, dg, dh, g, t, k65536, acc);
+      const int o = A.async_sc ? (s * bpi) & 3 : 0;
+      item_mma<F0, F1, NT, BSM>(sq, slot, bpi, o, ldw, bsrc, fmt0, kfmt, lut0, lut1, dg, dh, g, t, k65536, acc);
     }
     __syncwarp();
     issue(it + kStages);  // refill the stage just consumed
@@ -880,6 +889,20 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, kDecodeMinBlocks(NT)) k_til
   float* red = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(act_s) + (BSM ? (size_t)A.act_rows * KP * 2 : 0));
   const int slot_f = MODE == MODE_GATEUP ? 2 * NC * kTile : A.T * kTile;  // floats per warp slot
   uint8_t* route_p = reinterpret_cast<uint8_t*>(red + (size_t)kDecodeWarps * slot_f);
+  // gate/up: request the first activation groups ahead of the weight stream
+  uint4 pre0 = make_uint4(0u, 0u, 0u, 0u), pre1 = pre0, pre2 = pre0, pre3 = pre0;
+  const int act_groups = BSM ? A.act_rows * (K / 16) : 0;
+  if (BSM && MODE == MODE_GATEUP) {
+    const int g0 = threadIdx.x, g1 = threadIdx.x + blockDim.x;
+    if (g0 < act_groups) {
+      pre0 = ld_nc_u4(A.xraw + (size_t)g0 * 16);
+      pre1 = ld_nc_u4(A.xraw + (size_t)g0 * 16 + 8);
+    }
+    if (g1 < act_groups) {
+      pre2 = ld_nc_u4(A.xraw + (size_t)g1 * 16);
+      pre3 = ld_nc_u4(A.xraw + (size_t)g1 * 16 + 8);
+    }
+  }
   build_lut<F0>(lut0, A.V);
   if (MODE == MODE_GATEUP) build_lut<F1>(lut1, A.V);
   if (lane == 0) {
@@ -942,8 +965,9 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, kDecodeMinBlocks(NT)) k_til
   }
   if constexpr (BSM) {  // activation rows, slot-transposed and padded, once per CTA
     const int gpr = K / 16;
-    const int groups = A.act_rows * gpr;
-    for (int gi = threadIdx.x; gi < groups; gi += blockDim.x) {
+    for (int k = 0;; k++) {
+      const int gi = threadIdx.x + k * blockDim.x;
+      if (gi >= act_groups) break;
       const int r = gi / gpr, c0 = (gi - r * gpr) * 16;
       uint32_t o[8];
       if (MODE == MODE_DOWN) {
@@ -952,7 +976,8 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, kDecodeMinBlocks(NT)) k_til
         o[0] = a.x; o[1] = a.y; o[2] = a.z; o[3] = a.w; o[4] = b.x; o[5] = b.y; o[6] = b.z; o[7] = b.w;
       } else {
         const uint4* src = reinterpret_cast<const uint4*>(A.xraw + (size_t)gi * 16);
-        const uint4 a = ld_nc_u4(src), b = ld_nc_u4(src + 1);
+        const uint4 a = k == 0 ? pre0 : k == 1 ? pre2 : ld_nc_u4(src);
+        const uint4 b = k == 0 ? pre1 : k == 1 ? pre3 : ld_nc_u4(src + 1);
         const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
 #pragma unroll
         for (int i2 = 0; i2 < 4; i2++) {
@@ -1025,7 +1050,8 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, kDecodeMinBlocks(NT)) k_til
         consumed = q + 1;
         const uint32_t* sq = ring_qs + (size_t)st * stage_words;
         const uint8_t* slot = ring_slots + (size_t)st * slot_b;
-        item_mma<F0, F1, NT, BSM>(sq, slot, bpi, ldw, bsrc, fmt0, kfmt, lut0, lut1, dg, dh, g, t, k65536, acc);
+        const int o = A.async_sc ? (s * bpi) & 3 : 0;
+        item_mma<F0, F1, NT, BSM>(sq, slot, bpi, o, ldw, bsrc, fmt0, kfmt, lut0, lut1, dg, dh, g, t, k65536, acc);
         __syncwarp();
         issue(q + kStages);  // refill the stage just consumed
       }
@@ -1275,7 +1301,7 @@ static int act_rows_smem(int NT, int rows_needed, int cols) {
 static void split_args(UnitArgs& a, int cols) {
   a.bpi = item_blocks(cols);
   a.splits = (cols / 256) / a.bpi;
-  a.async_sc = a.bpi == 4;
+  a.async_sc = async_scales(cols) ? 1 : 0;
 }
 
 template <int MODE, int F0, int F1, int NT>
