@@ -200,36 +200,37 @@ class DecodeBench:
 
 
 def e2e_graph(torch, bench, stream, n):
-    """n steps, each: pinned-host x/ids/p -> device, decode, y -> pinned host."""
+    """n steps, each: one pinned-host -> device copy of the call's inputs (x,
+    ids and p packed in one buffer), the decode, and y -> pinned host."""
     T = bench.T
-    hx = torch.empty((n, T, S.HIDDEN), dtype=torch.bfloat16, pin_memory=True)
-    hx.copy_(bench.x[:n].cpu())
-    hids = bench.ids[:n].cpu().pin_memory()
-    hp = bench.p[:n].cpu().pin_memory()
+    nx, ni = T * S.HIDDEN * 2, T * S.TOPK * 4
+    step = nx + 2 * ni
+    hin = torch.empty((n, step), dtype=torch.uint8, pin_memory=True)
+    for c in range(n):
+        hin[c, :nx].copy_(bench.x[c].cpu().view(torch.uint8).reshape(-1))
+        hin[c, nx:nx + ni].copy_(bench.ids[c].cpu().view(torch.uint8).reshape(-1))
+        hin[c, nx + ni:].copy_(bench.p[c].cpu().view(torch.uint8).reshape(-1))
     hy = torch.empty((n, T, S.HIDDEN), dtype=torch.bfloat16, pin_memory=True)
-    dx = torch.empty((T, S.HIDDEN), dtype=torch.bfloat16, device=bench.x.device)
-    dids = torch.empty((T, S.TOPK), dtype=torch.int32, device=bench.x.device)
-    dp = torch.empty((T, S.TOPK), dtype=torch.float32, device=bench.x.device)
+    din = torch.empty((step,), dtype=torch.uint8, device=bench.x.device)
+    dx = din[:nx].view(torch.bfloat16).view(T, S.HIDDEN)
+    dids = din[nx:nx + ni].view(torch.int32).view(T, S.TOPK)
+    dp = din[nx + ni:].view(torch.float32).view(T, S.TOPK)
     dy = torch.empty((T, S.HIDDEN), dtype=torch.bfloat16, device=bench.x.device)
     g, u, d = bench.dw
 
     with torch.cuda.stream(stream):
-        bench.B.iqk_moe_decode(g, u, d, bench.values, bench.x[0], bench.ids[0], bench.p[0], y=dy, ws=bench.ws,
-                               stream=stream)
+        din.copy_(hin[0], non_blocking=True)
+        bench.B.iqk_moe_decode(g, u, d, bench.values, dx, dids, dp, y=dy, ws=bench.ws, stream=stream)
     torch.cuda.synchronize()
 
     def body():
         for c in range(n):
-            dx.copy_(hx[c], non_blocking=True)
-            dids.copy_(hids[c], non_blocking=True)
-            dp.copy_(hp[c], non_blocking=True)
+            din.copy_(hin[c], non_blocking=True)
             bench.B.iqk_moe_decode(g, u, d, bench.values, dx, dids, dp, y=dy, ws=bench.ws, stream=stream)
             hy[c].copy_(dy, non_blocking=True)
 
     graph = capture(torch, stream, body)
-    h2d = T * S.HIDDEN * 2 + T * S.TOPK * 4 * 2
-    d2h = T * S.HIDDEN * 2
-    return graph, h2d, d2h, hy
+    return graph, step, T * S.HIDDEN * 2, hy
 
 
 def floor_graph(torch, bench, stream, n):
@@ -252,6 +253,64 @@ def floor_graph(torch, bench, stream, n):
             B.iqk_floor(d, lists[c], out=outs[c][1], stream=stream)
 
     return capture(torch, stream, body)
+
+
+def prefill_leg(torch, B, weights, values, device, stream, peaks, calls=4, reps=3):
+    """Config 4: 2048 tokens routed top-6 over 256 experts, one prefill call =
+    route + grouped gate/up GEMM + SwiGLU + grouped down GEMM + combine."""
+    T = 2048
+    rng = S.rng_for(4)
+    ids, p = S.routing(rng, T, weights[0].experts, S.TOPK)
+    x = S.random_bf16(rng, (T, S.HIDDEN))
+    dw = [B.Weights.from_host(w, device) for w in weights]
+    xd = torch.from_numpy(x.view(np.int16)).to(device).view(torch.bfloat16)
+    idsd = torch.from_numpy(ids).to(device)
+    pd = torch.from_numpy(p).to(device)
+    y = torch.empty((T, S.HIDDEN), dtype=torch.bfloat16, device=device)
+    ws = B.workspace(B.iqk_moe_workspace_bytes(1, T, S.TOPK, weights[0].experts, S.HIDDEN, S.INTER), device)
+
+    def call():
+        B.iqk_moe_prefill(dw[0], dw[1], dw[2], values, xd, idsd, pd, y=y, ws=ws, stream=stream)
+
+    with torch.cuda.stream(stream):
+        call()
+    torch.cuda.synchronize()
+    g = capture(torch, stream, lambda: [call() for _ in range(calls)])
+    with torch.cuda.stream(stream):
+        g.replay()
+    torch.cuda.synchronize()
+    t = cuda_time(torch, stream, lambda: [g.replay() for _ in range(reps)])
+    per_call = t / (calls * reps)
+    flops = 2.0 * T * S.TOPK * 3 * S.INTER * S.HIDDEN
+    tf = flops / per_call / 1e12
+    status = B.iqk_moe_status(ws)
+    del g, dw
+    return {"workload": "routed-expert prefill, IQ2_KS, 2048 tokens, 256 experts top-6 (config 4)",
+            "us_per_call": per_call * 1e6, "tflops": tf, "flop_per_call": flops,
+            "roofline": {"bound": "tensor", "achieved": tf, "peak": peaks["bf16"], "unit": "TFLOP/s",
+                         "frac": tf / peaks["bf16"], "frac_of_sustained": tf / peaks["bf16_sustained"],
+                         "peak_source": peaks["source"] + " bf16_tflops (cuBLAS burst)"},
+            "weight_gbs": sum(w.nbytes() for w in weights) / per_call / 1e9, "status": status}
+
+
+def gemv_leg(torch, B, cfg, device, stream, calls=200):
+    """Configs 0 and 1: one matrix, one activation row (the inputs stay L2-resident)."""
+    w, x, values = S.matrix_case(cfg)
+    dw = B.Weights.from_host(w, device)
+    xd = torch.from_numpy(x.view(np.int16)).to(device).view(torch.bfloat16)
+    y = torch.empty((xd.shape[0], w.rows), dtype=torch.float32, device=device)
+    ws = B.workspace(B.iqk_gemv_workspace_bytes(xd.shape[0], w.rows, w.cols), device)
+    with torch.cuda.stream(stream):
+        B.iqk_gemv(dw, 0, values, xd, y=y, ws=ws, stream=stream)
+    torch.cuda.synchronize()
+    g = capture(torch, stream, lambda: [B.iqk_gemv(dw, 0, values, xd, y=y, ws=ws, stream=stream)
+                                        for _ in range(calls)])
+    with torch.cuda.stream(stream):
+        g.replay()
+    torch.cuda.synchronize()
+    t = cuda_time(torch, stream, lambda: g.replay()) / calls
+    nb = w.nbytes()
+    return {"us_per_call": t * 1e6, "weight_bytes": nb, "weight_gbs_l2_warm": nb / t / 1e9}
 
 
 # ------------------------------------------------------------ cpu oracle
@@ -362,10 +421,11 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work for cpu_baseline")
     ap.add_argument("--no-details", action="store_true")
-    ap.add_argument("--profile", choices=["decode"], default=None,
+    ap.add_argument("--profile", choices=["decode", "prefill"], default=None,
                     help="plain launches without graphs or reporting (for ncu captures)")
     ap.add_argument("--experts", type=int, default=S.EXPERTS,
                     help="experts resident in --profile mode (fewer keeps ncu captures small)")
+    ap.add_argument("--tokens", type=int, default=256, help="tokens per call in --profile prefill mode")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -396,6 +456,21 @@ def main():
         with torch.cuda.stream(stream):
             for c in range(args.warmup + args.steps):
                 dec.call(c % RING)
+        torch.cuda.synchronize()
+        return 0
+    if args.profile == "prefill":
+        rng = S.rng_for(4)
+        w_ks = S.moe_weights(rng, "iq2_ks", args.experts, S.HIDDEN, S.INTER)
+        T = args.tokens
+        ids, p = S.routing(rng, T, args.experts, S.TOPK)
+        x = S.random_bf16(rng, (T, S.HIDDEN))
+        dw = [B.Weights.from_host(w, device) for w in w_ks]
+        xd = torch.from_numpy(x.view(np.int16)).to(device).view(torch.bfloat16)
+        idsd, pd = torch.from_numpy(ids).to(device), torch.from_numpy(p).to(device)
+        ws = B.workspace(B.iqk_moe_workspace_bytes(1, T, S.TOPK, args.experts, S.HIDDEN, S.INTER), device)
+        with torch.cuda.stream(stream):
+            for _ in range(args.warmup + args.steps):
+                B.iqk_moe_prefill(dw[0], dw[1], dw[2], S.value_table("int", 4), xd, idsd, pd, ws=ws, stream=stream)
         torch.cuda.synchronize()
         return 0
 
@@ -472,6 +547,11 @@ def main():
             del db, gr
         del w_k
         torch.cuda.empty_cache()
+        log("config 4 prefill")
+        details["config4_prefill"] = prefill_leg(torch, B, w_ks, values, device, stream, peaks)
+        torch.cuda.empty_cache()
+        for cfg in (0, 1):
+            details[f"config{cfg}_gemv"] = gemv_leg(torch, B, cfg, device, stream)
 
     launches = 3 * K
     line = {

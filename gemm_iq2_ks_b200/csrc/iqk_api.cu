@@ -151,6 +151,7 @@ int iqk_gemv(const iqk_weights* w, int32_t expert, const float* values, const ui
   int rc;
   if ((rc = check_weights(w, &wd)) || (rc = check_values(values, &V))) return rc;
   if (expert < 0 || expert >= wd.experts || !x || !y) return IQK_EINVAL;
+  if (!aligned(x, 16) || !aligned(y, 4)) return IQK_EINVAL;  // x is read in 16-byte groups
   if (T < 1 || T > 64) return IQK_EUNSUPPORTED;
   if ((rc = check_ws(workspace, ws_bytes, gemv_ws(T, wd.rows, wd.cols).total))) return rc;
   const int sms = num_sms();

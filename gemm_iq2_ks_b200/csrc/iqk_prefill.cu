@@ -125,6 +125,85 @@ __device__ __forceinline__ bool pf_wait(uint64_t* bar, uint32_t par, volatile ui
   return false;
 }
 
+// One producer warp's share of an (item, N tile): rows 32q .. 32q + 31 of its
+// 128-row tile, all K chunks of 64. The decode of chunk c + 1 overlaps the
+// tensor-memory store of chunk c: the store's completion is awaited (and the
+// MMA warp signalled) only after the next chunk is in registers.
+template <int FMT>
+__device__ __forceinline__ bool pf_produce(const WDev& W, int64_t grow, int nch, int tile, int q, int r, int lane,
+                                           const uint32_t* qbuf, uint64_t* qs_full, uint64_t* qs_empty,
+                                           uint64_t* a_ready, uint64_t* a_free, uint32_t tmem, const uint2* lut,
+                                           const Values& V, uint32_t& qi, uint32_t& ai, volatile uint32_t* abort_flag,
+                                           int32_t* status) {
+  const int nb = nch >> 2;
+  BlkSc<FMT> sc = load_blk<FMT>(W, grow, 0);
+  BlkSc<FMT> scn = nb > 1 ? load_blk<FMT>(W, grow, 1) : sc;  // the next 256-block, requested one block ahead
+  const uint32_t tlane = tmem + ((uint32_t)(32 * q) << 16) + TM_A + (tile ? 32u : 0u);
+  uint32_t ra[32], rb[32];
+  int pend_sa = -1;  // stage of the chunk whose store is in flight
+  // decode chunk c into regs; returns the A stage it goes to, or -1 after a failed wait
+  auto decode = [&](int c, uint32_t (&regs)[32]) -> int {
+    const int s = qi % PF_SQ;
+    if ((c & 3) == 0) {
+      if (c > 0) {
+        sc = scn;
+        if ((c >> 2) + 1 < nb) scn = load_blk<FMT>(W, grow, (c >> 2) + 1);
+      }
+      if (!pf_wait(&qs_full[s], (qi / PF_SQ) & 1, abort_flag, status)) return -1;
+    }
+    const int sa = ai % PF_SA;
+    if (!pf_wait(&a_free[sa], ((ai / PF_SA) & 1) ^ 1, abort_flag, status)) return -1;
+    // qs tiles arrive with the 64-byte swizzle: 16-byte chunk j of row r sits at chunk j ^ ((r >> 1) & 3)
+    const uint4 qw = *reinterpret_cast<const uint4*>(qbuf + (size_t)s * (PF_Q_BYTES / 4) + (tile ? 128 * 16 : 0) +
+                                                     r * 16 + 4 * ((c & 3) ^ ((r >> 1) & 3)));
+    const uint32_t qv[4] = {qw.x, qw.y, qw.z, qw.w};
+#pragma unroll
+    for (int m = 0; m < 4; m++) {
+      const uint2 tw = table_words<FMT>(sc, c & 3, m, lut, V);
+#pragma unroll
+      for (int i = 0; i < 4; i++) {
+        const Pair2 pr = lookup_slot(qv[m], i, tw.x, tw.y);
+        regs[8 * m + 2 * i] = pr.lo;
+        regs[8 * m + 2 * i + 1] = pr.hi;
+      }
+    }
+    if ((c & 3) == 3) {  // the qs stage has been read in full
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&qs_empty[s]);
+      qi++;
+    }
+    ai++;
+    return sa;
+  };
+  auto publish = [&]() {  // the pending chunk's store is complete: hand its stage to the MMA warp
+    if (pend_sa < 0) return;
+    tmem_wait_st();
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&a_ready[pend_sa]);
+  };
+  for (int c = 0; c < nch; c += 2) {
+    int sa = decode(c, ra);
+    if (sa < 0) {
+      tmem_wait_st();
+      return false;
+    }
+    publish();
+    tmem_st32(tlane + 64u * sa, ra);
+    pend_sa = sa;
+    sa = decode(c + 1, rb);
+    if (sa < 0) {
+      tmem_wait_st();
+      return false;
+    }
+    publish();
+    tmem_st32(tlane + 64u * sa, rb);
+    pend_sa = sa;
+  }
+  publish();
+  return true;
+}
+
 template <int MODE, int F0, int F1>
 __global__ void __launch_bounds__(PF_THREADS, 1) k_pf_gemm(const __grid_constant__ CUtensorMap q0,
                                                            const __grid_constant__ CUtensorMap q1,
@@ -264,83 +343,11 @@ __global__ void __launch_bounds__(PF_THREADS, 1) k_pf_gemm(const __grid_constant
       for (int n0 = 0; n0 < ne; n0 += PF_NMAX) {
         const int ncols = ((ne - n0) < PF_NMAX ? (ne - n0) : PF_NMAX);
         const int npad = (ncols + 15) & ~15;
-        bool ok = true;
-        if (tile == 0) {
-          BlkSc<F0> sc = load_blk<F0>(W, grow, 0);
-          for (int c = 0; c < nch && ok; c++) {
-            const int s = qi % PF_SQ;
-            if ((c & 3) == 0) {
-              if (c > 0) sc = load_blk<F0>(W, grow, c >> 2);
-              ok = pf_wait(&qs_full[s], (qi / PF_SQ) & 1, abort_flag, A.status);
-              if (!ok) break;
-            }
-            const int sa = ai % PF_SA;
-            ok = pf_wait(&a_free[sa], ((ai / PF_SA) & 1) ^ 1, abort_flag, A.status);
-            if (!ok) break;
-            const uint4 qw = *reinterpret_cast<const uint4*>(qbuf + (size_t)s * (PF_Q_BYTES / 4) + r * 16 + 4 * (c & 3));
-            const uint32_t qv[4] = {qw.x, qw.y, qw.z, qw.w};
-            uint32_t regs[32];
-#pragma unroll
-            for (int m = 0; m < 4; m++) {
-              const uint2 tw = table_words<F0>(sc, c & 3, m, lut, A.V);
-#pragma unroll
-              for (int i = 0; i < 4; i++) {
-                const Pair2 pr = lookup_slot(qv[m], i, tw.x, tw.y);
-                regs[8 * m + 2 * i] = pr.lo;
-                regs[8 * m + 2 * i + 1] = pr.hi;
-              }
-            }
-            tmem_st32(tmem + ((uint32_t)(32 * q) << 16) + TM_A + 64u * sa, regs);
-            tmem_wait_st();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&a_ready[sa]);
-            ai++;
-            if ((c & 3) == 3) {
-              __syncwarp();
-              if (lane == 0) mbar_arrive(&qs_empty[s]);
-              qi++;
-            }
-          }
-        } else {
-          BlkSc<F1> sc = load_blk<F1>(W, grow, 0);
-          for (int c = 0; c < nch && ok; c++) {
-            const int s = qi % PF_SQ;
-            if ((c & 3) == 0) {
-              if (c > 0) sc = load_blk<F1>(W, grow, c >> 2);
-              ok = pf_wait(&qs_full[s], (qi / PF_SQ) & 1, abort_flag, A.status);
-              if (!ok) break;
-            }
-            const int sa = ai % PF_SA;
-            ok = pf_wait(&a_free[sa], ((ai / PF_SA) & 1) ^ 1, abort_flag, A.status);
-            if (!ok) break;
-            const uint4 qw =
-                *reinterpret_cast<const uint4*>(qbuf + (size_t)s * (PF_Q_BYTES / 4) + 128 * 16 + r * 16 + 4 * (c & 3));
-            const uint32_t qv[4] = {qw.x, qw.y, qw.z, qw.w};
-            uint32_t regs[32];
-#pragma unroll
-            for (int m = 0; m < 4; m++) {
-              const uint2 tw = table_words<F1>(sc, c & 3, m, lut, A.V);
-#pragma unroll
-              for (int i = 0; i < 4; i++) {
-                const Pair2 pr = lookup_slot(qv[m], i, tw.x, tw.y);
-                regs[8 * m + 2 * i] = pr.lo;
-                regs[8 * m + 2 * i + 1] = pr.hi;
-              }
-            }
-            tmem_st32(tmem + ((uint32_t)(32 * q) << 16) + TM_A + 64u * sa + 32u, regs);
-            tmem_wait_st();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&a_ready[sa]);
-            ai++;
-            if ((c & 3) == 3) {
-              __syncwarp();
-              if (lane == 0) mbar_arrive(&qs_empty[s]);
-              qi++;
-            }
-          }
-        }
+        const bool ok = tile == 0
+                            ? pf_produce<F0>(W, grow, nch, tile, q, r, lane, qbuf, qs_full, qs_empty, a_ready, a_free, tmem,
+                                             lut, A.V, qi, ai, abort_flag, A.status)
+                            : pf_produce<F1>(W, grow, nch, tile, q, r, lane, qbuf, qs_full, qs_empty, a_ready, a_free, tmem,
+                                             lut, A.V, qi, ai, abort_flag, A.status);
         if (!ok) break;
         // ---- epilogue of this (item, N tile)
         if (!pf_wait(d_full, di & 1, abort_flag, A.status)) break;
@@ -502,7 +509,7 @@ static int make_qs_tile_map(CUtensorMap* map, const WDev& w) {
   const cuuint32_t box[2] = {16, 128};
   const cuuint32_t estr[2] = {1, 1};
   CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<uint32_t*>(w.qs), dims, strides, box, estr,
-                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? 0 : -4;
 }

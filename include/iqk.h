@@ -123,7 +123,8 @@ int iqk_dequant_bf16(const iqk_weights* w, int32_t expert, const float* values /
  * iqk_gemv -- y[t][o] = sum_k w[o][k] * x[t][k] for one expert, t < T.
  * Defines: the fused decode GEMV of the page's "Surface" section (few
  * token-expert pairs, one pass over the reduction axis).
- * x: device bf16 [T][cols]; y: device float32 [T][rows]; 1 <= T <= 64.
+ * x: device bf16 [T][cols], 16-byte aligned; y: device float32 [T][rows];
+ * 1 <= T <= 64. A misaligned x returns IQK_EINVAL.
  * Accuracy: |y - y_exact| <= 2e-3 * sum_k |w[o][k] * x[t][k]| (weights enter the
  * tensor-core reduction as bfloat16 of (scale_index * value) with d applied
  * in float32; float32 accumulation).

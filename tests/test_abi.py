@@ -63,6 +63,7 @@ def test_host_validation_rejects_before_any_launch():
     assert L.iqk_gemv(ctypes.byref(w), 0, P, 4096, 65, 4096, 4096, 1 << 20, None) == B.IQK_EUNSUPPORTED
     assert L.iqk_gemv(ctypes.byref(w), 0, P, 4096, 1, 4096, None, 0, None) == B.IQK_EWORKSPACE
     assert L.iqk_gemv(ctypes.byref(w), 0, P, 4096, 1, 4096, 4097, 1 << 20, None) == B.IQK_EWORKSPACE
+    assert L.iqk_gemv(ctypes.byref(w), 0, P, 4098, 1, 4096, 4096, 1 << 20, None) == B.IQK_EINVAL  # x misaligned
 
 
 def test_moe_shape_checks():
