@@ -21,7 +21,7 @@ FMT = {"iq2_ks": 0, "iq2_k": 1}
 
 EXPORTS = (
     "iqk_strerror", "iqk_last_cuda_error", "iqk_version", "iqk_row_bytes",
-    "iqk_dequant", "iqk_dequant_bf16", "iqk_gemv_workspace_bytes", "iqk_gemv",
+    "iqk_dequant", "iqk_dequant_bf16", "iqk_gemv_workspace_bytes", "iqk_gemv", "iqk_gemv_static",
     "iqk_moe_workspace_bytes", "iqk_moe_decode", "iqk_moe_prefill", "iqk_moe_status",
     "iqk_route_workspace_bytes", "iqk_moe_route", "iqk_floor",
 )
@@ -61,6 +61,7 @@ def lib(build_if_missing: bool = True) -> ctypes.CDLL:
             "iqk_dequant_bf16": (ctypes.c_int, [W, i32, vp, vp, vp]),
             "iqk_gemv_workspace_bytes": (sz, [i32, i32, i32]),
             "iqk_gemv": (ctypes.c_int, [W, i32, vp, vp, i32, vp, vp, sz, vp]),
+            "iqk_gemv_static": (ctypes.c_int, [W, i32, vp, vp, i32, vp, vp]),
             "iqk_moe_workspace_bytes": (sz, [i32, i32, i32, i32, i32, i32]),
             "iqk_moe_decode": (ctypes.c_int, [W, W, W, vp, vp, i32, vp, vp, i32, vp, vp, sz, vp]),
             "iqk_moe_prefill": (ctypes.c_int, [W, W, W, vp, vp, i32, vp, vp, i32, vp, vp, sz, vp]),
@@ -189,6 +190,17 @@ def iqk_gemv(w: Weights, expert: int, values, x, y=None, ws=None, stream=None):
     v = _values(values)
     _check(lib().iqk_gemv(ctypes.byref(w.c), expert, v.ctypes.data, x.data_ptr(), T, y.data_ptr(), ws.data_ptr(),
                           ws.numel(), _stream(stream)), "iqk_gemv")
+    return y
+
+
+def iqk_gemv_static(w: Weights, expert: int, values, x, y=None, stream=None):
+    """iqk_gemv with the library's static scratch (no workspace argument)."""
+    torch = _torch()
+    T = x.shape[0]
+    y = _empty((T, w.rows), torch.float32, x.device) if y is None else y
+    v = _values(values)
+    _check(lib().iqk_gemv_static(ctypes.byref(w.c), expert, v.ctypes.data, x.data_ptr(), T, y.data_ptr(),
+                                 _stream(stream)), "iqk_gemv_static")
     return y
 
 

@@ -136,6 +136,23 @@ int iqk_gemv(const iqk_weights* w, int32_t expert, const float* values /* host [
              void* stream);
 
 /*
+ * iqk_gemv_static -- iqk_gemv without a workspace argument (the pages have no
+ * counterpart; this is a convenience of this library). The scratch is a
+ * file-scope device array of IQK_GEMV_STATIC_SCRATCH_BYTES (4 MiB) in each
+ * device context, so the call allocates nothing; it is for callers that
+ * cannot allocate device memory at the call site (a plain C host linking only
+ * this library, or a code path that must not enter an allocator).
+ * A shape whose scratch (iqk_gemv_workspace_bytes) exceeds the array returns
+ * IQK_EWORKSPACE; the first call on a device looks the array up with
+ * cudaGetSymbolAddress, so make it before capturing a stream that records the
+ * call. Calls overlapping in time on one device share the array and race:
+ * serialise them. Arguments and accuracy as iqk_gemv.
+ */
+#define IQK_GEMV_STATIC_SCRATCH_BYTES (4u << 20)
+int iqk_gemv_static(const iqk_weights* w, int32_t expert, const float* values /* host [8] */,
+                    const uint16_t* x, int32_t T, float* y, void* stream);
+
+/*
  * Routed-expert block (gate/up GEMV, SwiGLU, down GEMV, weighted combine).
  * Geometry on the page: 256 experts, six selected, gate and up [2048 x 4096],
  * down [4096 x 2048]; any experts >= 1, hidden and inter multiples of 256.
