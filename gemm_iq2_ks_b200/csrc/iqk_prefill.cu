@@ -10,8 +10,9 @@
 // its A operand.
 //
 // Launch sequence: grouping (iqk_route.cu) -> gather of token rows in expert
-// order -> gate/up grouped GEMM with SwiGLU epilogue -> down grouped GEMM with
-// routing-weight epilogue -> per-token combine in slot order.
+// order -> gate/up grouped GEMM with SwiGLU epilogue -> down grouped GEMM
+// (row scale in the epilogue) -> per-token combine, routing-weighted, in slot
+// order.
 #include <algorithm>
 
 #include "iqk_device.cuh"
@@ -20,10 +21,11 @@
 
 namespace iqk {
 
-constexpr int PF_WARPS = 10;
+constexpr int PF_WARPS = 11;
 constexpr int PF_THREADS = PF_WARPS * 32;
-constexpr int PF_TMA_WARP = 8;
+constexpr int PF_TMA_WARP = 8;   // qs tiles
 constexpr int PF_MMA_WARP = 9;
+constexpr int PF_BTMA_WARP = 10;  // token rows (B operand)
 constexpr int PF_SA = 4;      // A stages in tensor memory (64 k each)
 constexpr int PF_SB = 4;      // B stages in shared memory (64 k each)
 constexpr int PF_SQ = 3;      // qs stages in shared memory (256 k each)
@@ -257,12 +259,12 @@ __global__ void __launch_bounds__(PF_THREADS, 1) k_pf_gemm(const __grid_constant
   const int nitems = A.E * A.mtiles;
   const int nch = A.K / 64;
 
-  if (warp == PF_TMA_WARP) {
+  if (warp == PF_TMA_WARP) {  // qs tiles, one 256-block ahead of the producers per stage
     if (lane == 0) {
-      uint32_t qi = 0, bi = 0;
+      uint32_t qi = 0;
       for (int item = blockIdx.x; item < nitems && !*abort_flag; item += gridDim.x) {
         const int e = item / A.mtiles, mt = item % A.mtiles;
-        const int ne = A.counts[e], off = A.offsets[e];
+        const int ne = A.counts[e];
         int r0, r1;
         if (MODE == 0) {
           r0 = e * A.rows + 128 * mt;
@@ -271,20 +273,32 @@ __global__ void __launch_bounds__(PF_THREADS, 1) k_pf_gemm(const __grid_constant
           r0 = e * A.rows + 256 * mt;
           r1 = r0 + 128;
         }
-        for (int n0 = 0; n0 < ne; n0 += PF_NMAX) {
+        bool ok = true;
+        for (int n0 = 0; n0 < ne && ok; n0 += PF_NMAX) {
+          for (int c = 0; c < nch; c += 4) {
+            const int s = qi % PF_SQ;
+            if (!(ok = pf_wait(&qs_empty[s], ((qi / PF_SQ) & 1) ^ 1, abort_flag, A.status))) break;
+            uint32_t* dst = qbuf + (size_t)s * (PF_Q_BYTES / 4);
+            mbar_arrive_expect_tx(&qs_full[s], PF_Q_BYTES);
+            tma_load_2d(dst, &q0, (c >> 2) * 16, r0, &qs_full[s]);
+            tma_load_2d(dst + 128 * 16, &q1, (c >> 2) * 16, r1, &qs_full[s]);
+            qi++;
+          }
+        }
+      }
+    }
+  } else if (warp == PF_BTMA_WARP) {  // token rows of each K chunk
+    if (lane == 0) {
+      uint32_t bi = 0;
+      for (int item = blockIdx.x; item < nitems && !*abort_flag; item += gridDim.x) {
+        const int e = item / A.mtiles;
+        const int ne = A.counts[e], off = A.offsets[e];
+        bool ok = true;
+        for (int n0 = 0; n0 < ne && ok; n0 += PF_NMAX) {
           const int npad = (((ne - n0) < PF_NMAX ? (ne - n0) : PF_NMAX) + 15) & ~15;
           for (int c = 0; c < nch; c++) {
-            if ((c & 3) == 0) {
-              const int s = qi % PF_SQ;
-              if (!pf_wait(&qs_empty[s], ((qi / PF_SQ) & 1) ^ 1, abort_flag, A.status)) break;
-              uint32_t* dst = qbuf + (size_t)s * (PF_Q_BYTES / 4);
-              mbar_arrive_expect_tx(&qs_full[s], PF_Q_BYTES);
-              tma_load_2d(dst, &q0, (c >> 2) * 16, r0, &qs_full[s]);
-              tma_load_2d(dst + 128 * 16, &q1, (c >> 2) * 16, r1, &qs_full[s]);
-              qi++;
-            }
             const int s = bi % PF_SB;
-            if (!pf_wait(&b_empty[s], ((bi / PF_SB) & 1) ^ 1, abort_flag, A.status)) break;
+            if (!(ok = pf_wait(&b_empty[s], ((bi / PF_SB) & 1) ^ 1, abort_flag, A.status))) break;
             uint8_t* dst = bbuf + (size_t)s * PF_B_BYTES;
             mbar_arrive_expect_tx(&b_full[s], (uint32_t)npad * 128);
             for (int bx = 0; bx < npad / 16; bx++)
@@ -384,11 +398,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1) k_pf_gemm(const __grid_constant
 #pragma unroll
             for (int i = 0; i < 8; i++) {
               const int n = c0 + i;
-              if (n < ncols) {
-                const int pos = off + n0 + n;
-                const float pv = __ldg(A.p + __ldg(A.perm + pos));
-                A.outp[(size_t)pos * H + o] = v8[i] * dr * pv;
-              }
+              if (n < ncols) A.outp[(size_t)(off + n0 + n) * H + o] = v8[i] * dr;
             }
           }
         }
@@ -438,7 +448,8 @@ __global__ void __launch_bounds__(256) k_pf_gather(const uint16_t* __restrict__ 
 
 // y[t][o] = bf16(sum over slots j in order of outp[inv[t*topk + j]][o]).
 __global__ void __launch_bounds__(256) k_pf_combine(const float* __restrict__ outp, const int32_t* __restrict__ inv,
-                                                    int T, int topk, int H, uint16_t* __restrict__ y) {
+                                                    const float* __restrict__ p, int T, int topk, int H,
+                                                    uint16_t* __restrict__ y) {
   const int64_t n = (int64_t)T * (H / 4);
   for (int64_t g = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; g < n; g += (int64_t)gridDim.x * blockDim.x) {
     const int t = (int)(g / (H / 4)), o4 = (int)(g % (H / 4));
@@ -446,11 +457,12 @@ __global__ void __launch_bounds__(256) k_pf_combine(const float* __restrict__ ou
     for (int j = 0; j < topk; j++) {
       const int pos = inv[t * topk + j];
       if (pos < 0) continue;
+      const float pw = __ldg(p + t * topk + j);
       const float4 v = __ldg(reinterpret_cast<const float4*>(outp + (size_t)pos * H) + o4);
-      s.x += v.x;
-      s.y += v.y;
-      s.z += v.z;
-      s.w += v.w;
+      s.x += pw * v.x;
+      s.y += pw * v.y;
+      s.z += pw * v.z;
+      s.w += pw * v.w;
     }
     uint2 out;
     out.x = pack_bf16x2(s.x, s.y);
@@ -590,7 +602,7 @@ int launch_moe_prefill(const WDev& g, int fg, const WDev& u, int fu, const WDev&
   {
     const int64_t n = (int64_t)T * (H / 4);
     const int blocks = (int)std::min<int64_t>((n + 255) / 256, (int64_t)num_sms * 16);
-    k_pf_combine<<<std::max(blocks, 1), 256, 0, st>>>(outp, inv, T, topk, H, y);
+    k_pf_combine<<<std::max(blocks, 1), 256, 0, st>>>(outp, inv, p, T, topk, H, y);
   }
   return cudaGetLastError() == cudaSuccess ? 0 : -4;
 }
