@@ -35,6 +35,12 @@ METRIC = "MoE decode µs/token & weight GB/s vs HBM floor; prefill bf16 TFLOP/s"
 RING = 420  # calls per captured graph (10 permutation cycles of 42 calls)
 
 
+# DRAM bytes (read + write) of the two tile kernels of one config-2 decode
+# call, from one ncu capture of `bench.py --profile decode --experts 24`
+# (profiles/decode_config2_tile_kernels.md); per call, not per resident expert.
+DECODE_CALL_TRAFFIC = 41_550_592
+
+
 def env_int(k, d):
     try:
         return int(os.environ.get(k, d))
@@ -562,7 +568,7 @@ def main():
         "floor": {"us_per_token": floor_us, "decode_over_floor": us_per_token / floor_us if world == 1 else
                   (t / K * 1e6) / floor_us},
         "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                     "frac": gbs / peaks["hbm_gbs"], "traffic": None,
+                     "frac": gbs / peaks["hbm_gbs"], "traffic": DECODE_CALL_TRAFFIC,
                      "kernel": "one decode call (prep + gate/up+SwiGLU + down+combine, PDL-chained)",
                      "peak_source": peaks["source"] + " hbm_gbs (copy)"},
         "e2e": {"value": e2e_us, "unit": "us/token", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
