@@ -52,18 +52,23 @@ Chunking chunking(int rows, int cols) {
 
 // ---------------------------------------------------------- item scales
 // An item's scale slice (16 rows x bpi blocks) sits in a per-stage slot:
-//   IQ2_KS: scl [16][bpi] u32 | sch [16][4] u8 | sex [16][4] u8
+//   IQ2_KS: scl [16][bpi] u32 | sch [16][4] u8 | sex [16][4] u8 | dv [16] u16
 //   IQ2_K:  scl [16][2 bpi] u32 | sex [16][bpi] u16 | dv [16][bpi] u16
 // Every part starts on a 16-byte boundary (bpi = 1, 2 or 4). An IQ2_KS row of
 // sch / sex holds the aligned 4-byte window around the slice's bpi bytes
-// (cp.async copies 4 bytes at least); the slice starts `o` bytes into it. The
-// IQ2_KS row scale is read straight from global memory at the start of the item.
+// (cp.async copies 4 bytes at least); the slice starts `o` bytes into it.
 template <int FMT>
 struct Slot {
   static __host__ __device__ __forceinline__ uint32_t b_off(int bpi) { return FMT == FMT_KS ? 64u * bpi : 128u * bpi; }
   static __host__ __device__ __forceinline__ uint32_t c_off(int bpi) { return FMT == FMT_KS ? 64u * bpi + 64u : 160u * bpi; }
-  static __host__ __device__ __forceinline__ uint32_t bytes(int bpi) { return FMT == FMT_KS ? 64u * bpi + 128u : 192u * bpi; }
+  static __host__ __device__ __forceinline__ uint32_t dv_off(int bpi) { return 64u * bpi + 128u; }  // IQ2_KS
+  static __host__ __device__ __forceinline__ uint32_t bytes(int bpi) { return FMT == FMT_KS ? 64u * bpi + 160u : 192u * bpi; }
 };
+
+// IQ2_KS row scale of slot row r (zero past the tile's last row).
+__device__ __forceinline__ float d_smem_ks(const uint8_t* slot, int bpi, int r) {
+  return __half2float(__ushort_as_half(reinterpret_cast<const uint16_t*>(slot + Slot<FMT_KS>::dv_off(bpi))[r]));
+}
 
 // Bytes between consecutive slots: the larger format's slot, rounded up to
 // 128 so that every ring stage and slot keeps a 128-byte aligned base.
@@ -455,6 +460,14 @@ __device__ __forceinline__ void stage_scales(uint8_t* slot, const WDev& w, int64
         else cp_async4(dst, src);
       }
     }
+    if (FMT == FMT_KS) {  // the tile's 16 row scales: two 16-byte copies, or plain loads off the grid
+      uint16_t* sdv = reinterpret_cast<uint16_t*>(slot + Slot<FMT>::dv_off(bpi));
+      if (valid == kTile && ((reinterpret_cast<uintptr_t>(w.dv + R0) & 15) == 0)) {
+        if (lane < 2) cp_async16(sdv + 8 * lane, w.dv + R0 + 8 * lane);
+      } else if (lane < kTile) {
+        sdv[lane] = lane < valid ? __ldg(w.dv + R0 + lane) : (uint16_t)0;
+      }
+    }
     cp_async_arrive(bar);
     return;
   }
@@ -472,6 +485,8 @@ __device__ __forceinline__ void stage_scales(uint8_t* slot, const WDev& w, int64
       sb[4 * r + b] = r < valid ? __ldg(w.sch + o) : (uint8_t)0;
       sc[4 * r + b] = r < valid ? __ldg(reinterpret_cast<const uint8_t*>(w.sex) + o) : (uint8_t)0;
     }
+    uint16_t* sdv = reinterpret_cast<uint16_t*>(slot + Slot<FMT>::dv_off(bpi));
+    if (lane < kTile) sdv[lane] = lane < valid ? __ldg(w.dv + R0 + lane) : (uint16_t)0;
   } else {
     uint32_t* d32 = reinterpret_cast<uint32_t*>(slot);
     for (int i = lane; i < 32 * bpi; i += 32) {
@@ -631,9 +646,6 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, kDecodeMinBlocks(NT)) k_str
     if (id >= nitems) break;
     int u, mat, tile, s;
     item_of(id, u, mat, tile, s);
-    const int e = expert_of(u);
-    const int64_t R0 = (int64_t)e * rows + (int64_t)tile * kTile;
-    const int valid = min(kTile, rows - tile * kTile);
     int p0 = 0, ncols = A.T;
     if (MODE == MODE_GATEUP || MODE == MODE_DOWN) {
       p0 = rt.ustart[u];
@@ -653,13 +665,6 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, kDecodeMinBlocks(NT)) k_str
     }
     const bool fmt0 = (MODE != MODE_GATEUP) || mat == 0;
     const bool kfmt = fmt0 ? (F0 == FMT_K) : (F1 == FMT_K);
-    // IQ2_KS row scales of rows g and g + 8, applied after the slice's MMAs
-    float dg = 0.f, dh = 0.f;
-    if (MODE != MODE_FLOOR && !kfmt) {
-      const uint16_t* dv = fmt0 ? A.w0.dv : A.w1.dv;
-      if (g < valid) dg = __half2float(__ushort_as_half(__ldg(dv + R0 + g)));
-      if (g + 8 < valid) dh = __half2float(__ushort_as_half(__ldg(dv + R0 + g + 8)));
-    }
     const int st = it % kStages;
     if (!mbar_wait_bounded(&bar[st], (uint32_t)((it / kStages) & 1))) {
       if (!waited) griddep_wait();
@@ -701,9 +706,10 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, kDecodeMinBlocks(NT)) k_str
           xg ^= ((uint32_t)sb[g * 4 + o + i] ^ (uint32_t)sc[g * 4 + o + i]) << sh;
           xh ^= ((uint32_t)sb[(g + 8) * 4 + o + i] ^ (uint32_t)sc[(g + 8) * 4 + o + i]) << sh;
         }
-        if (s == 0 && t == 0) {  // the row scale belongs to the first slice
-          if (g < valid) xg ^= __ldg(A.w0.dv + R0 + g);
-          if (g + 8 < valid) xh ^= __ldg(A.w0.dv + R0 + g + 8);
+        if (s == 0 && t == 0) {  // the row scale belongs to the first slice (zero past the last row)
+          const uint16_t* sdv = reinterpret_cast<const uint16_t*>(slot + Slot<FMT_KS>::dv_off(bpi));
+          xg ^= sdv[g];
+          xh ^= sdv[g + 8];
         }
       } else {
         const uint16_t* sb = reinterpret_cast<const uint16_t*>(slot + Slot<FMT_K>::b_off(bpi));
@@ -716,6 +722,8 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, kDecodeMinBlocks(NT)) k_str
       }
     } else {
       const int o = A.async_sc ? (s * bpi) & 3 : 0;
+      // IQ2_KS row scales of rows g and g + 8, applied after the slice's MMAs
+      const float dg = kfmt ? 0.f : d_smem_ks(slot, bpi, g), dh = kfmt ? 0.f : d_smem_ks(slot, bpi, g + 8);
       item_mma<F0, F1, NT, BSM>(sq, slot, bpi, o, ldw, bsrc, fmt0, kfmt, lut0, lut1, dg, dh, g, t, k65536, acc);
     }
     __syncwarp();
@@ -1010,8 +1018,6 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, kDecodeMinBlocks(NT)) k_til
     for (int k = 0; k < cnt_w; k++, q++) {
       int u, mat, tile, s;
       item_at(q, u, mat, tile, s);
-      const int64_t R0 = (int64_t)rt.uexp[u] * rows + (int64_t)tile * kTile;
-      const int valid = min(kTile, rows - tile * kTile);
       const int p0 = rt.ustart[u];
       const int ncols = rt.ustart[u + 1] - p0;
       const uint16_t* bsrc[NT];
@@ -1026,12 +1032,6 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, kDecodeMinBlocks(NT)) k_til
       }
       const bool fmt0 = (MODE != MODE_GATEUP) || mat == 0;
       const bool kfmt = fmt0 ? (F0 == FMT_K) : (F1 == FMT_K);
-      float dg = 0.f, dh = 0.f;
-      if (!kfmt) {
-        const uint16_t* dv = fmt0 ? A.w0.dv : A.w1.dv;
-        if (g < valid) dg = __half2float(__ushort_as_half(__ldg(dv + R0 + g)));
-        if (g + 8 < valid) dh = __half2float(__ushort_as_half(__ldg(dv + R0 + g + 8)));
-      }
       float acc[NT][4];
 #pragma unroll
       for (int n = 0; n < NT; n++)
@@ -1051,6 +1051,7 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, kDecodeMinBlocks(NT)) k_til
         const uint32_t* sq = ring_qs + (size_t)st * stage_words;
         const uint8_t* slot = ring_slots + (size_t)st * slot_b;
         const int o = A.async_sc ? (s * bpi) & 3 : 0;
+        const float dg = kfmt ? 0.f : d_smem_ks(slot, bpi, g), dh = kfmt ? 0.f : d_smem_ks(slot, bpi, g + 8);
         item_mma<F0, F1, NT, BSM>(sq, slot, bpi, o, ldw, bsrc, fmt0, kfmt, lut0, lut1, dg, dh, g, t, k65536, acc);
         __syncwarp();
         issue(q + kStages);  // refill the stage just consumed
