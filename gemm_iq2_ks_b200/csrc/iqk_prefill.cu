@@ -26,12 +26,17 @@ constexpr int PF_THREADS = PF_WARPS * 32;
 constexpr int PF_TMA_WARP = 8;   // qs tiles
 constexpr int PF_MMA_WARP = 9;
 constexpr int PF_BTMA_WARP = 10;  // token rows (B operand)
-constexpr int PF_SA = 4;      // A stages in tensor memory (64 k each)
+constexpr int PF_SA = 2;      // A stages in tensor memory (64 k each)
 constexpr int PF_SB = 4;      // B stages in shared memory (64 k each)
 constexpr int PF_SQ = 3;      // qs stages in shared memory (256 k each)
-constexpr int PF_NMAX = 128;  // pairs per N tile
-constexpr uint32_t TM_D0 = 0, TM_D1 = 128, TM_A = 256;
-constexpr int PF_B_BYTES = PF_NMAX * 128;       // one B stage: 128 rows x 64 bf16
+// Two CTAs share an SM, each with half of tensor memory (256 columns): two
+// 64-column accumulators (pairs per N tile <= 64) and two A stages. The two
+// CTAs' pipelines interleave, which hides the long round trip of an A stage
+// (decode, store, signal, MMA, commit) better than one deeper pipeline.
+constexpr int PF_NMAX = 64;  // pairs per N tile
+constexpr uint32_t TM_COLS = 256;
+constexpr uint32_t TM_D0 = 0, TM_D1 = 64, TM_A = 128;
+constexpr int PF_B_BYTES = PF_NMAX * 128;       // one B stage: 64 rows x 64 bf16
 constexpr int PF_Q_BYTES = 2 * 128 * 16 * 4;    // one qs stage: two 128-row tiles x 16 words
 constexpr int PF_NBAR = 2 * PF_SQ + 2 * PF_SB + 2 * PF_SA + 2;
 constexpr size_t PF_SMEM = (size_t)PF_SB * PF_B_BYTES + (size_t)PF_SQ * PF_Q_BYTES + PF_NBAR * 8 + 2 * 64 * 8 + 64 +
@@ -207,7 +212,7 @@ __device__ __forceinline__ bool pf_produce(const WDev& W, int64_t grow, int nch,
 }
 
 template <int MODE, int F0, int F1>
-__global__ void __launch_bounds__(PF_THREADS, 1) k_pf_gemm(const __grid_constant__ CUtensorMap q0,
+__global__ void __launch_bounds__(PF_THREADS, 2) k_pf_gemm(const __grid_constant__ CUtensorMap q0,
                                                            const __grid_constant__ CUtensorMap q1,
                                                            const __grid_constant__ CUtensorMap bmap,
                                                            const __grid_constant__ PfArgs A) {
@@ -250,7 +255,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1) k_pf_gemm(const __grid_constant
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == PF_MMA_WARP) tmem_alloc(tmem_holder, 512);
+  if (warp == PF_MMA_WARP) tmem_alloc(tmem_holder, TM_COLS);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -412,7 +417,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1) k_pf_gemm(const __grid_constant
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == PF_MMA_WARP) tmem_dealloc(tmem, 512);
+  if (warp == PF_MMA_WARP) tmem_dealloc(tmem, TM_COLS);
 }
 
 // ------------------------------------------------ gather, combine, sizing
@@ -535,7 +540,7 @@ static int launch_gemm(const CUtensorMap& m0, const CUtensorMap& m1, const CUten
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)PF_SMEM) != cudaSuccess) return -4;
     attr = true;
   }
-  const int grid = std::max(1, std::min(num_sms, a.E * a.mtiles));
+  const int grid = std::max(1, std::min(2 * num_sms, a.E * a.mtiles));
   kern<<<grid, PF_THREADS, PF_SMEM, st>>>(m0, m1, mb, a);
   return cudaGetLastError() == cudaSuccess ? 0 : -4;
 }
