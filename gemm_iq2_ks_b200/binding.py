@@ -24,6 +24,7 @@ EXPORTS = (
     "iqk_dequant", "iqk_dequant_bf16", "iqk_gemv_workspace_bytes", "iqk_gemv", "iqk_gemv_static",
     "iqk_moe_workspace_bytes", "iqk_moe_decode", "iqk_moe_prefill", "iqk_moe_status",
     "iqk_route_workspace_bytes", "iqk_moe_route", "iqk_floor",
+    "iqk_switch_linear_workspace_bytes", "iqk_switch_linear",
 )
 
 
@@ -69,6 +70,8 @@ def lib(build_if_missing: bool = True) -> ctypes.CDLL:
             "iqk_route_workspace_bytes": (sz, [i32, i32, i32]),
             "iqk_moe_route": (ctypes.c_int, [vp, i32, i32, i32, vp, vp, vp, vp, sz, vp]),
             "iqk_floor": (ctypes.c_int, [W, vp, i32, vp, vp]),
+            "iqk_switch_linear_workspace_bytes": (sz, [i32, i32, i32, i32, i32, i32]),
+            "iqk_switch_linear": (ctypes.c_int, [W, vp, vp, i32, vp, i32, vp, i32, vp, sz, vp]),
         }
         for name, (res, args) in sig.items():
             f = getattr(L, name)
@@ -201,6 +204,27 @@ def iqk_gemv_static(w: Weights, expert: int, values, x, y=None, stream=None):
     v = _values(values)
     _check(lib().iqk_gemv_static(ctypes.byref(w.c), expert, v.ctypes.data, x.data_ptr(), T, y.data_ptr(),
                                  _stream(stream)), "iqk_gemv_static")
+    return y
+
+
+def iqk_switch_linear_workspace_bytes(mode: int, T: int, topk: int, experts: int, rows: int, cols: int) -> int:
+    return lib().iqk_switch_linear_workspace_bytes(mode, T, topk, experts, rows, cols)
+
+
+def iqk_switch_linear(w: Weights, values, x, ids, mode: int = 0, y=None, ws=None, stream=None):
+    """y[t, j] = W_{ids[t, j]} x[t] (float32 [T, topk, rows])."""
+    torch = _torch()
+    T, topk = ids.shape
+    y = _empty((T, topk, w.rows), torch.float32, x.device) if y is None else y
+    if ws is None:
+        need = iqk_switch_linear_workspace_bytes(mode, T, topk, w.experts, w.rows, w.cols)
+        if need == 0:
+            raise RuntimeError("iqk_switch_linear: the mode cannot take this shape")
+        ws = workspace(need, x.device)
+    v = _values(values)
+    _check(lib().iqk_switch_linear(ctypes.byref(w.c), v.ctypes.data, x.data_ptr(), T, ids.data_ptr(), topk,
+                                   y.data_ptr(), mode, ws.data_ptr(), ws.numel(), _stream(stream)),
+           "iqk_switch_linear")
     return y
 
 

@@ -252,6 +252,63 @@ int iqk_floor(const iqk_weights* w, const int32_t* expert_list, int32_t n_expert
 
 }  // extern "C"
 
+// ------------------------------------------------------------ switch linear
+namespace {
+// Pair count at or below which the auto mode takes the decode-style kernel.
+constexpr int kSwitchDecodeMaxPairs = IQK_SWITCH_DECODE_MAX_PAIRS;
+
+bool switch_decode_ok(int T, int topk) { return T <= 64 && T * topk <= kMaxPairs; }
+bool switch_gemm_ok(const WDev& w, int T) { return w.rows % 256 == 0 && T <= 65536; }
+
+int switch_pick(int mode, const WDev& w, int T, int topk) {
+  const bool dec = switch_decode_ok(T, topk), gem = switch_gemm_ok(w, T);
+  if (mode == 1) return dec ? 1 : -1;
+  if (mode == 2) return gem ? 2 : -1;
+  if (mode != 0) return -2;
+  if (dec && (T * topk <= kSwitchDecodeMaxPairs || !gem)) return 1;
+  return gem ? 2 : -1;
+}
+}  // namespace
+
+extern "C" size_t iqk_switch_linear_workspace_bytes(int32_t mode, int32_t T, int32_t topk, int32_t experts,
+                                                    int32_t rows, int32_t cols) {
+  if (T < 1 || topk < 1 || topk > 16 || experts < 1 || rows < 1 || cols <= 0 || cols % 256) return 0;
+  WDev w = {};
+  w.rows = rows;
+  w.cols = cols;
+  w.experts = experts;
+  const int pick = switch_pick(mode, w, T, topk);
+  if (pick == 1) return switch_ws(T, topk, experts, rows, cols).total;
+  if (pick == 2) return switch_gemm_ws(T, topk, experts, rows, cols);
+  return 0;
+}
+
+extern "C" int iqk_switch_linear(const iqk_weights* w, const float* values, const uint16_t* x, int32_t T,
+                                 const int32_t* ids, int32_t topk, float* y, int32_t mode, void* workspace,
+                                 size_t ws_bytes, void* stream) {
+  WDev wd;
+  Values V;
+  int rc;
+  if ((rc = check_weights(w, &wd)) || (rc = check_values(values, &V))) return rc;
+  if (!x || !ids || !y || !aligned(x, 16) || !aligned(y, 16)) return IQK_EINVAL;
+  if (topk < 1 || topk > 16) return IQK_EINVAL;
+  if (T == 0) return IQK_OK;
+  if (T < 0) return IQK_EINVAL;
+  const int pick = switch_pick(mode, wd, T, topk);
+  if (pick == -2) return IQK_EINVAL;
+  if (pick < 0) return IQK_EUNSUPPORTED;
+  const size_t need =
+      pick == 1 ? switch_ws(T, topk, wd.experts, wd.rows, wd.cols).total : switch_gemm_ws(T, topk, wd.experts, wd.rows, wd.cols);
+  if ((rc = check_ws(workspace, ws_bytes, need))) return rc;
+  const int sms = num_sms();
+  if (sms < 0) return cuda_fail(cudaGetLastError());
+  if (pick == 1)
+    return from_launch(launch_switch_decode(wd, w->fmt, V, x, T, ids, topk, y, (char*)workspace, (cudaStream_t)stream,
+                                            sms));
+  return from_launch(
+      launch_switch_gemm(wd, w->fmt, V, x, T, ids, topk, y, (char*)workspace, (cudaStream_t)stream, sms));
+}
+
 // ------------------------------------------------------- no-allocation GEMV
 // iqk_gemv_static runs the same launches as iqk_gemv, with its scratch in a
 // file-scope device array instead of a caller-provided workspace. The array

@@ -389,7 +389,9 @@ __global__ void __launch_bounds__(256) k_prep(const uint16_t* __restrict__ x, in
 //           token's slots in slot order, weighted by p, into y (bf16).
 //   FLOOR:  identical loads; the decode is replaced by an XOR of every loaded
 //           byte into out[expert][row].
-enum : int { MODE_GEMV = 0, MODE_GATEUP = 1, MODE_DOWN = 2, MODE_FLOOR = 3 };
+//   SWITCH: one projection per (token, slot) pair, no combine: the tile's
+//           last item writes y[pair][row] = sum over slices (fp32).
+enum : int { MODE_GEMV = 0, MODE_GATEUP = 1, MODE_DOWN = 2, MODE_FLOOR = 3, MODE_SWITCH = 4 };
 
 struct UnitArgs {
   WDev w0, w1;
@@ -545,7 +547,7 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, kDecodeMinBlocks(NT)) k_str
   }
   RouteView rt{};
   int D = 1;
-  if (MODE == MODE_GATEUP || MODE == MODE_DOWN) {
+  if (MODE == MODE_GATEUP || MODE == MODE_DOWN || MODE == MODE_SWITCH) {
     rt = carve_route(route_p, npairs);
     build_route(A.ids, npairs, A.w0.experts, rt);  // ends with __syncthreads
     D = rt.scalars[0];
@@ -637,6 +639,10 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, kDecodeMinBlocks(NT)) k_str
     for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < A.T * rows; i += gridDim.x * blockDim.x) A.out16[i] = 0;
     return;
   }
+  if (MODE == MODE_SWITCH && D == 0) {
+    for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < npairs * rows; i += gridDim.x * blockDim.x) A.yf[i] = 0.f;
+    return;
+  }
   const uint16_t* act_base = BSM ? act_s : A.act;
   constexpr int SEG = BSM ? 80 : 64;    // elements between the segments of lanes t and t + 1
   constexpr int BLKE = BSM ? 320 : 256;  // elements between consecutive 256-weight blocks
@@ -647,7 +653,7 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, kDecodeMinBlocks(NT)) k_str
     int u, mat, tile, s;
     item_of(id, u, mat, tile, s);
     int p0 = 0, ncols = A.T;
-    if (MODE == MODE_GATEUP || MODE == MODE_DOWN) {
+    if (MODE == MODE_GATEUP || MODE == MODE_DOWN || MODE == MODE_SWITCH) {
       p0 = rt.ustart[u];
       ncols = rt.ustart[u + 1] - p0;
     }
@@ -658,7 +664,7 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, kDecodeMinBlocks(NT)) k_str
       const int col = 8 * n + g < ncols ? 8 * n + g : 0;
       int arow = 0;
       if (MODE == MODE_GEMV) arow = col;
-      else if (MODE == MODE_GATEUP) arow = rt.sorted[p0 + col] / A.topk;
+      else if (MODE == MODE_GATEUP || MODE == MODE_SWITCH) arow = rt.sorted[p0 + col] / A.topk;
       else if (MODE == MODE_DOWN) arow = rt.sorted[p0 + col];
       bsrc[n] = act_base + (size_t)arow * KP + (size_t)s * bpi * BLKE + SEG * t;
       if (!BSM && MODE != MODE_FLOOR) prefetch_l1(bsrc[n]);
@@ -839,6 +845,18 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, kDecodeMinBlocks(NT)) k_str
       prev = __shfl_sync(0xffffffffu, prev, 0);
       if (prev != D * S - 1) continue;
       __threadfence();
+      if (MODE == MODE_SWITCH) {  // every pair's rows of this tile (zero for out-of-range ids)
+        for (int o = lane; o < npairs * kTile; o += 32) {
+          const int pair = o / kTile, r = o % kTile;
+          const int row = tile * kTile + r;
+          if (row >= rows) continue;
+          float v = 0.f;
+          if (rt.ids[pair] >= 0)
+            for (int ss = 0; ss < S; ss++) v += __ldcg(slab + ((size_t)pair * S + ss) * kTile + r);
+          A.yf[(size_t)pair * rows + row] = v;
+        }
+        continue;
+      }
       for (int o = lane; o < A.T * kTile; o += 32) {
         const int tok = o / kTile, r = o % kTile;
         const int row = tile * kTile + r;
@@ -1244,7 +1262,8 @@ static int launch_stream(const CUtensorMap& m0, const CUtensorMap& m1, const Uni
   UnitArgs args = a;
   args.div_s = FastDiv::of((uint32_t)a.splits);
   args.div_tiles = FastDiv::of((uint32_t)((a.w0.rows + kTile - 1) / kTile));
-  const size_t smem = stream_smem<F0, F1>(a.w0.cols, a.T * a.topk, MODE == MODE_GATEUP || MODE == MODE_DOWN,
+  const size_t smem = stream_smem<F0, F1>(a.w0.cols, a.T * a.topk,
+                                          MODE == MODE_GATEUP || MODE == MODE_DOWN || MODE == MODE_SWITCH,
                                           BSM ? a.act_rows : 0);
   if (set_smem(kern, smem)) return -4;
   const int grid = occupancy_grid(kern, smem, items, num_sms);
@@ -1461,6 +1480,67 @@ int launch_moe_decode(const WDev& g, int fg, const WDev& u, int fu, const WDev& 
   IQK_DEC_N(1, 0, 0) IQK_DEC_N(1, 0, 1) IQK_DEC_N(1, 1, 0) IQK_DEC_N(1, 1, 1)
 #undef IQK_DEC_N
 #undef IQK_DEC
+  return -3;
+}
+
+SwitchWs switch_ws(int T, int topk, int experts, int rows, int cols) {
+  SwitchWs ws;
+  const int npairs = T * topk;
+  const int tiles = (rows + kTile - 1) / kTile;
+  const int S = (cols / 256) / item_blocks(cols);
+  size_t o = 0;
+  ws.status = o;
+  o = align256(o + 16);
+  ws.xperm = o;
+  o = align256(o + (size_t)T * cols * 2);
+  ws.cnt = o;
+  o = align256(o + (size_t)tiles * 4);
+  ws.part = o;
+  o = align256(o + (size_t)tiles * npairs * S * kTile * 4);
+  ws.total = o;
+  (void)experts;
+  return ws;
+}
+
+template <int FMT, int NT>
+static int switch_impl(const WDev& w, const Values& V, const uint16_t* x, int T, const int32_t* ids, int topk,
+                       float* y, char* ws, cudaStream_t st, int num_sms) {
+  const SwitchWs L = switch_ws(T, topk, w.experts, w.rows, w.cols);
+  const int npairs = T * topk;
+  UnitArgs a = {};
+  split_args(a, w.cols);
+  CUtensorMap map;
+  if (make_qs_map(&map, w, a.bpi)) return -4;
+  uint16_t* xp = reinterpret_cast<uint16_t*>(ws + L.xperm);
+  int32_t* status = reinterpret_cast<int32_t*>(ws + L.status);
+  int32_t* cnt = reinterpret_cast<int32_t*>(ws + L.cnt);
+  const int tiles = (w.rows + kTile - 1) / kTile;
+  const int pblocks = std::max(1, std::min(num_sms, (int)(((int64_t)T * (w.cols / 16) + 63) / 64)));
+  k_prep<<<pblocks, 256, 0, st>>>(x, T, w.cols, xp, cnt, tiles, ids, npairs, w.experts, status);
+  if (cudaGetLastError() != cudaSuccess) return -4;
+  a.w0 = w;
+  a.w1 = w;
+  a.V = V;
+  a.ids = ids;
+  a.act = xp;
+  a.T = T;
+  a.topk = topk;
+  a.yf = y;
+  a.cnt = cnt;
+  a.part = reinterpret_cast<float*>(ws + L.part);
+  a.status = status;
+  const int dmax = std::min(npairs, w.experts);
+  return launch_stream_any<MODE_SWITCH, FMT, FMT, NT>(map, map, a, dmax * tiles * a.splits, st, num_sms, true, 0);
+}
+
+int launch_switch_decode(const WDev& w, int fmt, const Values& V, const uint16_t* x, int T, const int32_t* ids,
+                         int topk, float* y, char* ws, cudaStream_t st, int num_sms) {
+  const int NT = nt_for(T);
+#define IQK_SW(F, N) \
+  if (fmt == F && NT == N) return switch_impl<F, N>(w, V, x, T, ids, topk, y, ws, st, num_sms);
+  IQK_SW(FMT_KS, 1) IQK_SW(FMT_KS, 2) IQK_SW(FMT_KS, 4) IQK_SW(FMT_KS, 8)
+  IQK_SW(FMT_K, 1) IQK_SW(FMT_K, 2) IQK_SW(FMT_K, 4) IQK_SW(FMT_K, 8)
+#undef IQK_SW
   return -3;
 }
 

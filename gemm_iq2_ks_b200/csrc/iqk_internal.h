@@ -85,6 +85,18 @@ int launch_moe_decode(const WDev& g, int fg, const WDev& u, int fu, const WDev& 
                       const Values& V, const uint16_t* x, int T, const int32_t* ids, const float* p,
                       int topk, uint16_t* y, char* ws, cudaStream_t st, int num_sms);
 
+// Routed single projection (switch linear), per (token, slot) pair, fp32.
+struct SwitchWs {
+  size_t status, xperm, cnt, part, total;
+};
+SwitchWs switch_ws(int T, int topk, int experts, int rows, int cols);
+int launch_switch_decode(const WDev& w, int fmt, const Values& V, const uint16_t* x, int T, const int32_t* ids,
+                         int topk, float* y, char* ws, cudaStream_t st, int num_sms);
+// Grouped-GEMM form (rows a multiple of 256); workspace from switch_gemm_ws.
+size_t switch_gemm_ws(int T, int topk, int experts, int rows, int cols);
+int launch_switch_gemm(const WDev& w, int fmt, const Values& V, const uint16_t* x, int T, const int32_t* ids,
+                       int topk, float* y, char* ws, cudaStream_t st, int num_sms);
+
 int launch_floor(const WDev& w, int fmt, const int32_t* experts, int n, uint32_t* out, cudaStream_t st,
                  int num_sms);
 

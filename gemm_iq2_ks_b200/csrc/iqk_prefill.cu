@@ -612,4 +612,99 @@ int launch_moe_prefill(const WDev& g, int fg, const WDev& u, int fu, const WDev&
   return cudaGetLastError() == cudaSuccess ? 0 : -4;
 }
 
+// ------------------------------------------------ switch linear, GEMM form
+// y[pair] = W_{ids[pair]} x[pair / topk] for many pairs: the same grouping,
+// gather and down-mode grouped GEMM as the prefill, then the per-pair rows are
+// put back in pair order (zero rows for out-of-range ids).
+
+__global__ void __launch_bounds__(256) k_sw_scatter(const float* __restrict__ outp, const int32_t* __restrict__ inv,
+                                                    int P, int rows, float* __restrict__ y) {
+  const int64_t n = (int64_t)P * (rows / 4);
+  for (int64_t g = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; g < n; g += (int64_t)gridDim.x * blockDim.x) {
+    const int pair = (int)(g / (rows / 4)), o4 = (int)(g % (rows / 4));
+    const int pos = inv[pair];
+    const float4 v = pos >= 0 ? __ldg(reinterpret_cast<const float4*>(outp + (size_t)pos * rows) + o4)
+                              : make_float4(0.f, 0.f, 0.f, 0.f);
+    reinterpret_cast<float4*>(y + (size_t)pair * rows)[o4] = v;
+  }
+}
+
+namespace {
+struct SwGemmWs {
+  size_t status, counts, offsets, perm, inv, cc, xs, outp, total;
+};
+SwGemmWs sw_gemm_ws(int T, int topk, int experts, int rows, int cols) {
+  SwGemmWs ws = {};
+  const int P = T * topk;
+  size_t o = 0;
+  ws.status = o;
+  o = align256(o + 16);
+  ws.counts = o;
+  o = align256(o + (size_t)experts * 4);
+  ws.offsets = o;
+  o = align256(o + (size_t)(experts + 1) * 4);
+  ws.perm = o;
+  o = align256(o + (size_t)P * 4);
+  ws.inv = o;
+  o = align256(o + (size_t)P * 4);
+  ws.cc = o;
+  o = align256(o + route_scratch_ints(P, experts) * 4);
+  ws.xs = o;
+  o = align256(o + (size_t)P * cols * 2);
+  ws.outp = o;
+  o = align256(o + (size_t)P * rows * 4);
+  ws.total = o;
+  return ws;
+}
+}  // namespace
+
+size_t switch_gemm_ws(int T, int topk, int experts, int rows, int cols) {
+  return sw_gemm_ws(T, topk, experts, rows, cols).total;
+}
+
+int launch_switch_gemm(const WDev& w, int fmt, const Values& V, const uint16_t* x, int T, const int32_t* ids,
+                       int topk, float* y, char* ws, cudaStream_t st, int num_sms) {
+  const int E = w.experts, K = w.cols, R = w.rows;
+  const SwGemmWs L = sw_gemm_ws(T, topk, E, R, K);
+  const int P = T * topk;
+  int32_t* status = reinterpret_cast<int32_t*>(ws + L.status);
+  int32_t* counts = reinterpret_cast<int32_t*>(ws + L.counts);
+  int32_t* offsets = reinterpret_cast<int32_t*>(ws + L.offsets);
+  int32_t* perm = reinterpret_cast<int32_t*>(ws + L.perm);
+  int32_t* inv = reinterpret_cast<int32_t*>(ws + L.inv);
+  int32_t* cc = reinterpret_cast<int32_t*>(ws + L.cc);
+  uint16_t* xs = reinterpret_cast<uint16_t*>(ws + L.xs);
+  float* outp = reinterpret_cast<float*>(ws + L.outp);
+  if (cudaMemsetAsync(inv, 0xFF, (size_t)P * 4, st) != cudaSuccess) return -4;
+  int rc = launch_route(ids, T, topk, E, counts, offsets, perm, status, cc, st);
+  if (rc) return rc;
+  {
+    const int64_t n = (int64_t)P * (K / 16);
+    const int blocks = (int)std::min<int64_t>((n + 255) / 256, (int64_t)num_sms * 16);
+    k_pf_gather<<<std::max(blocks, 1), 256, 0, st>>>(x, K, topk, perm, offsets, E, xs, inv);
+  }
+  CUtensorMap mw, mx;
+  if (make_qs_tile_map(&mw, w) || make_rows_map(&mx, xs, P, K)) return -4;
+  PfArgs a = {};
+  a.w0 = w;
+  a.w1 = w;
+  a.V = V;
+  a.counts = counts;
+  a.offsets = offsets;
+  a.perm = perm;
+  a.outp = outp;
+  a.status = status;
+  a.E = E;
+  a.K = K;
+  a.rows = R;
+  a.mtiles = R / 256;
+  if ((rc = dispatch_gemm<1>(fmt, fmt, mw, mw, mx, a, st, num_sms))) return rc;
+  {
+    const int64_t n = (int64_t)P * (R / 4);
+    const int blocks = (int)std::min<int64_t>((n + 255) / 256, (int64_t)num_sms * 16);
+    k_sw_scatter<<<std::max(blocks, 1), 256, 0, st>>>(outp, inv, P, R, y);
+  }
+  return cudaGetLastError() == cudaSuccess ? 0 : -4;
+}
+
 }  // namespace iqk

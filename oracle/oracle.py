@@ -246,6 +246,28 @@ def moe(gate, up, down, values, x_bits, ids, p, tokens=None):
     return dict(y_bits=bf16_round(y.astype(np.float32)), y=y, S=S, S_prop=S_prop, S_round=S_round, h_bits=hb)
 
 
+# -------------------------------------------------------------- switch linear
+
+def switch_linear(w, values, x_bits, ids):
+    """Routed single projection (mlx-iqk 0.1.1 page, section "Surface": the
+    switch linear's y = proj(x, indices)): y[t, j] = W_{ids[t, j]} x[t] in
+    float64 for every (token, slot) pair, with S[t, j] = sum_k |w x| for the
+    tolerance. Out-of-range ids give zero rows (and S = 0)."""
+    ids = np.asarray(ids, np.int64)
+    T, topk = ids.shape
+    x_bits = np.atleast_2d(x_bits)
+    y = np.zeros((T, topk, w.rows))
+    S = np.zeros((T, topk, w.rows))
+    for e in np.unique(ids):
+        if e < 0 or e >= w.experts:
+            continue
+        t_idx, j_idx = np.nonzero(ids == e)
+        ye, Se = gemv(dequant_expert(w, int(e), values), x_bits[t_idx])
+        y[t_idx, j_idx] = ye
+        S[t_idx, j_idx] = Se
+    return y, S
+
+
 # ----------------------------------------------------------------- route prep
 
 def route_prep(ids, experts: int):

@@ -87,6 +87,20 @@ def test_moe_shape_checks():
     assert L.iqk_moe_workspace_bytes(0, 1, 6, 4, 256, 512) > 0
 
 
+def test_switch_linear_mode_checks():
+    L = B.lib()
+    v = np.zeros(8, np.float32).ctypes.data
+    w = _w(experts=4, rows=200, cols=512)   # rows not a multiple of 256: no grouped GEMM
+    assert L.iqk_switch_linear_workspace_bytes(2, 4, 2, 4, 200, 512) == 0
+    assert L.iqk_switch_linear_workspace_bytes(1, 4, 2, 4, 200, 512) > 0
+    assert L.iqk_switch_linear_workspace_bytes(1, 65, 2, 4, 200, 512) == 0
+    assert L.iqk_switch_linear(ctypes.byref(w), v, 4096, 4, 4096, 2, 4096, 2, 4096, 1 << 20, None) == B.IQK_EUNSUPPORTED
+    assert L.iqk_switch_linear(ctypes.byref(w), v, 4096, 4, 4096, 2, 4096, 7, 4096, 1 << 20, None) == B.IQK_EINVAL
+    assert L.iqk_switch_linear(ctypes.byref(w), v, 4096, 4, 4096, 17, 4096, 1, 4096, 1 << 20, None) == B.IQK_EINVAL
+    assert L.iqk_switch_linear(ctypes.byref(w), v, 4096, 4, 4096, 2, 4096, 1, None, 0, None) == B.IQK_EWORKSPACE
+    assert L.iqk_switch_linear(ctypes.byref(w), v, 4096, 0, 4096, 2, 4096, 1, None, 0, None) == B.IQK_OK
+
+
 def test_strerror_covers_every_status():
     L = B.lib()
     for rc in range(0, -7, -1):

@@ -422,3 +422,28 @@ def test_pins_catch_planted_mistakes(name, old, new, tmp_path):
         if not same_bits(out, expected_matrix(fmt, codes, idx, alpha, d, values)):
             caught = True
     assert caught, f"planted mistake not caught: {name}"
+
+
+# ------------------------------------------------------------- switch linear
+
+def test_switch_linear_brute_force_and_out_of_range():
+    """Every (token, slot) output equals the brute-force sum over k of the
+    pinned dequantized weight times x; out-of-range ids give zero rows."""
+    rng = S.rng_for(77)
+    w = S.random_streams(rng, "iq2_k", 3, 5, 256)
+    x = S.random_bf16(rng, (2, 256))
+    vals = S.value_table("dyadic", 1)
+    ids = np.array([[2, 0, 7], [1, 2, -1]], np.int32)
+    y, Sabs = O.switch_linear(w, vals, x, ids)
+    xf = O.bf16_to_float(x).astype(np.float64)
+    for t in range(2):
+        for j in range(3):
+            e = ids[t, j]
+            if e < 0 or e >= 3:
+                assert not y[t, j].any() and not Sabs[t, j].any()
+                continue
+            wd = O.dequant_expert(w, int(e), vals).astype(np.float64)
+            for o in range(5):
+                acc = sum(wd[o, k] * xf[t, k] for k in range(256))
+                assert abs(y[t, j, o] - acc) <= 1e-9 * max(1.0, abs(acc))
+                assert abs(Sabs[t, j, o] - sum(abs(wd[o, k] * xf[t, k]) for k in range(256))) <= 1e-9 * max(1.0, Sabs[t, j, o])
