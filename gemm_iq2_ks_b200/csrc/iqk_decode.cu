@@ -507,6 +507,18 @@ __device__ __forceinline__ void stage_scales(uint8_t* slot, const WDev& w, int64
   __syncwarp();
 }
 
+// A distinct expert can collect more pairs than the launch's MMA columns only
+// when a token lists it more than once; those extra pairs are not computed.
+// Bit 3 of the status word reports it (after the dependency wait, so it is
+// ordered after the prep kernel's store of the word).
+__device__ __forceinline__ void report_column_overflow(const RouteView& rt, int D, int NC, int32_t* status) {
+  for (int u = 0; u < D; u++)
+    if (rt.ustart[u + 1] - rt.ustart[u] > NC) {
+      atomicOr(status, 8);
+      return;
+    }
+}
+
 // Timeout flag of the floor arm, which has no workspace; read with
 // cudaMemcpyFromSymbol when diagnosing.
 __device__ int32_t g_floor_status;
@@ -874,6 +886,8 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, kDecodeMinBlocks(NT)) k_str
     }
   }
   if (!waited) griddep_wait();  // this grid completes only after the one it depends on
+  if ((MODE == MODE_GATEUP || MODE == MODE_DOWN || MODE == MODE_SWITCH) && blockIdx.x == 0 && threadIdx.x == 0)
+    report_column_overflow(rt, D, NC, A.status);
 }
 
 // ------------------------------------------------------------- tile kernel
@@ -1131,6 +1145,7 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, kDecodeMinBlocks(NT)) k_til
   // let copies still in flight land before the CTA exits (only after a timeout)
   for (int qd = consumed; qd < issued; qd++) (void)mbar_wait_bounded(&bar[qd % kStages], (uint32_t)((qd / kStages) & 1));
   if (!waited) griddep_wait();  // this grid completes only after the one it depends on
+  if (blockIdx.x == 0 && threadIdx.x == 0) report_column_overflow(rt, D, NC, A.status);
 }
 
 // ================================================================== host

@@ -237,3 +237,27 @@ def test_floor_xor_bitexact(B, fmt, rows, cols):
     out = B.iqk_floor(dw, elist).cpu().numpy().view(np.uint32)
     assert np.array_equal(out[0], O.floor_xor(w, 3))
     assert np.array_equal(out[1], O.floor_xor(w, 1))
+
+
+def test_moe_decode_duplicate_ids(B):
+    """A token listing one expert twice: both slots are computed as separate
+    pairs while the expert's pairs fit the MMA columns; beyond that the call
+    reports IQK_EUNSUPPORTED through the status word."""
+    gate, up, down, x, ids, p = _moe_case(77, "iq2_ks", "iq2_ks", "iq2_ks", E=12, H=512, F=768, T=2, topk=4)
+    ids = ids.copy()
+    ids[0, 1] = ids[0, 0]
+    ids[1, 3] = ids[1, 2]
+    dg, du, dd = (B.Weights.from_host(w) for w in (gate, up, down))
+    vals = S.value_table("int", 3)
+    ws = B.workspace(B.iqk_moe_workspace_bytes(0, 2, 4, 12, 512, 768))
+    y = B.iqk_moe_decode(dg, du, dd, vals, to_dev_bf16(x), torch.from_numpy(ids).cuda(),
+                         torch.from_numpy(p).cuda(), ws=ws)
+    assert B.iqk_moe_status(ws) == B.IQK_OK
+    check_moe(from_dev_bf16(y), O.moe(gate, up, down, vals, x, ids, p), "duplicate ids")
+    # one token, twelve slots on the same expert: more pairs than the 8 MMA columns
+    ids12 = np.full((1, 12), 5, np.int32)
+    p12 = np.full((1, 12), 1.0 / 12, np.float32)
+    ws12 = B.workspace(B.iqk_moe_workspace_bytes(0, 1, 12, 12, 512, 768))
+    B.iqk_moe_decode(dg, du, dd, vals, to_dev_bf16(x[:1]), torch.from_numpy(ids12).cuda(),
+                     torch.from_numpy(p12).cuda(), ws=ws12)
+    assert B.iqk_moe_status(ws12) == B.IQK_EUNSUPPORTED
