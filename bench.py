@@ -131,6 +131,17 @@ def cuda_time(torch, stream, fn):
     return a.elapsed_time(b) * 1e-3  # seconds
 
 
+def job_time(torch, dist, t_local, steps, world, device):
+    """Max over ranks of the timed region (one all-reduce), and the whole-job
+    µs per token: every rank runs `steps` single-token calls of its own."""
+    t = float(t_local)
+    if dist is not None:
+        tt = torch.tensor([t], dtype=torch.float64, device=device)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        t = float(tt.item())
+    return t, t / (steps * world) * 1e6
+
+
 def log(msg):
     print(f"[bench {time.strftime('%H:%M:%S')}] {msg}", file=sys.stderr, flush=True)
 
@@ -501,15 +512,11 @@ def main():
     with ClockSampler(torch.cuda.get_device_properties(device)) as clk:
         t = cuda_time(torch, stream, lambda: run_steps(graphs, K))
     torch.cuda.synchronize()
+    t, us_per_token = job_time(torch, dist, t, K, world, device)
     if dist:
-        tt = torch.tensor([t], device=device)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
         dist.barrier()
-        t = float(tt.item())
-    tokens_all = K * 1 * world
-    us_per_token = t / tokens_all * 1e6 if world > 1 else t / K * 1e6
     bytes_per_call = dec.weight_bytes(K) / K
-    gbs = bytes_per_call * K / t / 1e9
+    gbs = bytes_per_call * K / t / 1e9  # one GPU's weight stream (each rank reads its own)
 
     log(f"decode timed: {t / K * 1e6:.2f} us/call")
     # e2e through the C ABI with host buffers (copies inside the timed region)
@@ -564,7 +571,7 @@ def main():
         "metric": METRIC, "value": us_per_token, "unit": "us/token", "n_gpus": world, "steps": K, "warmup": W,
         "ms_per_step": t / K * 1e3, "higher_is_better": False, "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16", "data": "synthetic", "config": config_block({"format": "iq2_ks", "global_batch": world}),
-        "weight_gbs": gbs, "hbm_frac": gbs / peaks["hbm_gbs"],
+        "weight_gbs": gbs * world, "hbm_frac": gbs / peaks["hbm_gbs"],
         "floor": {"us_per_token": floor_us, "decode_over_floor": us_per_token / floor_us if world == 1 else
                   (t / K * 1e6) / floor_us},
         "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
