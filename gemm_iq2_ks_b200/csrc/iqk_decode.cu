@@ -202,12 +202,15 @@ __device__ __forceinline__ void block_mma(const uint32_t* __restrict__ sq, int l
 
 // One item (16 rows x bpi blocks) of a matrix in format F0 (fmt0) or F1:
 // acc[n] = d * sum over the item's blocks of W * B, rows g and g + 8.
-template <int F0, int F1, int NT, bool BSM>
-__device__ __forceinline__ void item_mma(const uint32_t* sq, const uint8_t* slot, int bpi, int o, int ldw,
+template <int F0, int F1, int NT, bool BSM, int BPI = 0>
+__device__ __forceinline__ void item_mma(const uint32_t* sq, const uint8_t* slot, int bpi_rt, int o, int ldw_rt,
                                          const uint16_t* const (&bsrc)[NT], bool fmt0, bool kfmt, const uint2* lut0,
                                          const uint2* lut1, float dg, float dh, int g, int t, uint32_t k65536,
                                          float (&acc)[NT][4]) {
   constexpr int BLKE = BSM ? 320 : 256;  // elements between consecutive 256-weight blocks
+  // a compile-time block count (BPI > 0) lets the compiler interleave the blocks
+  const int bpi = BPI > 0 ? BPI : bpi_rt;
+  const int ldw = BPI > 0 ? 16 * BPI : ldw_rt;
   float part[4][NT][4];
 #pragma unroll
   for (int m = 0; m < 4; m++)
@@ -215,7 +218,8 @@ __device__ __forceinline__ void item_mma(const uint32_t* sq, const uint8_t* slot
     for (int n = 0; n < NT; n++)
 #pragma unroll
       for (int q = 0; q < 4; q++) part[m][n][q] = 0.f;
-  for (int b = 0; b < bpi; b++) {
+#pragma unroll
+  for (int b = 0; b < (BPI > 0 ? BPI : bpi); b++) {
     const uint16_t* src[NT];
 #pragma unroll
     for (int n = 0; n < NT; n++) {
@@ -1084,7 +1088,12 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, kDecodeMinBlocks(NT)) k_til
         const uint8_t* slot = ring_slots + (size_t)st * slot_b;
         const int o = A.async_sc ? (s * bpi) & 3 : 0;
         const float dg = kfmt ? 0.f : d_smem_ks(slot, bpi, g), dh = kfmt ? 0.f : d_smem_ks(slot, bpi, g + 8);
-        item_mma<F0, F1, NT, BSM>(sq, slot, bpi, o, ldw, bsrc, fmt0, kfmt, lut0, lut1, dg, dh, g, t, k65536, acc);
+        if (bpi == 4)
+          item_mma<F0, F1, NT, BSM, 4>(sq, slot, bpi, o, ldw, bsrc, fmt0, kfmt, lut0, lut1, dg, dh, g, t, k65536, acc);
+        else if (bpi == 2)
+          item_mma<F0, F1, NT, BSM, 2>(sq, slot, bpi, o, ldw, bsrc, fmt0, kfmt, lut0, lut1, dg, dh, g, t, k65536, acc);
+        else
+          item_mma<F0, F1, NT, BSM>(sq, slot, bpi, o, ldw, bsrc, fmt0, kfmt, lut0, lut1, dg, dh, g, t, k65536, acc);
         __syncwarp();
         issue(q + kStages);  // refill the stage just consumed
       }
