@@ -746,7 +746,13 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, kDecodeMinBlocks(NT)) k_str
       const int o = A.async_sc ? (s * bpi) & 3 : 0;
       // IQ2_KS row scales of rows g and g + 8, applied after the slice's MMAs
       const float dg = kfmt ? 0.f : d_smem_ks(slot, bpi, g), dh = kfmt ? 0.f : d_smem_ks(slot, bpi, g + 8);
-      item_mma<F0, F1, NT, BSM>(sq, slot, bpi, o, ldw, bsrc, fmt0, kfmt, lut0, lut1, dg, dh, g, t, k65536, acc);
+      // unrolled over the item's blocks where registers allow (one or two column groups)
+      if (NT <= 2 && bpi == 4)
+        item_mma<F0, F1, NT, BSM, 4>(sq, slot, bpi, o, ldw, bsrc, fmt0, kfmt, lut0, lut1, dg, dh, g, t, k65536, acc);
+      else if (NT <= 2 && bpi == 2)
+        item_mma<F0, F1, NT, BSM, 2>(sq, slot, bpi, o, ldw, bsrc, fmt0, kfmt, lut0, lut1, dg, dh, g, t, k65536, acc);
+      else
+        item_mma<F0, F1, NT, BSM>(sq, slot, bpi, o, ldw, bsrc, fmt0, kfmt, lut0, lut1, dg, dh, g, t, k65536, acc);
     }
     __syncwarp();
     issue(it + kStages);  // refill the stage just consumed
