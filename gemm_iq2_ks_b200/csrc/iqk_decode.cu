@@ -22,10 +22,11 @@
 #include "iqk_internal.h"
 
 // Selector arithmetic of the code lookup: 0 all shifts on the integer-logic
-// pipe; 1 the high-half selector by multiply-high; 2 as 1, plus slot 2's
-// pre-shift by multiply-high (integer-logic and FMA pipes about even).
+// pipe (the default: fastest measured on B200 with the unrolled item loop);
+// 1 the high-half selector by multiply-high; 2 as 1, plus slot 2's pre-shift
+// by multiply-high (moves work from the integer-logic pipe to the FMA pipe).
 #ifndef IQK_LOOKUP
-#define IQK_LOOKUP 2
+#define IQK_LOOKUP 0
 #endif
 
 namespace iqk {
