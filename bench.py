@@ -38,7 +38,7 @@ RING = 420  # calls per captured graph (10 permutation cycles of 42 calls)
 # DRAM bytes (read + write) of the two tile kernels of one config-2 decode
 # call, from one ncu capture of `bench.py --profile decode --experts 24`
 # (profiles/decode_config2_tile_kernels.md); per call, not per resident expert.
-DECODE_CALL_TRAFFIC = 41_574_656
+DECODE_CALL_TRAFFIC = 41_574_144
 
 
 def env_int(k, d):
@@ -330,6 +330,129 @@ def gemv_leg(torch, B, cfg, device, stream, calls=200):
     return {"us_per_call": t * 1e6, "weight_bytes": nb, "weight_gbs_l2_warm": nb / t / 1e9}
 
 
+# ------------------------------------------------------------- pricing
+# Every kernel priced against its own deleted-decode address floor (the page's
+# "Pricing" section): identical loads, decode removed, an integer signature
+# reaching the output. Per member and projection: the routed projection
+# decode (iqk_switch_linear on the decode kernel, one token, top-6) against
+# iqk_floor over the same experts, and the dequantizer (iqk_dequant) against
+# iqk_dequant_floor (same loads and same stores). Arms alternate inside a
+# cell. Declared gates:
+PRICE_BAR = {"decode": 2.5, "dequant": 1.10}  # kernel time / own floor time, at most
+FLOOR_BAND = (0.15, 1.05)  # a floor arm streams at this fraction of the measured HBM copy rate
+PRICE_MIN_RATIO = 0.95  # a kernel clearly faster than its own floor skips loads the floor makes
+
+
+class PriceCell:
+    """One (member, projection) cell: the four arms captured as graphs over a
+    ring of single-token routings (no expert repeats within experts/6 calls)."""
+
+    def __init__(self, torch, B, w, values, device, stream, seed, calls=168):
+        self.torch, self.B, self.stream = torch, B, stream
+        self.w, self.values = w, values
+        self.dw = B.Weights.from_host(w, device)
+        rng = S.rng_for(seed)
+        self.ids_h, _ = S.routing_ring(rng, calls, w.experts, S.TOPK)
+        self.x_h = S.random_bf16(rng, (calls, 1, w.cols))
+        self.ids = torch.from_numpy(self.ids_h).to(device)
+        self.x = torch.from_numpy(self.x_h.view(np.int16)).to(device).view(torch.bfloat16)
+        self.y = torch.empty((calls, 1, S.TOPK, w.rows), dtype=torch.float32, device=device)
+        self.ws = B.workspace(B.iqk_switch_linear_workspace_bytes(1, 1, S.TOPK, w.experts, w.rows, w.cols), device)
+        self.elist = [torch.from_numpy(np.unique(self.ids_h[c]).astype(np.int32)).to(device) for c in range(calls)]
+        self.fout = torch.empty((calls, S.TOPK, w.rows), dtype=torch.int32, device=device)
+        self.deq_e = [int(self.ids_h[c, 0, 0]) for c in range(calls)]
+        self.dq = torch.empty((w.rows, w.cols), dtype=torch.float32, device=device)
+        self.dqf = torch.empty((w.rows, w.cols), dtype=torch.int32, device=device)
+        self.calls = calls
+        row_b = B.iqk_row_bytes(w.fmt, w.cols)
+        self.decode_bytes = float(np.mean([len(l) for l in self.elist])) * w.rows * row_b
+        self.dequant_bytes = w.rows * row_b + w.rows * w.cols * 4  # streams read + float32 written
+
+    def decode(self, c):
+        self.B.iqk_switch_linear(self.dw, self.values, self.x[c], self.ids[c], mode=1, y=self.y[c], ws=self.ws,
+                                 stream=self.stream)
+
+    def floor(self, c):
+        l = self.elist[c]
+        self.B.iqk_floor(self.dw, l, out=self.fout[c, :l.numel()], stream=self.stream)
+
+    def dequant(self, c):
+        self.B.iqk_dequant(self.dw, self.deq_e[c], self.values, out=self.dq, stream=self.stream)
+
+    def dequant_floor(self, c):
+        self.B.iqk_dequant_floor(self.dw, self.deq_e[c], out=self.dqf, stream=self.stream)
+
+    def graph(self, arm, n):
+        torch = self.torch
+        fn = getattr(self, arm)
+        with torch.cuda.stream(self.stream):
+            fn(0)
+        torch.cuda.synchronize()
+        return capture(torch, self.stream, lambda: [fn(c) for c in range(n)])
+
+    def time(self, reps=5, dequant_calls=42):
+        """Median µs per call of each arm, the arms of a pair alternating."""
+        torch = self.torch
+        pairs = (("decode", "floor", self.calls), ("dequant", "dequant_floor", dequant_calls))
+        out = {}
+        for a, b, n in pairs:
+            ga, gb = self.graph(a, n), self.graph(b, n)
+            for g in (ga, gb):
+                with torch.cuda.stream(self.stream):
+                    g.replay()
+            torch.cuda.synchronize()
+            ta, tb = [], []
+            for _ in range(reps):
+                ta.append(cuda_time(torch, self.stream, ga.replay) / n)
+                tb.append(cuda_time(torch, self.stream, gb.replay) / n)
+            out[a], out[b] = statistics.median(ta) * 1e6, statistics.median(tb) * 1e6
+            del ga, gb
+        return out
+
+
+def price_gates(cells, hbm_gbs):
+    """Apply the declared gates to timed cells; returns the failures (empty = pass)."""
+    fails = []
+    lo, hi = FLOOR_BAND[0] * hbm_gbs, FLOOR_BAND[1] * hbm_gbs
+    for c in cells:
+        tag = f"{c['member']} {c['projection']}"
+        for k in ("decode", "dequant"):
+            r = c[f"{k}_over_floor"]
+            if r > PRICE_BAR[k]:
+                fails.append(f"{tag}: {k} {r:.3f}x its floor, above the declared bar {PRICE_BAR[k]}")
+            if r < PRICE_MIN_RATIO:
+                fails.append(f"{tag}: {k} {r:.3f}x its floor: faster than its own loads (deleted-load signature)")
+        for k in ("floor_gbs", "dequant_floor_gbs"):
+            if not lo <= c[k] <= hi:
+                fails.append(f"{tag}: {k} {c[k]:.0f} GB/s outside the floor band [{lo:.0f}, {hi:.0f}]")
+    return fails
+
+
+def pricing_leg(torch, B, members, device, stream, peaks, reps=5):
+    """The pricing table: members = {name: (gate streams, down streams, values)}."""
+    cells = []
+    for mi, (member, (wg, wd, values)) in enumerate(members.items()):
+        for pj, (proj, w) in enumerate((("gate/up", wg), ("down", wd))):
+            cell = PriceCell(torch, B, w, values, device, stream, seed=500 + 10 * mi + pj)
+            t = cell.time(reps)
+            cells.append({"member": member, "projection": proj,
+                          "decode_us": t["decode"], "floor_us": t["floor"],
+                          "decode_over_floor": t["decode"] / t["floor"],
+                          "dequant_us": t["dequant"], "dequant_floor_us": t["dequant_floor"],
+                          "dequant_over_floor": t["dequant"] / t["dequant_floor"],
+                          "floor_gbs": cell.decode_bytes / (t["floor"] * 1e-6) / 1e9,
+                          "dequant_floor_gbs": cell.dequant_bytes / (t["dequant_floor"] * 1e-6) / 1e9})
+            del cell
+            torch.cuda.empty_cache()
+    fails = price_gates(cells, peaks["hbm_gbs"])
+    return {"cells": cells,
+            "gates": {"ratio_bar": PRICE_BAR, "floor_band_of_hbm": FLOOR_BAND, "min_ratio": PRICE_MIN_RATIO,
+                      "hbm_gbs": peaks["hbm_gbs"], "pass": not fails, "failures": fails},
+            "arms": "decode = iqk_switch_linear (decode kernel, 1 token, top-6) vs iqk_floor on the same experts; "
+                    "dequant = iqk_dequant (float32) vs iqk_dequant_floor; medians of "
+                    f"{reps} alternating repeats"}
+
+
 # ------------------------------------------------------------ cpu oracle
 
 def oracle_decode_seconds(weights, values, budget_s, seed=99):
@@ -438,6 +561,7 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work for cpu_baseline")
     ap.add_argument("--no-details", action="store_true")
+    ap.add_argument("--no-price", action="store_true", help="skip the pricing table (kernels vs own floors)")
     ap.add_argument("--profile", choices=["decode", "prefill"], default=None,
                     help="plain launches without graphs or reporting (for ncu captures)")
     ap.add_argument("--experts", type=int, default=S.EXPERTS,
@@ -558,6 +682,11 @@ def main():
                                         "hbm_frac": by / per_call / 1e9 / peaks["hbm_gbs"],
                                         "mean_distinct_experts": float(db.distinct.mean())}
             del db, gr
+        if not args.no_price:
+            log("pricing against own floors")
+            details["pricing"] = pricing_leg(torch, B, {"IQ2_KS": (w_ks[0], w_ks[2], values),
+                                                        "IQ2_K": (w_k[0], w_k[2], S.value_table("f16", 3))},
+                                             device, stream, peaks)
         del w_k
         torch.cuda.empty_cache()
         log("config 4 prefill")

@@ -21,7 +21,7 @@ FMT = {"iq2_ks": 0, "iq2_k": 1}
 
 EXPORTS = (
     "iqk_strerror", "iqk_last_cuda_error", "iqk_version", "iqk_row_bytes",
-    "iqk_dequant", "iqk_dequant_bf16", "iqk_gemv_workspace_bytes", "iqk_gemv", "iqk_gemv_static",
+    "iqk_dequant", "iqk_dequant_bf16", "iqk_dequant_floor", "iqk_gemv_workspace_bytes", "iqk_gemv", "iqk_gemv_static",
     "iqk_moe_workspace_bytes", "iqk_moe_decode", "iqk_moe_prefill", "iqk_moe_status",
     "iqk_route_workspace_bytes", "iqk_moe_route", "iqk_floor",
     "iqk_switch_linear_workspace_bytes", "iqk_switch_linear",
@@ -60,6 +60,7 @@ def lib(build_if_missing: bool = True) -> ctypes.CDLL:
             "iqk_row_bytes": (ctypes.c_int64, [i32, i32]),
             "iqk_dequant": (ctypes.c_int, [W, i32, vp, vp, vp]),
             "iqk_dequant_bf16": (ctypes.c_int, [W, i32, vp, vp, vp]),
+            "iqk_dequant_floor": (ctypes.c_int, [W, i32, i32, vp, vp]),
             "iqk_gemv_workspace_bytes": (sz, [i32, i32, i32]),
             "iqk_gemv": (ctypes.c_int, [W, i32, vp, vp, i32, vp, vp, sz, vp]),
             "iqk_gemv_static": (ctypes.c_int, [W, i32, vp, vp, i32, vp, vp]),
@@ -172,6 +173,16 @@ def iqk_dequant_bf16(w: Weights, expert: int, values, out=None, stream=None):
     v = _values(values)
     _check(lib().iqk_dequant_bf16(ctypes.byref(w.c), expert, v.ctypes.data, out.data_ptr(), _stream(stream)),
            "iqk_dequant_bf16")
+    return out
+
+
+def iqk_dequant_floor(w: Weights, expert: int, bf16: bool = False, out=None, stream=None):
+    """The dequantizer's deleted-decode floor: int32 [rows][cols] (or
+    [rows][cols/2] with bf16), the integer signature of every loaded word."""
+    torch = _torch()
+    out = _empty((w.rows, w.cols // 2 if bf16 else w.cols), torch.int32, w.qs.device) if out is None else out
+    _check(lib().iqk_dequant_floor(ctypes.byref(w.c), expert, int(bool(bf16)), out.data_ptr(), _stream(stream)),
+           "iqk_dequant_floor")
     return out
 
 

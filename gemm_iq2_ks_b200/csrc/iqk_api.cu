@@ -125,7 +125,7 @@ int iqk_dequant(const iqk_weights* w, int32_t expert, const float* values, float
   if (expert < 0 || expert >= wd.experts || !out || !aligned(out, 16)) return IQK_EINVAL;
   const int sms = num_sms();
   if (sms < 0) return cuda_fail(cudaGetLastError());
-  return from_launch(launch_dequant(wd, w->fmt, expert, V, out, false, (cudaStream_t)stream, sms));
+  return from_launch(launch_dequant(wd, w->fmt, expert, V, out, false, false, (cudaStream_t)stream, sms));
 }
 
 int iqk_dequant_bf16(const iqk_weights* w, int32_t expert, const float* values, uint16_t* out, void* stream) {
@@ -136,7 +136,18 @@ int iqk_dequant_bf16(const iqk_weights* w, int32_t expert, const float* values, 
   if (expert < 0 || expert >= wd.experts || !out || !aligned(out, 16)) return IQK_EINVAL;
   const int sms = num_sms();
   if (sms < 0) return cuda_fail(cudaGetLastError());
-  return from_launch(launch_dequant(wd, w->fmt, expert, V, out, true, (cudaStream_t)stream, sms));
+  return from_launch(launch_dequant(wd, w->fmt, expert, V, out, true, false, (cudaStream_t)stream, sms));
+}
+
+int iqk_dequant_floor(const iqk_weights* w, int32_t expert, int32_t bf16, uint32_t* out, void* stream) {
+  WDev wd;
+  int rc;
+  if ((rc = check_weights(w, &wd))) return rc;
+  if (expert < 0 || expert >= wd.experts || !out || !aligned(out, 16)) return IQK_EINVAL;
+  const int sms = num_sms();
+  if (sms < 0) return cuda_fail(cudaGetLastError());
+  Values V{};
+  return from_launch(launch_dequant(wd, w->fmt, expert, V, out, bf16 != 0, true, (cudaStream_t)stream, sms));
 }
 
 size_t iqk_gemv_workspace_bytes(int32_t T, int32_t rows, int32_t cols) {

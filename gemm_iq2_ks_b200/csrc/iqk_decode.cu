@@ -418,6 +418,7 @@ struct UnitArgs {
   int splits;    // items per tile and matrix (blocks per row / bpi)
   int async_sc;  // scale slices by cp.async (blocks per row a multiple of four)
   int act_rows;  // BSM: activation rows copied into shared memory
+  int tpg;       // tile kernel, SWITCH: tiles per group (items per group = splits * tpg)
   FastDiv div_s, div_tiles;
 };
 
@@ -917,7 +918,7 @@ template <int MODE, int F0, int F1, int NT, bool BSM>
 __global__ void __launch_bounds__(kDecodeWarps * 32, kDecodeMinBlocks(NT)) k_tiles(const __grid_constant__ CUtensorMap m0,
                                                                              const __grid_constant__ CUtensorMap m1,
                                                                              const __grid_constant__ UnitArgs A) {
-  static_assert(MODE == MODE_GATEUP || MODE == MODE_DOWN, "tile kernel: gate/up or down");
+  static_assert(MODE == MODE_GATEUP || MODE == MODE_DOWN || MODE == MODE_SWITCH, "tile kernel: gate/up, down, switch");
   extern __shared__ __align__(128) uint8_t smem[];
   const int wid = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
   const int K = A.w0.cols;
@@ -938,12 +939,13 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, kDecodeMinBlocks(NT)) k_til
   const int KP = BSM ? K / 64 * 80 : K;  // activation row stride (elements), see k_stream
   uint16_t* act_s = reinterpret_cast<uint16_t*>(lut1 + 64);
   float* red = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(act_s) + (BSM ? (size_t)A.act_rows * KP * 2 : 0));
-  const int slot_f = MODE == MODE_GATEUP ? 2 * NC * kTile : A.T * kTile;  // floats per warp slot
+  // floats per warp slot: (mat, column, row) gate/up; (column, row) switch; (token, row) down
+  const int slot_f = MODE == MODE_GATEUP ? 2 * NC * kTile : MODE == MODE_SWITCH ? NC * kTile : A.T * kTile;
   uint8_t* route_p = reinterpret_cast<uint8_t*>(red + (size_t)kDecodeWarps * slot_f);
   // gate/up: request the first activation groups ahead of the weight stream
   uint4 pre0 = make_uint4(0u, 0u, 0u, 0u), pre1 = pre0, pre2 = pre0, pre3 = pre0;
   const int act_groups = BSM ? A.act_rows * (K / 16) : 0;
-  if (BSM && MODE == MODE_GATEUP) {
+  if (BSM && MODE != MODE_DOWN) {
     const int g0 = threadIdx.x, g1 = threadIdx.x + blockDim.x;
     if (g0 < act_groups) {
       pre0 = ld_nc_u4(A.xraw + (size_t)g0 * 16);
@@ -965,8 +967,12 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, kDecodeMinBlocks(NT)) k_til
   const int D = rt.scalars[0];
   const int rows = A.w0.rows;
   const int tiles = (rows + kTile - 1) / kTile;
-  const int n_it = MODE == MODE_GATEUP ? 2 * S : D * S;          // items per group
-  const int ngroups = MODE == MODE_GATEUP ? D * tiles : tiles;
+  // SWITCH: a group is `tpg` consecutive tiles of one expert (the last run
+  // may extend past the matrix: those items load its last tile and are dropped)
+  const int tpg = MODE == MODE_SWITCH ? A.tpg : 1;
+  const int ntg = (tiles + tpg - 1) / tpg;  // groups per expert (SWITCH)
+  const int n_it = MODE == MODE_GATEUP ? 2 * S : MODE == MODE_SWITCH ? S * tpg : D * S;  // items per group
+  const int ngroups = MODE == MODE_GATEUP ? D * tiles : MODE == MODE_SWITCH ? D * ntg : tiles;
   const int rounds = (int)blockIdx.x < ngroups ? (ngroups - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
   const int cnt_w = wid < n_it ? (n_it - 1 - wid) / kDecodeWarps + 1 : 0;  // this warp's items per group
   const int nq = rounds * cnt_w;
@@ -981,6 +987,10 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, kDecodeMinBlocks(NT)) k_til
       mat = js;
       u = (int)A.div_tiles.div((uint32_t)tg);
       tile = tg - u * tiles;
+    } else if (MODE == MODE_SWITCH) {
+      mat = 0;
+      u = (int)A.div_tiles.div((uint32_t)tg);  // div_tiles divides by ntg here
+      tile = min((tg - u * ntg) * tpg + js, tiles - 1);
     } else {
       mat = 0;
       u = js;
@@ -1044,6 +1054,13 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, kDecodeMinBlocks(NT)) k_til
     }
     __syncthreads();
   }
+  if (MODE == MODE_SWITCH && rt.scalars[1] < npairs) {  // out-of-range ids: zero rows
+    for (int pr = 0; pr < npairs; pr++) {
+      if (rt.ids[pr] >= 0) continue;
+      for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < rows; i += gridDim.x * blockDim.x)
+        A.yf[(size_t)pr * rows + i] = 0.f;
+    }
+  }
   if (MODE == MODE_DOWN && D == 0) {  // every id out of range: the block output is zero
     for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < A.T * rows; i += gridDim.x * blockDim.x) A.out16[i] = 0;
     return;
@@ -1069,7 +1086,7 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, kDecodeMinBlocks(NT)) k_til
         // columns past the last pair repeat column 0; their sums are never used
         const int col = 8 * n + g < ncols ? 8 * n + g : 0;
         const int pair = rt.sorted[p0 + col];
-        const int arow = MODE == MODE_GATEUP ? pair / A.topk : pair;
+        const int arow = MODE == MODE_DOWN ? pair : pair / A.topk;
         bsrc[n] = act_base + (size_t)arow * KP + (size_t)s * bpi * BLKE + SEG * t;
         if (!BSM) prefetch_l1(bsrc[n]);
       }
@@ -1104,8 +1121,9 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, kDecodeMinBlocks(NT)) k_til
         __syncwarp();
         issue(q + kStages);  // refill the stage just consumed
       }
-      // add into this warp's slot: (mat, column, row) for gate/up, (token, row) for down
-      if (MODE == MODE_GATEUP) {
+      // add into this warp's slot: (mat, column, row) for gate/up, (column, row)
+      // for switch (a warp's items in a group share one tile), (token, row) for down
+      if (MODE != MODE_DOWN) {
 #pragma unroll
         for (int n = 0; n < NT; n++)
 #pragma unroll
@@ -1133,7 +1151,7 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, kDecodeMinBlocks(NT)) k_til
       const int u = (int)A.div_tiles.div((uint32_t)tg);
       const int tile = tg - u * tiles;
       const int p0 = rt.ustart[u];
-      const int ncols = rt.ustart[u + 1] - p0;
+      const int ncols = min(rt.ustart[u + 1] - p0, NC);  // more columns: reported as overflow
       for (int o = threadIdx.x; o < ncols * kTile; o += blockDim.x) {
         const int col = o / kTile, row = o - col * kTile;
         const int f = tile * kTile + row;
@@ -1145,6 +1163,24 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, kDecodeMinBlocks(NT)) k_til
         }
         const float h = gv / (1.0f + __expf(-gv)) * uv;
         A.out16[(size_t)rt.sorted[p0 + col] * rows + perm16(f)] = f32_to_bf16_bits(h);
+      }
+    } else if (MODE == MODE_SWITCH) {
+      // y[pair][row] = sum of the tile's slices; with several tiles per group
+      // warp w holds slice w % S of tile w / S (one item each)
+      const int u = (int)A.div_tiles.div((uint32_t)tg);
+      const int t0 = (tg - u * ntg) * tpg;
+      const int p0 = rt.ustart[u];
+      const int ncols = min(rt.ustart[u + 1] - p0, NC);
+      const int per = ncols * kTile;
+      for (int o = threadIdx.x; o < tpg * per; o += blockDim.x) {
+        const int sub = o / per, rem = o - sub * per;
+        const int col = rem / kTile, row = rem - col * kTile;
+        const int f = (t0 + sub) * kTile + row;
+        if (t0 + sub >= tiles || f >= rows) continue;
+        const int w0 = tpg > 1 ? sub * S : 0, w1 = tpg > 1 ? w0 + S : kDecodeWarps;
+        float v = 0.f;
+        for (int w = w0; w < w1; w++) v += red[(size_t)w * slot_f + col * kTile + row];
+        A.yf[(size_t)rt.sorted[p0 + col] * rows + f] = v;
       }
     } else {
       for (int o = threadIdx.x; o < A.T * kTile; o += blockDim.x) {
@@ -1206,7 +1242,8 @@ template <int MODE, int F0, int F1, int NT>
 static size_t tiles_smem(int cols, int T, int npairs, int act_rows) {
   const int bpi = item_blocks(cols);
   const size_t warp = (size_t)kStages * ((size_t)kTile * bpi * 16 * 4 + slot_bytes2<F0, F1>(bpi));
-  const size_t red = (size_t)kDecodeWarps * (MODE == MODE_GATEUP ? 2 * 8 * NT * kTile : T * kTile) * 4;
+  const size_t red =
+      (size_t)kDecodeWarps * (MODE == MODE_GATEUP ? 2 * 8 * NT * kTile : MODE == MODE_SWITCH ? 8 * NT * kTile : T * kTile) * 4;
   return kDecodeWarps * warp + (size_t)kDecodeWarps * kStages * 8 + 2 * 64 * 8 + (size_t)act_rows * (cols / 64 * 80) * 2 +
          red + route_smem_bytes(npairs);
 }
@@ -1316,7 +1353,8 @@ static int launch_tiles(const CUtensorMap& m0, const CUtensorMap& m1, const Unit
   auto kern = k_tiles<MODE, F0, F1, NT, BSM>;
   UnitArgs args = a;
   args.div_s = FastDiv::of((uint32_t)a.splits);
-  args.div_tiles = FastDiv::of((uint32_t)((a.w0.rows + kTile - 1) / kTile));
+  const int tiles = (a.w0.rows + kTile - 1) / kTile;
+  args.div_tiles = FastDiv::of((uint32_t)(MODE == MODE_SWITCH ? (tiles + a.tpg - 1) / a.tpg : tiles));
   const size_t smem = tiles_smem<MODE, F0, F1, NT>(a.w0.cols, a.T, a.T * a.topk, BSM ? a.act_rows : 0);
   if (set_smem(kern, smem)) return -4;
   KernelCache* kc = kcache(reinterpret_cast<const void*>(kern));
@@ -1561,6 +1599,16 @@ static int switch_impl(const WDev& w, const Values& V, const uint16_t* x, int T,
   a.part = reinterpret_cast<float*>(ws + L.part);
   a.status = status;
   const int dmax = std::min(npairs, w.experts);
+  if constexpr (NT <= 2) {
+    // tile kernel: a group is tpg tiles of one expert, splits * tpg <= warps items
+    a.tpg = std::max(1, kDecodeWarps / a.splits);
+    const int groups = dmax * ((tiles + a.tpg - 1) / a.tpg);
+    const int ar = act_rows_smem(NT, T, w.cols);
+    a.act_rows = ar;
+    a.xraw = x;
+    return ar ? launch_tiles<MODE_SWITCH, FMT, FMT, NT, true>(map, map, a, groups, st, num_sms, true)
+              : launch_tiles<MODE_SWITCH, FMT, FMT, NT, false>(map, map, a, groups, st, num_sms, true);
+  }
   return launch_stream_any<MODE_SWITCH, FMT, FMT, NT>(map, map, a, dmax * tiles * a.splits, st, num_sms, true, 0);
 }
 

@@ -11,7 +11,12 @@ namespace iqk {
 
 // One thread per qs word (16 weights): one sub-block (IQ2_K) or half of one
 // (IQ2_KS); output written with 16-byte stores.
-template <int FMT, bool BF16>
+//
+// FLOOR: the same loads and the same stores with the decode deleted. The
+// loaded words are folded into one integer, m = q ^ scl ^ sch ^ (sex << 8) ^
+// (dv << 16), and output word k of the thread's 16 (8 for bf16) is m ^ k, so
+// every loaded byte reaches the output and nothing can be elided.
+template <int FMT, bool BF16, bool FLOOR>
 __global__ void __launch_bounds__(256) k_dequant(WDev w, int expert, Values V, void* __restrict__ out) {
   const int cols = w.cols;
   const int wpr = cols / 16;  // qs words per row
@@ -22,27 +27,43 @@ __global__ void __launch_bounds__(256) k_dequant(WDev w, int expert, Values V, v
     const int wk = (int)(gi - r * wpr);
     const int64_t er = (int64_t)expert * w.rows + r;
     const uint32_t q = __ldg(w.qs + er * wpr + wk);
+    uint32_t s, h, x, dvb;
     int idx, a;
-    float d;
     if (FMT == FMT_KS) {
       const int j = wk >> 1;  // 32-weight sub-block
       const int64_t sb = er * (cols / 256) + (j >> 3);
-      const uint32_t s = __ldg(w.scl + sb);
-      const uint32_t h = __ldg(w.sch + sb);
-      const uint32_t x = __ldg(reinterpret_cast<const uint8_t*>(w.sex) + sb);
+      s = __ldg(w.scl + sb);
+      h = __ldg(w.sch + sb);
+      x = __ldg(reinterpret_cast<const uint8_t*>(w.sex) + sb);
+      dvb = __ldg(w.dv + er);
       const int lo = (s >> (4 * (j & 7))) & 15;
       const int hi = (h >> (j & 7)) & 1;
       idx = (lo | (hi << 4)) - 16;
       a = (x >> (j & 7)) & 1;
-      d = __half2float(__ushort_as_half(__ldg(w.dv + er)));
     } else {
       const int j = wk;  // 16-weight sub-block
-      const uint32_t s = __ldg(w.scl + er * (cols / 128) + (j >> 3));
-      const uint32_t x = __ldg(reinterpret_cast<const uint16_t*>(w.sex) + er * (cols / 256) + (j >> 4));
+      s = __ldg(w.scl + er * (cols / 128) + (j >> 3));
+      h = 0u;
+      x = __ldg(reinterpret_cast<const uint16_t*>(w.sex) + er * (cols / 256) + (j >> 4));
+      dvb = __ldg(w.dv + er * (cols / 256) + (wk >> 4));
       idx = (int)((s >> (4 * (j & 7))) & 15) - 8;
       a = (x >> (j & 15)) & 1;
-      d = __half2float(__ushort_as_half(__ldg(w.dv + er * (cols / 256) + (wk >> 4))));
     }
+    if constexpr (FLOOR) {
+      const uint32_t m = q ^ s ^ h ^ (x << 8) ^ (dvb << 16);
+      uint32_t* o32 = static_cast<uint32_t*>(out);
+      if (!BF16) {
+        uint4* dst = reinterpret_cast<uint4*>(o32 + r * cols + 16 * wk);
+#pragma unroll
+        for (int v = 0; v < 4; v++) dst[v] = make_uint4(m ^ (4u * v), m ^ (4u * v + 1), m ^ (4u * v + 2), m ^ (4u * v + 3));
+      } else {
+        uint4* dst = reinterpret_cast<uint4*>(o32 + r * (cols / 2) + 8 * wk);
+        dst[0] = make_uint4(m, m ^ 1u, m ^ 2u, m ^ 3u);
+        dst[1] = make_uint4(m ^ 4u, m ^ 5u, m ^ 6u, m ^ 7u);
+      }
+      continue;
+    }
+    const float d = __half2float(__ushort_as_half((unsigned short)dvb));
     const float t = __fmul_rn(d, (float)idx);
     const float p0 = __fmul_rn(t, a ? V.v[4] : V.v[0]);
     const float p1 = __fmul_rn(t, a ? V.v[5] : V.v[1]);
@@ -69,7 +90,19 @@ __global__ void __launch_bounds__(256) k_dequant(WDev w, int expert, Values V, v
   }
 }
 
-int launch_dequant(const WDev& w, int fmt, int expert, const Values& V, void* out, bool bf16,
+template <bool FLOOR>
+static void dequant_kernel(int fmt, bool bf16, int64_t blocks, int threads, cudaStream_t st, const WDev& w,
+                           int expert, const Values& V, void* out) {
+  if (fmt == FMT_KS) {
+    if (bf16) k_dequant<FMT_KS, true, FLOOR><<<(unsigned)blocks, threads, 0, st>>>(w, expert, V, out);
+    else k_dequant<FMT_KS, false, FLOOR><<<(unsigned)blocks, threads, 0, st>>>(w, expert, V, out);
+  } else {
+    if (bf16) k_dequant<FMT_K, true, FLOOR><<<(unsigned)blocks, threads, 0, st>>>(w, expert, V, out);
+    else k_dequant<FMT_K, false, FLOOR><<<(unsigned)blocks, threads, 0, st>>>(w, expert, V, out);
+  }
+}
+
+int launch_dequant(const WDev& w, int fmt, int expert, const Values& V, void* out, bool bf16, bool floor,
                    cudaStream_t st, int num_sms) {
   const int64_t nwords = (int64_t)w.rows * (w.cols / 16);
   const int threads = 256;
@@ -77,13 +110,8 @@ int launch_dequant(const WDev& w, int fmt, int expert, const Values& V, void* ou
   const int64_t cap = (int64_t)num_sms * 16;
   if (blocks > cap) blocks = cap;
   if (blocks < 1) blocks = 1;
-  if (fmt == FMT_KS) {
-    if (bf16) k_dequant<FMT_KS, true><<<(unsigned)blocks, threads, 0, st>>>(w, expert, V, out);
-    else k_dequant<FMT_KS, false><<<(unsigned)blocks, threads, 0, st>>>(w, expert, V, out);
-  } else {
-    if (bf16) k_dequant<FMT_K, true><<<(unsigned)blocks, threads, 0, st>>>(w, expert, V, out);
-    else k_dequant<FMT_K, false><<<(unsigned)blocks, threads, 0, st>>>(w, expert, V, out);
-  }
+  if (floor) dequant_kernel<true>(fmt, bf16, blocks, threads, st, w, expert, V, out);
+  else dequant_kernel<false>(fmt, bf16, blocks, threads, st, w, expert, V, out);
   return cudaGetLastError() == cudaSuccess ? 0 : -4;
 }
 

@@ -12,7 +12,8 @@
 namespace iqk {
 
 // ---------------------------------------------------------------- dequant
-int launch_dequant(const WDev& w, int fmt, int expert, const Values& V, void* out, bool bf16,
+// floor: the same loads and stores with the decode deleted (integer signature).
+int launch_dequant(const WDev& w, int fmt, int expert, const Values& V, void* out, bool bf16, bool floor,
                    cudaStream_t st, int num_sms);
 
 // ------------------------------------------------------- decode (GEMV-type)

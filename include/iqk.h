@@ -120,6 +120,26 @@ int iqk_dequant_bf16(const iqk_weights* w, int32_t expert, const float* values /
                      uint16_t* out, void* stream);
 
 /*
+ * iqk_dequant_floor -- the dequantizer's own deleted-decode floor (page
+ * section "Pricing": identical loads, decode removed, an integer accumulator
+ * reaching the output). It performs the loads and the stores of iqk_dequant
+ * (bf16 == 0) or iqk_dequant_bf16 (bf16 != 0) with the reconstruction
+ * replaced by integer folding: for qs word wk of row r (weights 16*wk ..
+ * 16*wk+15), with the stream fields that word's weights read,
+ *   IQ2_KS: m = qs ^ scl_word ^ sch_byte ^ (sex_byte << 8) ^ (dv << 16)
+ *           (scl word, sch byte and sex byte of 256-block wk/16; the row's dv)
+ *   IQ2_K:  m = qs ^ scl_word ^ (sex_halfword << 8) ^ (dv << 16)
+ *           (scl word wk/8; sex halfword and dv of 256-block wk/16)
+ * and writes out[r][16*wk + k] = m ^ k, k < 16 (bf16 == 0; out uint32
+ * [rows][cols], the bytes of the float32 result) or out[r][8*wk + k] = m ^ k,
+ * k < 8 (bf16 != 0; out uint32 [rows][cols/2], the bytes of the bf16 result).
+ * out: device, 16-byte aligned, written completely.
+ * Errors: IQK_EINVAL (NULL, bad fmt, expert out of range, misaligned out),
+ * IQK_ESHAPE.
+ */
+int iqk_dequant_floor(const iqk_weights* w, int32_t expert, int32_t bf16, uint32_t* out, void* stream);
+
+/*
  * iqk_gemv -- y[t][o] = sum_k w[o][k] * x[t][k] for one expert, t < T.
  * Defines: the fused decode GEMV of the page's "Surface" section (few
  * token-expert pairs, one pass over the reduction axis).

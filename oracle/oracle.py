@@ -26,6 +26,9 @@ What it computes, and where each step is defined:
   expert ... each expert's weights read once" requires (section "Surface").
 * ``floor_xor``: the deleted-decode address floor's checksum (section
   "Pricing": identical loads, decode removed, an integer accumulator).
+* ``dequant_floor``: the dequantizer's own floor signature (same section):
+  per qs word, the XOR of the stream fields its 16 weights are decoded from,
+  written where the dequantizer writes those weights.
 """
 from __future__ import annotations
 
@@ -296,3 +299,37 @@ def floor_xor(w, e: int) -> np.ndarray:
     out = np.empty(rows, np.uint32)
     lib().oracle_floor_xor(rows, len(arrs), ptrs, _p(rb), _p(out))
     return out
+
+
+def dequant_floor(w, e: int, bf16: bool = False) -> np.ndarray:
+    """Signature the dequantizer's deleted-decode floor writes for expert ``e``.
+
+    Qs word wk of row r carries weights 16*wk .. 16*wk+15; the fields those
+    weights are decoded from (section "Format": IQ2_KS one scl word, one sch
+    and one sex byte per 256 weights and one dv per row; IQ2_K one scl word
+    per 128 weights, one sex halfword and one dv per 256) fold into
+    ``m = qs ^ scl ^ sch ^ (sex << 8) ^ (dv << 16)``. The floor stores m ^ k
+    in the k-th 32-bit word of the weights' output bytes: 16 words per qs word
+    for the float32 output, 8 for bfloat16. uint32 [rows][cols] or
+    [rows][cols / 2].
+    """
+    rows, cols = w.rows, w.cols
+    wpr = cols // 16
+    wk = np.arange(wpr)
+    q = np.asarray(w.qs[e]).reshape(rows, wpr).astype(np.uint32)
+    blk = wk // 16  # 256-weight block of each qs word
+    if w.fmt == "iq2_ks":
+        s = np.asarray(w.scl[e]).reshape(rows, -1)[:, blk].astype(np.uint32)
+        h = np.asarray(w.sch[e]).reshape(rows, -1)[:, blk].astype(np.uint32)
+        x = np.asarray(w.sex[e]).reshape(rows, -1)[:, blk].astype(np.uint32)
+        dv = np.repeat(np.asarray(w.dv[e]).reshape(rows, 1).astype(np.uint32), wpr, axis=1)
+    elif w.fmt == "iq2_k":
+        s = np.asarray(w.scl[e]).reshape(rows, -1)[:, wk // 8].astype(np.uint32)
+        h = np.zeros((rows, wpr), np.uint32)
+        x = np.asarray(w.sex[e]).reshape(rows, -1)[:, blk].astype(np.uint32)
+        dv = np.asarray(w.dv[e]).reshape(rows, -1)[:, blk].astype(np.uint32)
+    else:
+        raise ValueError(f"unknown format {w.fmt!r}")
+    m = q ^ s ^ h ^ (x << np.uint32(8)) ^ (dv << np.uint32(16))
+    n = 8 if bf16 else 16
+    return (m[:, :, None] ^ np.arange(n, dtype=np.uint32)[None, None, :]).reshape(rows, wpr * n)

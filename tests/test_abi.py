@@ -59,6 +59,11 @@ def test_host_validation_rejects_before_any_launch():
     assert L.iqk_dequant(ctypes.byref(w), 1, P, 4096, None) == B.IQK_EINVAL  # expert out of range
     assert L.iqk_dequant(ctypes.byref(w), 0, None, 4096, None) == B.IQK_EINVAL  # no table
     assert L.iqk_dequant(None, 0, P, 4096, None) == B.IQK_EINVAL
+    # dequantizer floor: same checks, no table
+    assert L.iqk_dequant_floor(ctypes.byref(_w(cols=100)), 0, 0, 4096, None) == B.IQK_ESHAPE
+    assert L.iqk_dequant_floor(ctypes.byref(w), 1, 0, 4096, None) == B.IQK_EINVAL  # expert out of range
+    assert L.iqk_dequant_floor(ctypes.byref(w), 0, 1, None, None) == B.IQK_EINVAL  # no output
+    assert L.iqk_dequant_floor(ctypes.byref(w), 0, 0, 4100, None) == B.IQK_EINVAL  # output misaligned
     # gemv: token count and workspace
     assert L.iqk_gemv(ctypes.byref(w), 0, P, 4096, 65, 4096, 4096, 1 << 20, None) == B.IQK_EUNSUPPORTED
     assert L.iqk_gemv(ctypes.byref(w), 0, P, 4096, 1, 4096, None, 0, None) == B.IQK_EWORKSPACE

@@ -239,6 +239,18 @@ def test_floor_xor_bitexact(B, fmt, rows, cols):
     assert np.array_equal(out[1], O.floor_xor(w, 1))
 
 
+@pytest.mark.parametrize("fmt,rows,cols", [("iq2_ks", 2048, 4096), ("iq2_k", 4096, 2048), ("iq2_ks", 37, 512),
+                                           ("iq2_k", 5, 256)])
+@pytest.mark.parametrize("bf16", [False, True])
+def test_dequant_floor_bitexact(B, fmt, rows, cols, bf16):
+    rng = S.rng_for(rows + 1)
+    w = S.random_streams(rng, fmt, 3, rows, cols)
+    dw = B.Weights.from_host(w)
+    for e in (2, 0):
+        out = B.iqk_dequant_floor(dw, e, bf16=bf16).cpu().numpy().view(np.uint32)
+        assert np.array_equal(out, O.dequant_floor(w, e, bf16=bf16)), (fmt, rows, cols, bf16, e)
+
+
 def test_moe_decode_duplicate_ids(B):
     """A token listing one expert twice: both slots are computed as separate
     pairs while the expert's pairs fit the MMA columns; beyond that the call

@@ -85,3 +85,35 @@ def test_switch_auto_config_geometry(B, T):
     sub = ids[toks]
     y_ref, Sabs = O.switch_linear(w, vals, x[toks], sub)
     check_fp32(y[toks], y_ref, Sabs, f"switch auto T={T}")
+
+
+@pytest.mark.parametrize("fmt,rows,cols,T", [
+    ("iq2_ks", 37, 256, 1),    # one slice per row: 8 tiles per group, ragged last group
+    ("iq2_k", 100, 1024, 3),   # two slices: 4 tiles per group
+    ("iq2_ks", 48, 5120, 2),   # five slices: one tile per group
+    ("iq2_k", 33, 9216, 1),    # nine slices: a warp takes two items of a group
+    ("iq2_ks", 200, 768, 12),  # two column groups, activations through the read-only path
+    ("iq2_k", 130, 2048, 16),  # sixteen columns per expert at most
+])
+def test_switch_decode_tile_geometries(B, fmt, rows, cols, T):
+    """The decode kernel's group shapes (tiles per group from the slices per
+    row) at ragged row counts, one and two MMA column groups."""
+    w, x, ids = _case(200 + rows, fmt, 10, rows, cols, T, 6)
+    vals = S.value_table("int", 9)
+    y, st = _run(B, w, x, ids, vals, mode=1)
+    y_ref, Sabs = O.switch_linear(w, vals, x, ids)
+    assert st == 0
+    check_fp32(y, y_ref, Sabs, f"switch decode {fmt} {rows}x{cols} T={T}")
+
+
+def test_switch_decode_duplicate_slot(B):
+    """A token listing one expert in two slots gets the same row in both."""
+    w, x, ids = _case(210, "iq2_ks", 6, 64, 512, 2, 3)
+    ids = ids.copy()
+    ids[0, 2] = ids[0, 0]
+    vals = S.value_table("int", 10)
+    y, st = _run(B, w, x, ids, vals, mode=1)
+    y_ref, Sabs = O.switch_linear(w, vals, x, ids)
+    assert st == 0
+    check_fp32(y, y_ref, Sabs, "switch decode duplicate slot")
+    assert np.array_equal(y[0, 0], y[0, 2])

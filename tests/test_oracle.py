@@ -447,3 +447,62 @@ def test_switch_linear_brute_force_and_out_of_range():
                 acc = sum(wd[o, k] * xf[t, k] for k in range(256))
                 assert abs(y[t, j, o] - acc) <= 1e-9 * max(1.0, abs(acc))
                 assert abs(Sabs[t, j, o] - sum(abs(wd[o, k] * xf[t, k]) for k in range(256))) <= 1e-9 * max(1.0, Sabs[t, j, o])
+
+
+# ------------------------------------------------------- dequantizer floor
+
+def _nonzero_index_streams(rng, fmt, rows, cols):
+    """Random streams in which no sub-block has scale index 0, so every field
+    of a 16-weight group moves at least one of its dequantized values."""
+    w = S.random_streams(rng, fmt, 2, rows, cols)
+    if fmt == "iq2_ks":
+        w.sch[:] = 0  # index = low nibble - 16, never 0
+    else:
+        for n in range(8):  # nibble 8 (index 0) -> 9
+            nib = (w.scl >> np.uint32(4 * n)) & np.uint32(15)
+            w.scl ^= np.where(nib == 8, np.uint32(1 << (4 * n)), np.uint32(0)).astype(np.uint32)
+    return w
+
+
+@pytest.mark.parametrize("fmt", ["iq2_ks", "iq2_k"])
+def test_dequant_floor_reads_what_the_dequantizer_reads(fmt):
+    """Flipping every bit of one element of any stream changes the floor's
+    output in exactly the 16-weight groups whose dequantized values change
+    (the pinned dequantizer decides which), for the float32 and the bfloat16
+    layouts alike: no loaded field is dropped, none is read at the wrong
+    place, and nothing else reaches the output."""
+    rng = S.rng_for(31)
+    rows, cols = 3, 512
+    vals = np.array([3, -5, 7, -11, 13, -17, 19, -23], np.float32)  # distinct, non-zero
+    w = _nonzero_index_streams(rng, fmt, rows, cols)
+    d0 = O.dequant_expert(w, 1, vals).view(np.uint32).reshape(rows, cols // 16, 16)
+    f0 = O.dequant_floor(w, 1).reshape(rows, cols // 16, 16)
+    b0 = O.dequant_floor(w, 1, bf16=True).reshape(rows, cols // 16, 8)
+    assert np.array_equal(f0 ^ f0[..., :1], np.broadcast_to(np.arange(16, dtype=np.uint32), f0.shape))
+    assert np.array_equal(b0 ^ b0[..., :1], np.broadcast_to(np.arange(8, dtype=np.uint32), b0.shape))
+    for name in ("qs", "scl", "sch", "sex", "dv"):
+        arr = getattr(w, name)
+        if arr is None:
+            continue
+        flat = arr[1].reshape(-1)
+        for pos in rng.choice(flat.size, size=min(6, flat.size), replace=False):
+            saved = flat[pos]
+            flat[pos] = saved ^ np.iinfo(arr.dtype).max
+            arr[1] = flat.reshape(arr[1].shape)
+            d1 = O.dequant_expert(w, 1, vals).view(np.uint32).reshape(rows, cols // 16, 16)
+            f1 = O.dequant_floor(w, 1).reshape(rows, cols // 16, 16)
+            b1 = O.dequant_floor(w, 1, bf16=True).reshape(rows, cols // 16, 8)
+            flat[pos] = saved
+            arr[1] = flat.reshape(arr[1].shape)
+            moved = np.any(d1 != d0, axis=2)
+            assert moved.any(), (name, pos)
+            assert np.array_equal(np.any(f1 != f0, axis=2), moved), (name, pos)
+            assert np.array_equal(np.any(b1 != b0, axis=2), moved), (name, pos)
+
+
+@pytest.mark.parametrize("fmt", ["iq2_ks", "iq2_k"])
+def test_dequant_floor_of_empty_streams_is_the_word_index(fmt):
+    """All-zero streams fold to 0, so output word k of every group is k."""
+    w = S.empty_streams(fmt, 1, 2, 256)
+    assert np.array_equal(O.dequant_floor(w, 0), np.tile(np.arange(16, dtype=np.uint32), (2, 16)))
+    assert np.array_equal(O.dequant_floor(w, 0, bf16=True), np.tile(np.arange(8, dtype=np.uint32), (2, 16)))
