@@ -338,7 +338,7 @@ def gemv_leg(torch, B, cfg, device, stream, calls=200):
 # iqk_floor over the same experts, and the dequantizer (iqk_dequant) against
 # iqk_dequant_floor (same loads and same stores). Arms alternate inside a
 # cell. Declared gates:
-PRICE_BAR = {"decode": 2.5, "dequant": 1.10}  # kernel time / own floor time, at most
+PRICE_BAR = {"decode": 3.0, "dequant": 1.10}  # kernel time / own floor time, at most
 FLOOR_BAND = (0.15, 1.05)  # a floor arm streams at this fraction of the measured HBM copy rate
 PRICE_MIN_RATIO = 0.95  # a kernel clearly faster than its own floor skips loads the floor makes
 

@@ -294,3 +294,83 @@ def iqk_floor(w: Weights, expert_list, out=None, stream=None):
     _check(lib().iqk_floor(ctypes.byref(w.c), expert_list.data_ptr(), n, out.data_ptr(), _stream(stream)),
            "iqk_floor")
     return out
+
+
+# --------------------------------------------------------------- module form
+
+class IqkSwitchLinear:
+    """The switch-linear projection of the mlx-iqk 0.1.1 page (section
+    "Surface"): ``proj = IqkSwitchLinear(member, num_experts, out_features,
+    in_features, values)``, ``proj.load_streams(streams)``, ``y = proj(x,
+    indices)`` with ``y[..., j, :] = W_{indices[..., j]} x[...]``.
+
+    The member (``"iq2_ks"`` or ``"iq2_k"``) is fixed per instance, so the
+    projections of one layer can carry different members. ``values`` is the
+    8-entry value table (entries 0-3 alphabet 0, 4-7 alphabet 1); the page
+    does not print it, so it is an argument. Every call goes through
+    ``iqk_switch_linear``: its auto mode runs the decode kernel for few
+    (token, slot) pairs and the grouped GEMM for many. Both group the pairs by
+    expert on the device, so each expert's weights are read once per call
+    whatever ``sorted_indices`` says; the flag is accepted for interface
+    parity and changes nothing.
+
+    Errors: widths that are not a positive multiple of 256 and mismatched
+    streams raise ValueError before any launch; a shape the kernels do not
+    take raises RuntimeError. Ids outside [0, num_experts) give zero rows and
+    make ``status()`` report IQK_EINVAL.
+    """
+
+    def __init__(self, member: str, num_experts: int, out_features: int, in_features: int, values,
+                 device="cuda"):
+        if member not in FMT:
+            raise ValueError(f"unknown member {member!r} (expected one of {sorted(FMT)})")
+        if in_features <= 0 or in_features % 256:
+            raise ValueError(f"in_features {in_features} is not a positive multiple of 256")
+        if out_features <= 0 or num_experts <= 0:
+            raise ValueError("out_features and num_experts must be positive")
+        self.member, self.num_experts = member, num_experts
+        self.out_features, self.in_features = out_features, in_features
+        self.values = _values(values)
+        self.device = device
+        self.weights: Optional[Weights] = None
+        self._ws = {}
+        self._last_ws = None
+
+    def load_streams(self, streams) -> "IqkSwitchLinear":
+        """Take host streams (fmt, experts, rows, cols and the five planes) or
+        device ``Weights``; their member and shape must match the instance."""
+        got = (streams.fmt, streams.experts, streams.rows, streams.cols)
+        want = (self.member, self.num_experts, self.out_features, self.in_features)
+        if got != want:
+            raise ValueError(f"streams are {got}, the projection is {want}")
+        self.weights = streams if isinstance(streams, Weights) else Weights.from_host(streams, self.device)
+        return self
+
+    def __call__(self, x, indices, sorted_indices: bool = False, mode: int = 0, stream=None):
+        if self.weights is None:
+            raise RuntimeError("IqkSwitchLinear: load_streams() first")
+        torch = _torch()
+        if x.dtype != torch.bfloat16 or x.shape[-1] != self.in_features:
+            raise ValueError(f"x must be bfloat16 [..., {self.in_features}]")
+        if indices.shape[:-1] != x.shape[:-1]:
+            raise ValueError("indices must be [..., k] over the same leading shape as x")
+        lead, k = tuple(x.shape[:-1]), indices.shape[-1]
+        xt = x.reshape(-1, self.in_features).contiguous()
+        ids = indices.reshape(-1, k).to(torch.int32).contiguous()
+        T = xt.shape[0]
+        key = (mode, T, k)
+        ws = self._ws.get(key)
+        if ws is None:
+            need = iqk_switch_linear_workspace_bytes(mode, T, k, self.num_experts, self.out_features,
+                                                     self.in_features)
+            if need == 0:
+                raise RuntimeError(f"IqkSwitchLinear: mode {mode} cannot take {T} tokens x {k} slots")
+            ws = self._ws[key] = workspace(need, x.device)
+        self._last_ws = ws
+        y = iqk_switch_linear(self.weights, self.values, xt, ids, mode=mode, ws=ws, stream=stream)
+        return y.reshape(*lead, k, self.out_features)
+
+    def status(self, stream=None) -> int:
+        """Status of the last call as iqk_moe_status reports it: IQK_OK,
+        IQK_EINVAL (an id was out of range), IQK_EUNSUPPORTED or IQK_ETIMEOUT."""
+        return 0 if self._last_ws is None else iqk_moe_status(self._last_ws, stream)

@@ -349,6 +349,9 @@ __global__ void __launch_bounds__(256) k_prep(const uint16_t* __restrict__ x, in
                                               int nzero, const int32_t* __restrict__ ids, int npairs, int E,
                                               int32_t* __restrict__ status) {
   griddep_launch();
+  // Launched as a dependent of the previous call's down kernel: everything
+  // below writes workspace that kernel may still use.
+  griddep_wait();
   const int tid = blockIdx.x * blockDim.x + threadIdx.x;
   const int nth = gridDim.x * blockDim.x;
   for (int i = tid; i < nzero; i += nth) zero[i] = 0;
@@ -611,7 +614,9 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, kDecodeMinBlocks(NT)) k_str
     }
   };
   for (int s = 0; s < kStages; s++) issue(s);
-  if (MODE == MODE_GATEUP) griddep_launch();
+  // Dependents may launch now: the next kernel of a call waits before it
+  // writes, and the first kernel of the next call (prep or zeroing) too.
+  griddep_launch();
   // Results of the preceding kernel in the stream (the prep kernel's counters,
   // transposed activations and status word; the gate/up kernel's h) are read
   // only after griddepcontrol.wait. The raw activation rows are inputs of the
@@ -649,7 +654,7 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, kDecodeMinBlocks(NT)) k_str
       dst[1] = make_uint4(o[4], o[5], o[6], o[7]);
     }
     __syncthreads();
-  } else {
+  } else if (MODE != MODE_FLOOR) {  // the floor reads no activations: it waits before its first atomic
     griddep_wait();
     waited = true;
   }
@@ -847,6 +852,10 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, kDecodeMinBlocks(NT)) k_str
             uv += __ldcg(ub + ((size_t)ss * NC + col) * kTile + r);
           }
           const float h = gv / (1.0f + __expf(-gv)) * uv;
+          if (!waited) {  // h may still be read by the previous call's down kernel
+            griddep_wait();
+            waited = true;
+          }
           A.out16[(size_t)rt.sorted[p0 + col] * rows + perm16(f)] = f32_to_bf16_bits(h);
         }
     } else {
@@ -1016,7 +1025,10 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, kDecodeMinBlocks(NT)) k_til
     issued = q + 1;
   };
   for (int q = 0; q < kStages; q++) issue(q);
-  if (MODE == MODE_GATEUP) griddep_launch();
+  // gate/up lets its down kernel launch; the last kernel of a call lets the
+  // next call's prep (which waits before writing) and first kernel start
+  // their weight loads early
+  griddep_launch();
   // The raw activation rows are inputs of the call and can be read before the
   // dependency wait; h (DOWN) is the preceding kernel's result.
   bool waited = false;
@@ -1055,6 +1067,10 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, kDecodeMinBlocks(NT)) k_til
     __syncthreads();
   }
   if (MODE == MODE_SWITCH && rt.scalars[1] < npairs) {  // out-of-range ids: zero rows
+    if (!waited) {  // y may still be written by the previous call
+      griddep_wait();
+      waited = true;
+    }
     for (int pr = 0; pr < npairs; pr++) {
       if (rt.ids[pr] >= 0) continue;
       for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < rows; i += gridDim.x * blockDim.x)
@@ -1152,6 +1168,10 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, kDecodeMinBlocks(NT)) k_til
       const int tile = tg - u * tiles;
       const int p0 = rt.ustart[u];
       const int ncols = min(rt.ustart[u + 1] - p0, NC);  // more columns: reported as overflow
+      if (!waited) {  // h may still be read by the previous call's down kernel
+        griddep_wait();
+        waited = true;
+      }
       for (int o = threadIdx.x; o < ncols * kTile; o += blockDim.x) {
         const int col = o / kTile, row = o - col * kTile;
         const int f = tile * kTile + row;
@@ -1172,6 +1192,10 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, kDecodeMinBlocks(NT)) k_til
       const int p0 = rt.ustart[u];
       const int ncols = min(rt.ustart[u + 1] - p0, NC);
       const int per = ncols * kTile;
+      if (!waited) {  // y may still be written by the previous call
+        griddep_wait();
+        waited = true;
+      }
       for (int o = threadIdx.x; o < tpg * per; o += blockDim.x) {
         const int sub = o / per, rem = o - sub * per;
         const int col = rem / kTile, row = rem - col * kTile;
@@ -1304,6 +1328,29 @@ static cudaLaunchAttribute pdl_attr() {
   return a;
 }
 
+// The prep kernel as a programmatic dependent of whatever precedes it on the
+// stream (the previous call's last kernel triggers early); it waits before
+// its first write.
+static int launch_prep(int blocks, cudaStream_t st, const uint16_t* x, int T, int cols, uint16_t* xp, int32_t* zero,
+                       int nzero, const int32_t* ids, int npairs, int E, int32_t* status) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(blocks);
+  cfg.blockDim = dim3(256);
+  cfg.stream = st;
+  cudaLaunchAttribute at[1] = {pdl_attr()};
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, k_prep, x, T, cols, xp, zero, nzero, ids, npairs, E, status) == cudaSuccess ? 0 : -4;
+}
+
+// Zeroes n words after the preceding kernel completes (programmatic
+// dependent, like the prep kernel).
+__global__ void __launch_bounds__(256) k_zero(uint32_t* __restrict__ out, size_t n) {
+  griddep_launch();
+  griddep_wait();
+  for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x) out[i] = 0u;
+}
+
 GemvWs gemv_ws(int T, int rows, int cols) {
   GemvWs ws;
   const int tiles = (rows + kTile - 1) / kTile;
@@ -1420,8 +1467,7 @@ static int gemv_impl(const WDev& w, int expert, const Values& V, const uint16_t*
   const int tiles = (w.rows + kTile - 1) / kTile;
   const int pblocks = std::max(1, std::min(num_sms, (int)(((int64_t)T * (w.cols / 16) + 63) / 64)));
   const int nzero = (int)((L.part - L.cnt) / 4);  // the tile counters
-  k_prep<<<pblocks, 256, 0, st>>>(x, T, w.cols, xp, cnt, nzero, nullptr, 0, 1, status);
-  if (cudaGetLastError() != cudaSuccess) return -4;
+  if (launch_prep(pblocks, st, x, T, w.cols, xp, cnt, nzero, nullptr, 0, 1, status)) return -4;
   a.w0 = w;
   a.w1 = w;
   a.V = V;
@@ -1493,8 +1539,7 @@ static int decode_impl(const WDev& g, const WDev& u, const WDev& d, const Values
   int32_t* cnt3 = reinterpret_cast<int32_t*>(ws + L.cnt3);
   const int nzero = (int)((L.part2 - L.cnt2) / 4);  // both counter arrays
   const int pblocks = std::max(1, std::min(num_sms, (int)(((int64_t)T * (g.cols / 16) + 63) / 64)));
-  k_prep<<<pblocks, 256, 0, st>>>(x, T, g.cols, xp, cnt2, nzero, ids, npairs, g.experts, status);
-  if (cudaGetLastError() != cudaSuccess) return -4;
+  if (launch_prep(pblocks, st, x, T, g.cols, xp, cnt2, nzero, ids, npairs, g.experts, status)) return -4;
   a.w0 = g;
   a.w1 = u;
   a.V = V;
@@ -1585,8 +1630,7 @@ static int switch_impl(const WDev& w, const Values& V, const uint16_t* x, int T,
   int32_t* cnt = reinterpret_cast<int32_t*>(ws + L.cnt);
   const int tiles = (w.rows + kTile - 1) / kTile;
   const int pblocks = std::max(1, std::min(num_sms, (int)(((int64_t)T * (w.cols / 16) + 63) / 64)));
-  k_prep<<<pblocks, 256, 0, st>>>(x, T, w.cols, xp, cnt, tiles, ids, npairs, w.experts, status);
-  if (cudaGetLastError() != cudaSuccess) return -4;
+  if (launch_prep(pblocks, st, x, T, w.cols, xp, cnt, tiles, ids, npairs, w.experts, status)) return -4;
   a.w0 = w;
   a.w1 = w;
   a.V = V;
@@ -1629,7 +1673,17 @@ int launch_floor(const WDev& w, int fmt, const int32_t* experts, int n, uint32_t
   split_args(a, w.cols);
   CUtensorMap map;
   if (make_qs_map(&map, w, a.bpi)) return -4;
-  if (cudaMemsetAsync(out, 0, (size_t)n * w.rows * 4, st) != cudaSuccess) return -4;
+  {
+    const size_t nw = (size_t)n * w.rows;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)std::max<size_t>(1, std::min<size_t>((nw + 255) / 256, (size_t)num_sms)));
+    cfg.blockDim = dim3(256);
+    cfg.stream = st;
+    cudaLaunchAttribute at[1] = {pdl_attr()};
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, k_zero, out, nw) != cudaSuccess) return -4;
+  }
   a.w0 = w;
   a.w1 = w;
   a.elist = experts;
@@ -1639,8 +1693,8 @@ int launch_floor(const WDev& w, int fmt, const int32_t* experts, int n, uint32_t
   a.topk = 1;
   a.status = nullptr;  // the floor reports a timeout through g_floor_status
   const int items = n * ((w.rows + kTile - 1) / kTile) * a.splits;
-  if (fmt == FMT_KS) return launch_stream<MODE_FLOOR, FMT_KS, FMT_KS, 1, false>(map, map, a, items, st, num_sms, false);
-  return launch_stream<MODE_FLOOR, FMT_K, FMT_K, 1, false>(map, map, a, items, st, num_sms, false);
+  if (fmt == FMT_KS) return launch_stream<MODE_FLOOR, FMT_KS, FMT_KS, 1, false>(map, map, a, items, st, num_sms, true);
+  return launch_stream<MODE_FLOOR, FMT_K, FMT_K, 1, false>(map, map, a, items, st, num_sms, true);
 }
 
 }  // namespace iqk
