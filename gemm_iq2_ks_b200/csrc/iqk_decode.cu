@@ -299,7 +299,12 @@ __device__ __forceinline__ RouteView carve_route(uint8_t* p, int n) {
   return r;
 }
 
-__device__ __forceinline__ void build_route(const int32_t* __restrict__ ids, int n, int E, RouteView r) {
+// Distinct-expert list of a call. With `chunk`, an expert's pairs are split
+// into runs of at most `chunk` (each run its own entry u, so a tile kernel's
+// MMA columns always suffice; such an expert's weights are then read once per
+// run).
+__device__ __forceinline__ void build_route(const int32_t* __restrict__ ids, int n, int E, RouteView r,
+                                            int chunk = 1 << 30) {
   for (int p = threadIdx.x; p < n; p += blockDim.x) {
     const int e = ids[p];
     r.ids[p] = (e >= 0 && e < E) ? e : -1;
@@ -325,16 +330,25 @@ __device__ __forceinline__ void build_route(const int32_t* __restrict__ ids, int
   for (int k = threadIdx.x; k < nv; k += blockDim.x)
     r.first[k] = (k == 0) || (r.ids[r.sorted[k - 1]] != r.ids[r.sorted[k]]);
   __syncthreads();
+  if (chunk < nv) {  // bit 1: a run start inside an expert (bit 0, read here, stays put)
+    for (int k = threadIdx.x; k < nv; k += blockDim.x) {
+      if (r.first[k] & 1) continue;
+      int j = k;
+      while (!(r.first[j] & 1)) j--;
+      if ((k - j) % chunk == 0) r.first[k] |= 2;
+    }
+    __syncthreads();
+  }
   for (int k = threadIdx.x; k < nv; k += blockDim.x) {
     if (!r.first[k]) continue;
     int u = 0;
-    for (int q = 0; q < k; q++) u += r.first[q];
+    for (int q = 0; q < k; q++) u += r.first[q] != 0;
     r.uexp[u] = r.ids[r.sorted[k]];
     r.ustart[u] = (int16_t)k;
   }
   if (threadIdx.x == 0) {
     int D = 0;
-    for (int q = 0; q < nv; q++) D += r.first[q];
+    for (int q = 0; q < nv; q++) D += r.first[q] != 0;
     r.scalars[0] = D;
     r.ustart[D] = (int16_t)nv;
   }
@@ -972,7 +986,7 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, kDecodeMinBlocks(NT)) k_til
     fence_mbar_init();
   }
   const RouteView rt = carve_route(route_p, npairs);
-  build_route(A.ids, npairs, A.w0.experts, rt);  // ends with __syncthreads
+  build_route(A.ids, npairs, A.w0.experts, rt, NC);  // ends with __syncthreads; runs of <= NC pairs
   const int D = rt.scalars[0];
   const int rows = A.w0.rows;
   const int tiles = (rows + kTile - 1) / kTile;
@@ -1274,6 +1288,21 @@ static size_t tiles_smem(int cols, int T, int npairs, int act_rows) {
 
 static int nt_for(int cols_needed) { return cols_needed <= 8 ? 1 : cols_needed <= 16 ? 2 : cols_needed <= 32 ? 4 : 8; }
 
+// MMA column groups of a routed call. The tile kernels split an expert's
+// pairs into runs of 8 * NT, so one group serves any routing; two pay off
+// only when experts average more than 8 pairs (fewer weight re-reads).
+// Calls above 64 tokens use the stream kernel at nt_for(T).
+static int routed_nt(int T, int npairs, int E) {
+  if (T > 64) return nt_for(T);
+  const int distinct = std::max(1, std::min(E, npairs));
+  return (npairs + distinct - 1) / distinct > 8 ? 2 : 1;
+}
+
+// Upper bound on the tile kernels' run count (distinct experts plus splits).
+static int route_runs_max(int npairs, int E, int NT) {
+  return std::min(npairs, std::min(E, npairs) + npairs / (8 * NT));
+}
+
 // Per (kernel, dynamic smem) caches so that a call made during stream
 // capture issues no attribute or occupancy queries after the first call.
 struct KernelCache {
@@ -1557,8 +1586,9 @@ static int decode_impl(const WDev& g, const WDev& u, const WDev& d, const Values
   if constexpr (NT <= 2) {
     const int ar = act_rows_smem(NT, T, g.cols);
     a.act_rows = ar;
-    rc = ar ? launch_tiles<MODE_GATEUP, FG, FU, NT, true>(mg, mu, a, L.dmax * L.c2.tiles, st, num_sms, true)
-            : launch_tiles<MODE_GATEUP, FG, FU, NT, false>(mg, mu, a, L.dmax * L.c2.tiles, st, num_sms, true);
+    const int groups = route_runs_max(npairs, g.experts, NT) * L.c2.tiles;
+    rc = ar ? launch_tiles<MODE_GATEUP, FG, FU, NT, true>(mg, mu, a, groups, st, num_sms, true)
+            : launch_tiles<MODE_GATEUP, FG, FU, NT, false>(mg, mu, a, groups, st, num_sms, true);
   } else {
     rc = launch_stream_any<MODE_GATEUP, FG, FU, NT>(mg, mu, a, L.dmax * 2 * L.c2.tiles * a.splits, st, num_sms, true,
                                                     0);
@@ -1584,7 +1614,7 @@ static int decode_impl(const WDev& g, const WDev& u, const WDev& d, const Values
 int launch_moe_decode(const WDev& g, int fg, const WDev& u, int fu, const WDev& d, int fd, const Values& V,
                       const uint16_t* x, int T, const int32_t* ids, const float* p, int topk, uint16_t* y, char* ws,
                       cudaStream_t st, int num_sms) {
-  const int NT = nt_for(T);
+  const int NT = routed_nt(T, T * topk, g.experts);
   const int key = fg * 4 + fu * 2 + fd;
 #define IQK_DEC(G, U, D, N)                  \
   if (key == G * 4 + U * 2 + D && NT == N) \
@@ -1646,7 +1676,7 @@ static int switch_impl(const WDev& w, const Values& V, const uint16_t* x, int T,
   if constexpr (NT <= 2) {
     // tile kernel: a group is tpg tiles of one expert, splits * tpg <= warps items
     a.tpg = std::max(1, kDecodeWarps / a.splits);
-    const int groups = dmax * ((tiles + a.tpg - 1) / a.tpg);
+    const int groups = route_runs_max(npairs, w.experts, NT) * ((tiles + a.tpg - 1) / a.tpg);
     const int ar = act_rows_smem(NT, T, w.cols);
     a.act_rows = ar;
     a.xraw = x;
@@ -1658,7 +1688,7 @@ static int switch_impl(const WDev& w, const Values& V, const uint16_t* x, int T,
 
 int launch_switch_decode(const WDev& w, int fmt, const Values& V, const uint16_t* x, int T, const int32_t* ids,
                          int topk, float* y, char* ws, cudaStream_t st, int num_sms) {
-  const int NT = nt_for(T);
+  const int NT = routed_nt(T, T * topk, w.experts);
 #define IQK_SW(F, N) \
   if (fmt == F && NT == N) return switch_impl<F, N>(w, V, x, T, ids, topk, y, ws, st, num_sms);
   IQK_SW(FMT_KS, 1) IQK_SW(FMT_KS, 2) IQK_SW(FMT_KS, 4) IQK_SW(FMT_KS, 8)

@@ -175,19 +175,22 @@ int iqk_gemv(const iqk_weights* w, int32_t expert, const float* values /* host [
  *   ids: device int32 [T][topk]; y: device float32 [T][topk][rows],
  *        16-byte aligned; 1 <= topk <= 16.
  *   mode 1: the decode-style kernel (T <= 64, T * topk <= 1024): one weight
- *           read per distinct expert, shared by its pairs;
+ *           read per run of at most 8 (or 16) pairs of one expert, shared
+ *           by the run's pairs;
  *   mode 2: grouped by expert, tcgen05 grouped GEMM (rows a multiple of 256,
  *           T <= 65536);
  *   mode 0: mode 1 up to IQK_SWITCH_DECODE_MAX_PAIRS pairs, else mode 2 (the
  *           page's switch linear also picks its kernel by pair count; the
- *           crossover here is measured, see the design notes).
+ *           crossover is measured on B200 at the routed gate geometry,
+ *           2048 x 4096 with 256 experts: mode 1 is faster up to 64 tokens
+ *           at top-6, 384 pairs).
  * Accuracy as iqk_gemv. Out-of-range ids give zero rows and set bit 0 of the
  * status word (iqk_moe_status reads it from this workspace too).
  * workspace: >= iqk_switch_linear_workspace_bytes(mode, T, topk, E, rows,
  * cols) bytes (0 means the mode cannot take the shape), 256-byte aligned.
  * Returns IQK_EUNSUPPORTED when the chosen mode cannot take the shape.
  */
-#define IQK_SWITCH_DECODE_MAX_PAIRS 96
+#define IQK_SWITCH_DECODE_MAX_PAIRS 384
 size_t iqk_switch_linear_workspace_bytes(int32_t mode, int32_t T, int32_t topk, int32_t experts, int32_t rows,
                                          int32_t cols);
 int iqk_switch_linear(const iqk_weights* w, const float* values /* host [8] */, const uint16_t* x, int32_t T,

@@ -253,8 +253,8 @@ def test_dequant_floor_bitexact(B, fmt, rows, cols, bf16):
 
 def test_moe_decode_duplicate_ids(B):
     """A token listing one expert twice: both slots are computed as separate
-    pairs while the expert's pairs fit the MMA columns; beyond that the call
-    reports IQK_EUNSUPPORTED through the status word."""
+    pairs. One token listing one expert in all twelve slots: more pairs than
+    one MMA column group, split into runs, each run a separate pass."""
     gate, up, down, x, ids, p = _moe_case(77, "iq2_ks", "iq2_ks", "iq2_ks", E=12, H=512, F=768, T=2, topk=4)
     ids = ids.copy()
     ids[0, 1] = ids[0, 0]
@@ -266,10 +266,23 @@ def test_moe_decode_duplicate_ids(B):
                          torch.from_numpy(p).cuda(), ws=ws)
     assert B.iqk_moe_status(ws) == B.IQK_OK
     check_moe(from_dev_bf16(y), O.moe(gate, up, down, vals, x, ids, p), "duplicate ids")
-    # one token, twelve slots on the same expert: more pairs than the 8 MMA columns
     ids12 = np.full((1, 12), 5, np.int32)
     p12 = np.full((1, 12), 1.0 / 12, np.float32)
     ws12 = B.workspace(B.iqk_moe_workspace_bytes(0, 1, 12, 12, 512, 768))
-    B.iqk_moe_decode(dg, du, dd, vals, to_dev_bf16(x[:1]), torch.from_numpy(ids12).cuda(),
-                     torch.from_numpy(p12).cuda(), ws=ws12)
-    assert B.iqk_moe_status(ws12) == B.IQK_EUNSUPPORTED
+    y12 = B.iqk_moe_decode(dg, du, dd, vals, to_dev_bf16(x[:1]), torch.from_numpy(ids12).cuda(),
+                           torch.from_numpy(p12).cuda(), ws=ws12)
+    assert B.iqk_moe_status(ws12) == B.IQK_OK
+    check_moe(from_dev_bf16(y12), O.moe(gate, up, down, vals, x[:1], ids12, p12), "twelve slots, one expert")
+
+
+@pytest.mark.parametrize("T,topk,E,dup", [(2, 10, 20, True), (33, 6, 12, False), (40, 4, 64, False)])
+def test_moe_decode_runs_of_pairs(B, T, topk, E, dup):
+    """Experts with more pairs than the MMA columns: split into runs (one
+    column group when experts average at most 8 pairs, two otherwise)."""
+    gate, up, down, x, ids, p = _moe_case(300 + T, "iq2_k", "iq2_ks", "iq2_ks", E=E, H=512, F=256, T=T, topk=topk)
+    if dup:  # token 0 puts one expert in every slot: 10 pairs, 2 runs of one column group
+        ids = ids.copy()
+        ids[0, :] = ids[1, 0]
+    values = S.value_table("f16", 6)
+    y = _run_decode(B, gate, up, down, values, x, ids, p)
+    check_moe(y, O.moe(gate, up, down, values, x, ids, p), f"decode runs T={T} topk={topk} E={E}")

@@ -71,11 +71,11 @@ def test_switch_out_of_range_id(B, mode):
     check_fp32(y, y_ref, Sabs, f"switch bad id mode {mode}")
 
 
-@pytest.mark.parametrize("T", [1, 64])
+@pytest.mark.parametrize("T", [1, 64, 100])
 def test_switch_auto_config_geometry(B, T):
     """Gate-projection geometry of the routed block (2048 x 4096, 32 experts
-    resident); auto mode picks the decode kernel at 6 pairs and the grouped
-    GEMM at 384. Sampled rows are checked against the oracle."""
+    resident); auto mode picks the decode kernel at 6 and 384 pairs and the
+    grouped GEMM at 600. Sampled rows are checked against the oracle."""
     w, x, ids = _case(120 + T, "iq2_ks", 32, 2048, 4096, T, 6)
     vals = S.value_table("int", 8)
     y, st = _run(B, w, x, ids, vals, mode=0)
@@ -117,3 +117,18 @@ def test_switch_decode_duplicate_slot(B):
     assert st == 0
     check_fp32(y, y_ref, Sabs, "switch decode duplicate slot")
     assert np.array_equal(y[0, 0], y[0, 2])
+
+
+@pytest.mark.parametrize("T,topk,E", [(1, 12, 4), (40, 6, 10), (64, 6, 256)])
+def test_switch_decode_runs_of_pairs(B, T, topk, E):
+    """More pairs per expert than one MMA column group (split into runs), and
+    the mid-size token counts the decode kernel now takes."""
+    rng = S.rng_for(220 + T)
+    w = S.random_streams(rng, "iq2_k", E, 96, 512)
+    x = S.random_bf16(rng, (T, 512))
+    ids = rng.integers(0, E, size=(T, topk)).astype(np.int32)  # repeats within a token allowed
+    vals = S.value_table("int", 11)
+    y, st = _run(B, w, x, ids, vals, mode=1)
+    y_ref, Sabs = O.switch_linear(w, vals, x, ids)
+    assert st == 0
+    check_fp32(y, y_ref, Sabs, f"switch decode runs T={T} topk={topk} E={E}")
