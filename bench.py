@@ -38,7 +38,7 @@ RING = 420  # calls per captured graph (10 permutation cycles of 42 calls)
 # DRAM bytes (read + write) of the two tile kernels of one config-2 decode
 # call, from one ncu capture of `bench.py --profile decode --experts 24`
 # (profiles/decode_config2_tile_kernels.md); per call, not per resident expert.
-DECODE_CALL_TRAFFIC = 41_574_912
+DECODE_CALL_TRAFFIC = 41_575_424
 
 
 def env_int(k, d):

@@ -230,7 +230,6 @@ int iqk_moe_status(const void* workspace, void* stream) {
   e = cudaMemcpy(&s, workspace, 4, cudaMemcpyDeviceToHost);
   if (e != cudaSuccess) return cuda_fail(e);
   if (s & 2) return IQK_ETIMEOUT;
-  if (s & 8) return IQK_EUNSUPPORTED;
   if (s & 1) return IQK_EINVAL;
   return IQK_OK;
 }

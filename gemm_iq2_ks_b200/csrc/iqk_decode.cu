@@ -397,22 +397,20 @@ __global__ void __launch_bounds__(256) k_prep(const uint16_t* __restrict__ x, in
   }
 }
 
-// ------------------------------------------------------------ stream kernel
-// One kernel for the GEMV-shaped jobs and the floor arm. An item is 16 rows
-// of one matrix over a slice of `bpi` blocks of the reduction width; its
-// columns are the tokens (GEMV) or the (token, slot) pairs routed to one
-// distinct expert. Each warp streams its items through a ring of kStages
-// stages, one item per stage, so loads run up to kStages items ahead of the
-// decode.
+// ------------------------------------------------------- kernel modes
+// An item is 16 rows of one matrix over a slice of `bpi` blocks of the
+// reduction width; its MMA columns are the tokens (GEMV) or the (token, slot)
+// pairs of one run of a distinct expert (routed modes). Each warp streams
+// its items through a ring of kStages stages, one item per stage, so loads
+// run up to kStages items ahead of the decode.
+//   stream kernel (items spread over every warp of the grid):
 //   GEMV:   slices of a tile meet in the workspace; y[t][row] = sum (fp32).
-//   GATEUP: gate and up slices of a tile write partials; the tile's last
-//           item forms h = bf16(silu(g) * u) in the slot-transposed layout.
-//   DOWN:   partials per (tile, pair, slice); the tile's last item sums each
-//           token's slots in slot order, weighted by p, into y (bf16).
 //   FLOOR:  identical loads; the decode is replaced by an XOR of every loaded
 //           byte into out[expert][row].
-//   SWITCH: one projection per (token, slot) pair, no combine: the tile's
-//           last item writes y[pair][row] = sum over slices (fp32).
+//   tile kernel (a CTA reduces a group of items in shared memory):
+//   GATEUP: gate and up slices of a tile; h = bf16(silu(g) * u), slot-transposed.
+//   DOWN:   every run's slices of a tile; y = sum_j p_j * (...), bf16.
+//   SWITCH: one projection per (token, slot) pair; y[pair][row] (fp32).
 enum : int { MODE_GEMV = 0, MODE_GATEUP = 1, MODE_DOWN = 2, MODE_FLOOR = 3, MODE_SWITCH = 4 };
 
 struct UnitArgs {
@@ -425,7 +423,7 @@ struct UnitArgs {
   int T, topk, expert;
   const int32_t* elist;  // FLOOR: experts to stream
   int nexp;
-  float* yf;        // GEMV output [T][rows]
+  float* yf;        // GEMV output [T][rows]; SWITCH output [pairs][rows]
   uint16_t* out16;  // GATEUP: h [pairs][inter]; DOWN: y [T][hidden]
   uint32_t* outx;   // FLOOR: [nexp][rows], zeroed before the launch
   int32_t* cnt;
@@ -530,18 +528,6 @@ __device__ __forceinline__ void stage_scales(uint8_t* slot, const WDev& w, int64
   __syncwarp();
 }
 
-// A distinct expert can collect more pairs than the launch's MMA columns only
-// when a token lists it more than once; those extra pairs are not computed.
-// Bit 3 of the status word reports it (after the dependency wait, so it is
-// ordered after the prep kernel's store of the word).
-__device__ __forceinline__ void report_column_overflow(const RouteView& rt, int D, int NC, int32_t* status) {
-  for (int u = 0; u < D; u++)
-    if (rt.ustart[u + 1] - rt.ustart[u] > NC) {
-      atomicOr(status, 8);
-      return;
-    }
-}
-
 // Timeout flag of the floor arm, which has no workspace; read with
 // cudaMemcpyFromSymbol when diagnosing.
 __device__ int32_t g_floor_status;
@@ -550,6 +536,7 @@ template <int MODE, int F0, int F1, int NT, bool BSM>
 __global__ void __launch_bounds__(kDecodeWarps * 32, kDecodeMinBlocks(NT)) k_stream(const __grid_constant__ CUtensorMap m0,
                                                                          const __grid_constant__ CUtensorMap m1,
                                                                          const __grid_constant__ UnitArgs A) {
+  static_assert(MODE == MODE_GEMV || MODE == MODE_FLOOR, "stream kernel: GEMV or floor");
   extern __shared__ __align__(128) uint8_t smem[];
   const int wid = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
   const int K = A.w0.cols;
@@ -559,7 +546,6 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, kDecodeMinBlocks(NT)) k_str
   const uint32_t slot_b = slot_bytes2<F0, F1>(bpi);
   const uint32_t k65536 = opaque_u32(65536u);
   constexpr int NC = 8 * NT;
-  const int npairs = A.T * A.topk;
   const size_t warp_bytes = (size_t)kStages * (stage_words * 4 + slot_b);
   uint32_t* ring_qs = reinterpret_cast<uint32_t*>(smem + wid * warp_bytes);
   uint8_t* ring_slots = smem + wid * warp_bytes + (size_t)kStages * stage_words * 4;
@@ -571,97 +557,66 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, kDecodeMinBlocks(NT)) k_str
   // BSM rows keep each lane's 64-element segment in 80 elements (160 bytes),
   // so the four segments a warp reads at once start in different bank groups
   const int KP = BSM ? K / 64 * 80 : K;  // activation row stride (elements)
-  uint8_t* route_p = reinterpret_cast<uint8_t*>(act_s) + (BSM ? (size_t)A.act_rows * KP * 2 : 0);
-  if (MODE != MODE_FLOOR) {
-    build_lut<F0>(lut0, A.V);
-    if (MODE == MODE_GATEUP) build_lut<F1>(lut1, A.V);
-  }
+  if (MODE == MODE_GEMV) build_lut<F0>(lut0, A.V);
   if (lane == 0) {
     for (int s = 0; s < kStages; s++) mbar_init(&bar[s], 1);
     fence_mbar_init();
   }
-  RouteView rt{};
-  int D = 1;
-  if (MODE == MODE_GATEUP || MODE == MODE_DOWN || MODE == MODE_SWITCH) {
-    rt = carve_route(route_p, npairs);
-    build_route(A.ids, npairs, A.w0.experts, rt);  // ends with __syncthreads
-    D = rt.scalars[0];
-  } else {
-    if (MODE == MODE_FLOOR) D = A.nexp;
-    __syncthreads();
-  }
-  constexpr int NMAT = MODE == MODE_GATEUP ? 2 : 1;
+  __syncthreads();
+  const int D = MODE == MODE_FLOOR ? A.nexp : 1;  // matrices streamed
   const int rows = A.w0.rows;
   const int tiles = (rows + kTile - 1) / kTile;
-  const int nitems = D * NMAT * tiles * S;
+  const int nitems = D * tiles * S;
   const int W = gridDim.x * kDecodeWarps;
   const int gw = blockIdx.x * kDecodeWarps + wid;
-  // item id -> (u, tile, mat, s): the slices of a tile, then gate / up, are adjacent
-  auto item_of = [&](int id, int& u, int& mat, int& tile, int& s) {
-    int r = (int)A.div_s.div((uint32_t)id);
+  // item id -> (u, tile, s): the slices of a tile are adjacent
+  auto item_of = [&](int id, int& u, int& tile, int& s) {
+    const int r = (int)A.div_s.div((uint32_t)id);
     s = id - r * S;
-    mat = r % NMAT;
-    r /= NMAT;
     u = (int)A.div_tiles.div((uint32_t)r);
     tile = r - u * tiles;
   };
-  auto expert_of = [&](int u) -> int {
-    if (MODE == MODE_GEMV) return A.expert;
-    if (MODE == MODE_FLOOR) return A.elist[u];
-    return rt.uexp[u];
-  };
+  auto expert_of = [&](int u) -> int { return MODE == MODE_FLOOR ? A.elist[u] : A.expert; };
   auto issue = [&](int it) {
     const int id = gw + it * W;
     if (id >= nitems) return;
     const int st = it % kStages;
-    int u, mat, tile, s;
-    item_of(id, u, mat, tile, s);
+    int u, tile, s;
+    item_of(id, u, tile, s);
     const int64_t R0 = (int64_t)expert_of(u) * rows + (int64_t)tile * kTile;
     const int valid = min(kTile, rows - tile * kTile);
     uint8_t* slot = ring_slots + (size_t)st * slot_b;
-    if (mat == 0) stage_scales<F0>(slot, A.w0, R0, valid, s, bpi, A.async_sc, &bar[st], lane);
-    else stage_scales<F1>(slot, A.w1, R0, valid, s, bpi, A.async_sc, &bar[st], lane);
+    stage_scales<F0>(slot, A.w0, R0, valid, s, bpi, A.async_sc, &bar[st], lane);
     __syncwarp();
     if (lane == 0) {
       mbar_arrive_expect_tx(&bar[st], (uint32_t)stage_words * 4);
-      tma_load_2d(ring_qs + (size_t)st * stage_words, mat ? &m1 : &m0, s * ldw, (int)R0, &bar[st]);
+      tma_load_2d(ring_qs + (size_t)st * stage_words, &m0, s * ldw, (int)R0, &bar[st]);
     }
   };
   for (int s = 0; s < kStages; s++) issue(s);
   // Dependents may launch now: the next kernel of a call waits before it
   // writes, and the first kernel of the next call (prep or zeroing) too.
   griddep_launch();
-  // Results of the preceding kernel in the stream (the prep kernel's counters,
-  // transposed activations and status word; the gate/up kernel's h) are read
-  // only after griddepcontrol.wait. The raw activation rows are inputs of the
-  // call, complete before the prep kernel started, so a BSM launch copies them
+  // Results of the preceding kernel in the stream (the prep kernel's counters
+  // and transposed activations) are read only after griddepcontrol.wait. The
+  // raw activation rows are inputs of the call, so a BSM launch copies them
   // first and defers the wait to its first epilogue.
   bool waited = false;
   if constexpr (BSM) {  // the call's activation rows, slot-transposed and padded, once per CTA
-    if (MODE == MODE_DOWN) {  // h comes from the gate/up kernel, already slot-transposed
-      griddep_wait();
-      waited = true;
-    }
     const int gpr = K / 16;  // 16-element groups per row
     const int groups = A.act_rows * gpr;
     for (int gi = threadIdx.x; gi < groups; gi += blockDim.x) {
       const int r = gi / gpr, c0 = (gi - r * gpr) * 16;
       uint32_t o[8];
-      if (MODE == MODE_DOWN) {
-        const uint4* src = reinterpret_cast<const uint4*>(A.act + (size_t)gi * 16);
-        const uint4 a = ld_nc_u4(src), b = ld_nc_u4(src + 1);
-        o[0] = a.x; o[1] = a.y; o[2] = a.z; o[3] = a.w; o[4] = b.x; o[5] = b.y; o[6] = b.z; o[7] = b.w;
-      } else {
-        const uint4* src = reinterpret_cast<const uint4*>(A.xraw + (size_t)gi * 16);
-        const uint4 a = ld_nc_u4(src), b = ld_nc_u4(src + 1);
-        const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+      const uint4* src = reinterpret_cast<const uint4*>(A.xraw + (size_t)gi * 16);
+      const uint4 a = ld_nc_u4(src), b = ld_nc_u4(src + 1);
+      const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
 #pragma unroll
-        for (int i2 = 0; i2 < 4; i2++) {
-          const int wa = i2 >> 1;
-          const uint32_t sel = (i2 & 1) ? 0x7632u : 0x5410u;
-          o[2 * i2] = prmt(w[wa], w[wa + 2], sel);
-          o[2 * i2 + 1] = prmt(w[wa + 4], w[wa + 6], sel);
-        }
+      for (int i2 = 0; i2 < 4; i2++) {
+        const int wa = i2 >> 1;
+        const uint32_t sel = (i2 & 1) ? 0x7632u : 0x5410u;
+        o[2 * i2] = prmt(w[wa], w[wa + 2], sel);
+        o[2 * i2 + 1] = prmt(w[wa + 4], w[wa + 6], sel);
       }
       uint4* dst = reinterpret_cast<uint4*>(act_s + (size_t)r * KP + (c0 >> 6) * 80 + (c0 & 63));
       dst[0] = make_uint4(o[0], o[1], o[2], o[3]);
@@ -672,14 +627,6 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, kDecodeMinBlocks(NT)) k_str
     griddep_wait();
     waited = true;
   }
-  if (MODE == MODE_DOWN && D == 0) {  // every id out of range: the block output is zero
-    for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < A.T * rows; i += gridDim.x * blockDim.x) A.out16[i] = 0;
-    return;
-  }
-  if (MODE == MODE_SWITCH && D == 0) {
-    for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < npairs * rows; i += gridDim.x * blockDim.x) A.yf[i] = 0.f;
-    return;
-  }
   const uint16_t* act_base = BSM ? act_s : A.act;
   constexpr int SEG = BSM ? 80 : 64;    // elements between the segments of lanes t and t + 1
   constexpr int BLKE = BSM ? 320 : 256;  // elements between consecutive 256-weight blocks
@@ -687,27 +634,18 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, kDecodeMinBlocks(NT)) k_str
   for (int it = 0;; it++) {
     const int id = gw + it * W;
     if (id >= nitems) break;
-    int u, mat, tile, s;
-    item_of(id, u, mat, tile, s);
-    int p0 = 0, ncols = A.T;
-    if (MODE == MODE_GATEUP || MODE == MODE_DOWN || MODE == MODE_SWITCH) {
-      p0 = rt.ustart[u];
-      ncols = rt.ustart[u + 1] - p0;
-    }
+    int u, tile, s;
+    item_of(id, u, tile, s);
     const uint16_t* bsrc[NT];
 #pragma unroll
     for (int n = 0; n < NT; n++) {
-      // columns past the last token or pair repeat column 0; their sums are never stored
-      const int col = 8 * n + g < ncols ? 8 * n + g : 0;
-      int arow = 0;
-      if (MODE == MODE_GEMV) arow = col;
-      else if (MODE == MODE_GATEUP || MODE == MODE_SWITCH) arow = rt.sorted[p0 + col] / A.topk;
-      else if (MODE == MODE_DOWN) arow = rt.sorted[p0 + col];
-      bsrc[n] = act_base + (size_t)arow * KP + (size_t)s * bpi * BLKE + SEG * t;
+      // columns past the last token repeat column 0; their sums are never stored
+      const int col = 8 * n + g < A.T ? 8 * n + g : 0;
+      bsrc[n] = act_base + (size_t)col * KP + (size_t)s * bpi * BLKE + SEG * t;
       if (!BSM && MODE != MODE_FLOOR) prefetch_l1(bsrc[n]);
     }
-    const bool fmt0 = (MODE != MODE_GATEUP) || mat == 0;
-    const bool kfmt = fmt0 ? (F0 == FMT_K) : (F1 == FMT_K);
+    const bool fmt0 = true;
+    const bool kfmt = F0 == FMT_K;
     const int st = it % kStages;
     if (!mbar_wait_bounded(&bar[st], (uint32_t)((it / kStages) & 1))) {
       if (!waited) griddep_wait();
@@ -834,95 +772,9 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, kDecodeMinBlocks(NT)) k_str
           for (int ss = 0; ss < S; ss++) sum += __ldcg(base + ((size_t)ss * NC + col) * kTile + r);
           A.yf[(size_t)col * rows + row] = sum;
         }
-    } else if (MODE == MODE_GATEUP) {
-      const size_t ut = (size_t)u * tiles + tile;
-      float* slotp = A.part + ((ut * 2 + mat) * S + s) * NC * kTile;
-#pragma unroll
-      for (int n = 0; n < NT; n++)
-#pragma unroll
-        for (int q = 0; q < 4; q++) slotp[(8 * n + 2 * t + (q & 1)) * kTile + g + 8 * (q >> 1)] = acc[n][q];
-      __syncwarp();
-      int prev = 0;
-      if (lane == 0) {
-        __threadfence();
-        prev = atomicAdd(A.cnt + ut, 1);
-      }
-      prev = __shfl_sync(0xffffffffu, prev, 0);
-      if (prev != 2 * S - 1) continue;
-      __threadfence();
-      const float* gb = A.part + (ut * 2) * S * NC * kTile;
-      const float* ub = gb + (size_t)S * NC * kTile;
-#pragma unroll
-      for (int n = 0; n < NT; n++)
-#pragma unroll
-        for (int q = 0; q < 4; q++) {
-          const int col = 8 * n + 2 * t + (q & 1);
-          const int r = g + 8 * (q >> 1);
-          const int f = tile * kTile + r;
-          if (col >= ncols || f >= rows) continue;
-          float gv = 0.f, uv = 0.f;
-          for (int ss = 0; ss < S; ss++) {
-            gv += __ldcg(gb + ((size_t)ss * NC + col) * kTile + r);
-            uv += __ldcg(ub + ((size_t)ss * NC + col) * kTile + r);
-          }
-          const float h = gv / (1.0f + __expf(-gv)) * uv;
-          if (!waited) {  // h may still be read by the previous call's down kernel
-            griddep_wait();
-            waited = true;
-          }
-          A.out16[(size_t)rt.sorted[p0 + col] * rows + perm16(f)] = f32_to_bf16_bits(h);
-        }
-    } else {
-      float* slab = A.part + (size_t)tile * npairs * S * kTile;
-#pragma unroll
-      for (int n = 0; n < NT; n++)
-#pragma unroll
-        for (int q = 0; q < 4; q++) {
-          const int col = 8 * n + 2 * t + (q & 1);
-          if (col >= ncols) continue;
-          const int pair = rt.sorted[p0 + col];
-          slab[((size_t)pair * S + s) * kTile + g + 8 * (q >> 1)] = acc[n][q];
-        }
-      __syncwarp();
-      int prev = 0;
-      if (lane == 0) {
-        __threadfence();
-        prev = atomicAdd(A.cnt + tile, 1);
-      }
-      prev = __shfl_sync(0xffffffffu, prev, 0);
-      if (prev != D * S - 1) continue;
-      __threadfence();
-      if (MODE == MODE_SWITCH) {  // every pair's rows of this tile (zero for out-of-range ids)
-        for (int o = lane; o < npairs * kTile; o += 32) {
-          const int pair = o / kTile, r = o % kTile;
-          const int row = tile * kTile + r;
-          if (row >= rows) continue;
-          float v = 0.f;
-          if (rt.ids[pair] >= 0)
-            for (int ss = 0; ss < S; ss++) v += __ldcg(slab + ((size_t)pair * S + ss) * kTile + r);
-          A.yf[(size_t)pair * rows + row] = v;
-        }
-        continue;
-      }
-      for (int o = lane; o < A.T * kTile; o += 32) {
-        const int tok = o / kTile, r = o % kTile;
-        const int row = tile * kTile + r;
-        if (row >= rows) continue;
-        float sum = 0.f;
-        for (int jj = 0; jj < A.topk; jj++) {
-          const int pair = tok * A.topk + jj;
-          if (rt.ids[pair] < 0) continue;
-          float v = 0.f;
-          for (int ss = 0; ss < S; ss++) v += __ldcg(slab + ((size_t)pair * S + ss) * kTile + r);
-          sum += __ldg(A.p + pair) * v;
-        }
-        A.out16[(size_t)tok * rows + row] = f32_to_bf16_bits(sum);
-      }
     }
   }
   if (!waited) griddep_wait();  // this grid completes only after the one it depends on
-  if ((MODE == MODE_GATEUP || MODE == MODE_DOWN || MODE == MODE_SWITCH) && blockIdx.x == 0 && threadIdx.x == 0)
-    report_column_overflow(rt, D, NC, A.status);
 }
 
 // ------------------------------------------------------------- tile kernel
@@ -1235,7 +1087,6 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, kDecodeMinBlocks(NT)) k_til
   // let copies still in flight land before the CTA exits (only after a timeout)
   for (int qd = consumed; qd < issued; qd++) (void)mbar_wait_bounded(&bar[qd % kStages], (uint32_t)((qd / kStages) & 1));
   if (!waited) griddep_wait();  // this grid completes only after the one it depends on
-  if (blockIdx.x == 0 && threadIdx.x == 0) report_column_overflow(rt, D, NC, A.status);
 }
 
 // ================================================================== host
@@ -1269,11 +1120,11 @@ int make_qs_map(CUtensorMap* map, const WDev& w, int nb) {
 constexpr size_t kActSmemMax = 40 * 1024;
 
 template <int F0, int F1>
-static size_t stream_smem(int cols, int npairs, bool route, int act_rows) {
+static size_t stream_smem(int cols, int act_rows) {
   const int bpi = item_blocks(cols);
   const size_t warp = (size_t)kStages * ((size_t)kTile * bpi * 16 * 4 + slot_bytes2<F0, F1>(bpi));
   return kDecodeWarps * warp + (size_t)kDecodeWarps * kStages * 8 + 2 * 64 * 8 +
-         (size_t)act_rows * (cols / 64 * 80) * 2 + (route ? route_smem_bytes(npairs) : 0);
+         (size_t)act_rows * (cols / 64 * 80) * 2;
 }
 
 template <int MODE, int F0, int F1, int NT>
@@ -1291,9 +1142,7 @@ static int nt_for(int cols_needed) { return cols_needed <= 8 ? 1 : cols_needed <
 // MMA column groups of a routed call. The tile kernels split an expert's
 // pairs into runs of 8 * NT, so one group serves any routing; two pay off
 // only when experts average more than 8 pairs (fewer weight re-reads).
-// Calls above 64 tokens use the stream kernel at nt_for(T).
-static int routed_nt(int T, int npairs, int E) {
-  if (T > 64) return nt_for(T);
+static int routed_nt(int npairs, int E) {
   const int distinct = std::max(1, std::min(E, npairs));
   return (npairs + distinct - 1) / distinct > 8 ? 2 : 1;
 }
@@ -1406,9 +1255,7 @@ static int launch_stream(const CUtensorMap& m0, const CUtensorMap& m1, const Uni
   UnitArgs args = a;
   args.div_s = FastDiv::of((uint32_t)a.splits);
   args.div_tiles = FastDiv::of((uint32_t)((a.w0.rows + kTile - 1) / kTile));
-  const size_t smem = stream_smem<F0, F1>(a.w0.cols, a.T * a.topk,
-                                          MODE == MODE_GATEUP || MODE == MODE_DOWN || MODE == MODE_SWITCH,
-                                          BSM ? a.act_rows : 0);
+  const size_t smem = stream_smem<F0, F1>(a.w0.cols, BSM ? a.act_rows : 0);
   if (set_smem(kern, smem)) return -4;
   const int grid = occupancy_grid(kern, smem, items, num_sms);
   if (grid < 0) return -4;
@@ -1527,9 +1374,7 @@ int launch_gemv(const WDev& w, int fmt, int expert, const Values& V, const uint1
 DecodeWs decode_ws(int T, int topk, int experts, int hidden, int inter) {
   DecodeWs ws;
   const int npairs = T * topk;
-  ws.dmax = std::min(npairs, experts);
-  ws.nt = nt_for(T);
-  ws.nc = 8 * ws.nt;
+  (void)experts;
   ws.c2 = chunking(inter, hidden);
   ws.c3 = chunking(hidden, inter);
   size_t o = 0;
@@ -1539,14 +1384,6 @@ DecodeWs decode_ws(int T, int topk, int experts, int hidden, int inter) {
   o = align256(o + (size_t)T * hidden * 2);
   ws.hperm = o;
   o = align256(o + (size_t)npairs * inter * 2);
-  ws.cnt2 = o;
-  o = align256(o + (size_t)ws.dmax * ws.c2.tiles * 4);
-  ws.cnt3 = o;
-  o = align256(o + (size_t)ws.c3.tiles * 4);
-  ws.part2 = o;
-  o = align256(o + (size_t)ws.dmax * ws.c2.tiles * 2 * ws.c2.nkc * ws.nc * kTile * 4);
-  ws.part3 = o;
-  o = align256(o + (size_t)ws.c3.tiles * npairs * ws.c3.nkc * kTile * 4);
   ws.total = o;
   return ws;
 }
@@ -1555,6 +1392,7 @@ template <int FG, int FU, int FD, int NT>
 static int decode_impl(const WDev& g, const WDev& u, const WDev& d, const Values& V, const uint16_t* x, int T,
                        const int32_t* ids, const float* p, int topk, uint16_t* y, char* ws, cudaStream_t st,
                        int num_sms) {
+  static_assert(NT == 1 || NT == 2, "routed decode: one or two MMA column groups");
   const DecodeWs L = decode_ws(T, topk, g.experts, g.cols, g.rows);
   const int npairs = T * topk;
   UnitArgs a = {};
@@ -1564,11 +1402,9 @@ static int decode_impl(const WDev& g, const WDev& u, const WDev& d, const Values
   int32_t* status = reinterpret_cast<int32_t*>(ws + L.status);
   uint16_t* xp = reinterpret_cast<uint16_t*>(ws + L.xperm);
   uint16_t* hp = reinterpret_cast<uint16_t*>(ws + L.hperm);
-  int32_t* cnt2 = reinterpret_cast<int32_t*>(ws + L.cnt2);
-  int32_t* cnt3 = reinterpret_cast<int32_t*>(ws + L.cnt3);
-  const int nzero = (int)((L.part2 - L.cnt2) / 4);  // both counter arrays
+  const int ar = act_rows_smem(NT, T, g.cols);  // x rows in shared memory, else transposed by the prep kernel
   const int pblocks = std::max(1, std::min(num_sms, (int)(((int64_t)T * (g.cols / 16) + 63) / 64)));
-  if (launch_prep(pblocks, st, x, T, g.cols, xp, cnt2, nzero, ids, npairs, g.experts, status)) return -4;
+  if (launch_prep(pblocks, st, x, ar ? 0 : T, g.cols, xp, nullptr, 0, ids, npairs, g.experts, status)) return -4;
   a.w0 = g;
   a.w1 = u;
   a.V = V;
@@ -1579,20 +1415,11 @@ static int decode_impl(const WDev& g, const WDev& u, const WDev& d, const Values
   a.T = T;
   a.topk = topk;
   a.out16 = hp;
-  a.cnt = cnt2;
-  a.part = reinterpret_cast<float*>(ws + L.part2);
   a.status = status;
-  int rc;
-  if constexpr (NT <= 2) {
-    const int ar = act_rows_smem(NT, T, g.cols);
-    a.act_rows = ar;
-    const int groups = route_runs_max(npairs, g.experts, NT) * L.c2.tiles;
-    rc = ar ? launch_tiles<MODE_GATEUP, FG, FU, NT, true>(mg, mu, a, groups, st, num_sms, true)
-            : launch_tiles<MODE_GATEUP, FG, FU, NT, false>(mg, mu, a, groups, st, num_sms, true);
-  } else {
-    rc = launch_stream_any<MODE_GATEUP, FG, FU, NT>(mg, mu, a, L.dmax * 2 * L.c2.tiles * a.splits, st, num_sms, true,
-                                                    0);
-  }
+  a.act_rows = ar;
+  const int groups = route_runs_max(npairs, g.experts, NT) * L.c2.tiles;
+  const int rc = ar ? launch_tiles<MODE_GATEUP, FG, FU, NT, true>(mg, mu, a, groups, st, num_sms, true)
+                    : launch_tiles<MODE_GATEUP, FG, FU, NT, false>(mg, mu, a, groups, st, num_sms, true);
   if (rc) return rc;
   UnitArgs b = a;
   split_args(b, d.cols);
@@ -1600,26 +1427,20 @@ static int decode_impl(const WDev& g, const WDev& u, const WDev& d, const Values
   b.w1 = d;
   b.act = hp;
   b.out16 = y;
-  b.cnt = cnt3;
-  b.part = reinterpret_cast<float*>(ws + L.part3);
-  if constexpr (NT <= 2) {
-    const int ar = act_rows_smem(NT, npairs, d.cols);
-    b.act_rows = ar;
-    return ar ? launch_tiles<MODE_DOWN, FD, FD, NT, true>(md, md, b, L.c3.tiles, st, num_sms, true)
-              : launch_tiles<MODE_DOWN, FD, FD, NT, false>(md, md, b, L.c3.tiles, st, num_sms, true);
-  }
-  return launch_stream_any<MODE_DOWN, FD, FD, NT>(md, md, b, L.dmax * L.c3.tiles * b.splits, st, num_sms, true, 0);
+  b.act_rows = act_rows_smem(NT, npairs, d.cols);
+  return b.act_rows ? launch_tiles<MODE_DOWN, FD, FD, NT, true>(md, md, b, L.c3.tiles, st, num_sms, true)
+                    : launch_tiles<MODE_DOWN, FD, FD, NT, false>(md, md, b, L.c3.tiles, st, num_sms, true);
 }
 
 int launch_moe_decode(const WDev& g, int fg, const WDev& u, int fu, const WDev& d, int fd, const Values& V,
                       const uint16_t* x, int T, const int32_t* ids, const float* p, int topk, uint16_t* y, char* ws,
                       cudaStream_t st, int num_sms) {
-  const int NT = routed_nt(T, T * topk, g.experts);
+  const int NT = routed_nt(T * topk, g.experts);
   const int key = fg * 4 + fu * 2 + fd;
 #define IQK_DEC(G, U, D, N)                  \
   if (key == G * 4 + U * 2 + D && NT == N) \
     return decode_impl<G, U, D, N>(g, u, d, V, x, T, ids, p, topk, y, ws, st, num_sms);
-#define IQK_DEC_N(G, U, D) IQK_DEC(G, U, D, 1) IQK_DEC(G, U, D, 2) IQK_DEC(G, U, D, 4) IQK_DEC(G, U, D, 8)
+#define IQK_DEC_N(G, U, D) IQK_DEC(G, U, D, 1) IQK_DEC(G, U, D, 2)
   IQK_DEC_N(0, 0, 0) IQK_DEC_N(0, 0, 1) IQK_DEC_N(0, 1, 0) IQK_DEC_N(0, 1, 1)
   IQK_DEC_N(1, 0, 0) IQK_DEC_N(1, 0, 1) IQK_DEC_N(1, 1, 0) IQK_DEC_N(1, 1, 1)
 #undef IQK_DEC_N
@@ -1629,26 +1450,22 @@ int launch_moe_decode(const WDev& g, int fg, const WDev& u, int fu, const WDev& 
 
 SwitchWs switch_ws(int T, int topk, int experts, int rows, int cols) {
   SwitchWs ws;
-  const int npairs = T * topk;
-  const int tiles = (rows + kTile - 1) / kTile;
-  const int S = (cols / 256) / item_blocks(cols);
+  (void)topk;
+  (void)experts;
+  (void)rows;
   size_t o = 0;
   ws.status = o;
   o = align256(o + 16);
   ws.xperm = o;
   o = align256(o + (size_t)T * cols * 2);
-  ws.cnt = o;
-  o = align256(o + (size_t)tiles * 4);
-  ws.part = o;
-  o = align256(o + (size_t)tiles * npairs * S * kTile * 4);
   ws.total = o;
-  (void)experts;
   return ws;
 }
 
 template <int FMT, int NT>
 static int switch_impl(const WDev& w, const Values& V, const uint16_t* x, int T, const int32_t* ids, int topk,
                        float* y, char* ws, cudaStream_t st, int num_sms) {
+  static_assert(NT == 1 || NT == 2, "switch decode: one or two MMA column groups");
   const SwitchWs L = switch_ws(T, topk, w.experts, w.rows, w.cols);
   const int npairs = T * topk;
   UnitArgs a = {};
@@ -1657,42 +1474,34 @@ static int switch_impl(const WDev& w, const Values& V, const uint16_t* x, int T,
   if (make_qs_map(&map, w, a.bpi)) return -4;
   uint16_t* xp = reinterpret_cast<uint16_t*>(ws + L.xperm);
   int32_t* status = reinterpret_cast<int32_t*>(ws + L.status);
-  int32_t* cnt = reinterpret_cast<int32_t*>(ws + L.cnt);
   const int tiles = (w.rows + kTile - 1) / kTile;
+  const int ar = act_rows_smem(NT, T, w.cols);  // x rows in shared memory, else transposed by the prep kernel
   const int pblocks = std::max(1, std::min(num_sms, (int)(((int64_t)T * (w.cols / 16) + 63) / 64)));
-  if (launch_prep(pblocks, st, x, T, w.cols, xp, cnt, tiles, ids, npairs, w.experts, status)) return -4;
+  if (launch_prep(pblocks, st, x, ar ? 0 : T, w.cols, xp, nullptr, 0, ids, npairs, w.experts, status)) return -4;
   a.w0 = w;
   a.w1 = w;
   a.V = V;
   a.ids = ids;
   a.act = xp;
+  a.xraw = x;
   a.T = T;
   a.topk = topk;
   a.yf = y;
-  a.cnt = cnt;
-  a.part = reinterpret_cast<float*>(ws + L.part);
   a.status = status;
-  const int dmax = std::min(npairs, w.experts);
-  if constexpr (NT <= 2) {
-    // tile kernel: a group is tpg tiles of one expert, splits * tpg <= warps items
-    a.tpg = std::max(1, kDecodeWarps / a.splits);
-    const int groups = route_runs_max(npairs, w.experts, NT) * ((tiles + a.tpg - 1) / a.tpg);
-    const int ar = act_rows_smem(NT, T, w.cols);
-    a.act_rows = ar;
-    a.xraw = x;
-    return ar ? launch_tiles<MODE_SWITCH, FMT, FMT, NT, true>(map, map, a, groups, st, num_sms, true)
-              : launch_tiles<MODE_SWITCH, FMT, FMT, NT, false>(map, map, a, groups, st, num_sms, true);
-  }
-  return launch_stream_any<MODE_SWITCH, FMT, FMT, NT>(map, map, a, dmax * tiles * a.splits, st, num_sms, true, 0);
+  a.act_rows = ar;
+  // a group is tpg tiles of one run, splits * tpg <= warps items
+  a.tpg = std::max(1, kDecodeWarps / a.splits);
+  const int groups = route_runs_max(npairs, w.experts, NT) * ((tiles + a.tpg - 1) / a.tpg);
+  return ar ? launch_tiles<MODE_SWITCH, FMT, FMT, NT, true>(map, map, a, groups, st, num_sms, true)
+            : launch_tiles<MODE_SWITCH, FMT, FMT, NT, false>(map, map, a, groups, st, num_sms, true);
 }
 
 int launch_switch_decode(const WDev& w, int fmt, const Values& V, const uint16_t* x, int T, const int32_t* ids,
                          int topk, float* y, char* ws, cudaStream_t st, int num_sms) {
-  const int NT = routed_nt(T, T * topk, w.experts);
+  const int NT = routed_nt(T * topk, w.experts);
 #define IQK_SW(F, N) \
   if (fmt == F && NT == N) return switch_impl<F, N>(w, V, x, T, ids, topk, y, ws, st, num_sms);
-  IQK_SW(FMT_KS, 1) IQK_SW(FMT_KS, 2) IQK_SW(FMT_KS, 4) IQK_SW(FMT_KS, 8)
-  IQK_SW(FMT_K, 1) IQK_SW(FMT_K, 2) IQK_SW(FMT_K, 4) IQK_SW(FMT_K, 8)
+  IQK_SW(FMT_KS, 1) IQK_SW(FMT_KS, 2) IQK_SW(FMT_K, 1) IQK_SW(FMT_K, 2)
 #undef IQK_SW
   return -3;
 }

@@ -42,7 +42,7 @@ constexpr int kStages = IQK_DECODE_STAGES;      // ring stages per warp, one ite
 constexpr int kDecodeMinBlocks(int nt) {
   return nt >= 4 ? (8 / kDecodeWarps > 0 ? 8 / kDecodeWarps : 1) : (16 / kDecodeWarps > 0 ? 16 / kDecodeWarps : 1);
 }
-constexpr int kMaxPairs = 1024;  // decode: T * topk
+constexpr int kMaxPairs = 1024;  // routed decode and switch: T * topk
 
 // n / d for 0 <= n < 2^31 as (umulhi(n, m) + n) >> s, with m and s fixed on
 // the host (division by an invariant integer, Granlund and Montgomery 1994).
@@ -67,10 +67,10 @@ struct GemvWs {
 };
 GemvWs gemv_ws(int T, int rows, int cols);
 
-// Workspace carve-up for iqk_moe_decode.
+// Workspace carve-up for iqk_moe_decode: status word, transposed x (read
+// through L1 when it does not fit shared memory), h.
 struct DecodeWs {
-  size_t status, xperm, hperm, cnt2, cnt3, part2, part3, total;
-  int dmax, nt, nc;
+  size_t status, xperm, hperm, total;
   Chunking c2, c3;
 };
 DecodeWs decode_ws(int T, int topk, int experts, int hidden, int inter);
@@ -88,7 +88,7 @@ int launch_moe_decode(const WDev& g, int fg, const WDev& u, int fu, const WDev& 
 
 // Routed single projection (switch linear), per (token, slot) pair, fp32.
 struct SwitchWs {
-  size_t status, xperm, cnt, part, total;
+  size_t status, xperm, total;
 };
 SwitchWs switch_ws(int T, int topk, int experts, int rows, int cols);
 int launch_switch_decode(const WDev& w, int fmt, const Values& V, const uint16_t* x, int T, const int32_t* ids,

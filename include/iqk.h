@@ -222,11 +222,8 @@ int iqk_gemv_static(const iqk_weights* w, int32_t expert, const float* values /*
  *   gate, up: [E][inter][hidden];  down: [E][hidden][inter]  (same E)
  *   x:   device bf16 [T][hidden]
  *   ids: device int32 [T][topk], expert of slot j of token t (0 <= id < E;
- *        ids within a token should be distinct -- duplicates are computed as
- *        separate pairs, except in iqk_moe_decode / iqk_switch_linear's
- *        decode kernel when they give one expert more pairs than the call's
- *        MMA columns (8 * ceil(T / 8) rounded up to 8, 16, 32 or 64): those
- *        extra pairs are dropped and bit 3 of the status word is set)
+ *        a token may list one expert in several slots: each slot is its own
+ *        pair, weighted by its own p)
  *   p:   device float32 [T][topk], routing weight of each slot
  *   y:   device bf16 [T][hidden], written completely:
  *        y[t] = bf16_rn( sum_j p[t][j] * down_e( bf16_rn( silu(gate_e x_t) * up_e x_t ) ) )
@@ -234,7 +231,9 @@ int iqk_gemv_static(const iqk_weights* w, int32_t expert, const float* values /*
  *   1 <= topk <= 16.
  *
  * iqk_moe_decode: few tokens (1 <= T <= 64); one weight read per distinct
- *   expert per call, shared by the tokens routed to it.
+ *   expert per call, shared by the tokens routed to it (an expert with more
+ *   than 8 pairs -- 16 when experts average more than 8 -- is read once per
+ *   run of that many).
  * iqk_moe_prefill: many tokens (1 <= T <= 65536); pairs grouped by expert,
  *   weights dequantized once per expert into bfloat16 tensor-core operands.
  *
@@ -255,10 +254,9 @@ int iqk_moe_prefill(const iqk_weights* gate, const iqk_weights* up, const iqk_we
 /*
  * iqk_moe_status -- synchronises `stream`, then reads the status word a
  * decode/prefill/switch call left in `workspace`: IQK_OK; IQK_ETIMEOUT if a
- * bounded device wait expired; IQK_EUNSUPPORTED if duplicate ids gave one
- * expert more pairs than the decode kernel's MMA columns (those pairs were
- * dropped); IQK_EINVAL if any expert id was outside [0, E) (those pairs were
- * skipped). The first applicable code in that order is returned.
+ * bounded device wait expired; IQK_EINVAL if any expert id was outside
+ * [0, E) (those pairs were skipped). The first applicable code in that order
+ * is returned.
  */
 int iqk_moe_status(const void* workspace, void* stream);
 
