@@ -22,7 +22,8 @@ FMT = {"iq2_ks": 0, "iq2_k": 1}
 EXPORTS = (
     "iqk_strerror", "iqk_last_cuda_error", "iqk_version", "iqk_row_bytes",
     "iqk_dequant", "iqk_dequant_bf16", "iqk_dequant_floor", "iqk_gemv_workspace_bytes", "iqk_gemv", "iqk_gemv_static",
-    "iqk_moe_workspace_bytes", "iqk_moe_decode", "iqk_moe_prefill", "iqk_moe_status",
+    "iqk_moe_workspace_bytes", "iqk_moe_decode", "iqk_moe_decode_shard", "iqk_f32_to_bf16",
+    "iqk_moe_prefill", "iqk_moe_status",
     "iqk_route_workspace_bytes", "iqk_moe_route", "iqk_floor",
     "iqk_switch_linear_workspace_bytes", "iqk_switch_linear",
 )
@@ -66,6 +67,8 @@ def lib(build_if_missing: bool = True) -> ctypes.CDLL:
             "iqk_gemv_static": (ctypes.c_int, [W, i32, vp, vp, i32, vp, vp]),
             "iqk_moe_workspace_bytes": (sz, [i32, i32, i32, i32, i32, i32]),
             "iqk_moe_decode": (ctypes.c_int, [W, W, W, vp, vp, i32, vp, vp, i32, vp, vp, sz, vp]),
+            "iqk_moe_decode_shard": (ctypes.c_int, [W, W, W, vp, vp, i32, vp, vp, i32, i32, vp, vp, sz, vp]),
+            "iqk_f32_to_bf16": (ctypes.c_int, [vp, vp, ctypes.c_int64, vp]),
             "iqk_moe_prefill": (ctypes.c_int, [W, W, W, vp, vp, i32, vp, vp, i32, vp, vp, sz, vp]),
             "iqk_moe_status": (ctypes.c_int, [vp, vp]),
             "iqk_route_workspace_bytes": (sz, [i32, i32, i32]),
@@ -264,6 +267,30 @@ def iqk_moe_decode(gate: Weights, up: Weights, down: Weights, values, x, ids, p,
 
 def iqk_moe_prefill(gate: Weights, up: Weights, down: Weights, values, x, ids, p, y=None, ws=None, stream=None):
     return _moe(lib().iqk_moe_prefill, 1, gate, up, down, values, x, ids, p, y, ws, stream)
+
+
+def iqk_moe_decode_shard(gate: Weights, up: Weights, down: Weights, values, x, ids, p, expert_base: int,
+                         y=None, ws=None, stream=None):
+    """One expert-parallel rank's float32 partial [T, hidden] (its experts
+    [expert_base, expert_base + gate.experts); other ids skipped)."""
+    torch = _torch()
+    T, topk = ids.shape
+    y = _empty((T, down.rows), torch.float32, x.device) if y is None else y
+    if ws is None:
+        ws = workspace(iqk_moe_workspace_bytes(0, T, topk, gate.experts, gate.cols, gate.rows), x.device)
+    v = _values(values)
+    _check(lib().iqk_moe_decode_shard(ctypes.byref(gate.c), ctypes.byref(up.c), ctypes.byref(down.c), v.ctypes.data,
+                                      x.data_ptr(), T, ids.data_ptr(), p.data_ptr(), topk, expert_base,
+                                      y.data_ptr(), ws.data_ptr(), ws.numel(), _stream(stream)),
+           "iqk_moe_decode_shard")
+    return y
+
+
+def iqk_f32_to_bf16(x, out=None, stream=None):
+    torch = _torch()
+    out = _empty(tuple(x.shape), torch.bfloat16, x.device) if out is None else out
+    _check(lib().iqk_f32_to_bf16(x.data_ptr(), out.data_ptr(), x.numel(), _stream(stream)), "iqk_f32_to_bf16")
+    return out
 
 
 def iqk_moe_status(ws, stream=None) -> int:

@@ -304,9 +304,9 @@ __device__ __forceinline__ RouteView carve_route(uint8_t* p, int n) {
 // MMA columns always suffice; such an expert's weights are then read once per
 // run).
 __device__ __forceinline__ void build_route(const int32_t* __restrict__ ids, int n, int E, RouteView r,
-                                            int chunk = 1 << 30) {
+                                            int chunk = 1 << 30, int ebase = 0) {
   for (int p = threadIdx.x; p < n; p += blockDim.x) {
-    const int e = ids[p];
+    const int e = ids[p] - ebase;  // an expert-parallel shard holds experts [ebase, ebase + E)
     r.ids[p] = (e >= 0 && e < E) ? e : -1;
   }
   __syncthreads();
@@ -434,6 +434,7 @@ struct UnitArgs {
   int async_sc;  // scale slices by cp.async (blocks per row a multiple of four)
   int act_rows;  // BSM: activation rows copied into shared memory
   int tpg;       // tile kernel, SWITCH: tiles per group (items per group = splits * tpg)
+  int ebase;     // routed modes: first expert id the weights hold (expert-parallel shard)
   FastDiv div_s, div_tiles;
 };
 
@@ -838,7 +839,7 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, kDecodeMinBlocks(NT)) k_til
     fence_mbar_init();
   }
   const RouteView rt = carve_route(route_p, npairs);
-  build_route(A.ids, npairs, A.w0.experts, rt, NC);  // ends with __syncthreads; runs of <= NC pairs
+  build_route(A.ids, npairs, A.w0.experts, rt, NC, A.ebase);  // ends with __syncthreads; runs of <= NC pairs
   const int D = rt.scalars[0];
   const int rows = A.w0.rows;
   const int tiles = (rows + kTile - 1) / kTile;
@@ -943,8 +944,11 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, kDecodeMinBlocks(NT)) k_til
         A.yf[(size_t)pr * rows + i] = 0.f;
     }
   }
-  if (MODE == MODE_DOWN && D == 0) {  // every id out of range: the block output is zero
-    for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < A.T * rows; i += gridDim.x * blockDim.x) A.out16[i] = 0;
+  if (MODE == MODE_DOWN && D == 0) {  // no pair on these experts: the block output is zero
+    for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < A.T * rows; i += gridDim.x * blockDim.x) {
+      if (A.yf) A.yf[i] = 0.f;
+      else A.out16[i] = 0;
+    }
     return;
   }
   const uint16_t* act_base = BSM ? act_s : A.act;
@@ -1079,7 +1083,8 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, kDecodeMinBlocks(NT)) k_til
         if (f >= rows) continue;
         float y = 0.f;
         for (int w = 0; w < kDecodeWarps; w++) y += red[(size_t)w * slot_f + tok * kTile + row];
-        A.out16[(size_t)tok * rows + f] = f32_to_bf16_bits(y);
+        if (A.yf) A.yf[(size_t)tok * rows + f] = y;  // an expert-parallel partial, summed across ranks
+        else A.out16[(size_t)tok * rows + f] = f32_to_bf16_bits(y);
       }
     }
     __syncthreads();  // slots free for the next group
@@ -1227,6 +1232,19 @@ __global__ void __launch_bounds__(256) k_zero(uint32_t* __restrict__ out, size_t
   griddep_launch();
   griddep_wait();
   for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x) out[i] = 0u;
+}
+
+// out[i] = bf16_rn(in[i]): the last step of an expert-parallel decode, after
+// the ranks' float32 partials are summed.
+__global__ void __launch_bounds__(256) k_to_bf16(const float* __restrict__ in, uint16_t* __restrict__ out, int64_t n) {
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x)
+    out[i] = f32_to_bf16_bits(in[i]);
+}
+
+int launch_to_bf16(const float* in, uint16_t* out, int64_t n, cudaStream_t st, int num_sms) {
+  const int64_t blocks = std::max<int64_t>(1, std::min<int64_t>((n + 255) / 256, (int64_t)num_sms * 8));
+  k_to_bf16<<<(unsigned)blocks, 256, 0, st>>>(in, out, n);
+  return cudaGetLastError() == cudaSuccess ? 0 : -4;
 }
 
 GemvWs gemv_ws(int T, int rows, int cols) {
@@ -1390,8 +1408,8 @@ DecodeWs decode_ws(int T, int topk, int experts, int hidden, int inter) {
 
 template <int FG, int FU, int FD, int NT>
 static int decode_impl(const WDev& g, const WDev& u, const WDev& d, const Values& V, const uint16_t* x, int T,
-                       const int32_t* ids, const float* p, int topk, uint16_t* y, char* ws, cudaStream_t st,
-                       int num_sms) {
+                       const int32_t* ids, const float* p, int topk, uint16_t* y, float* yf, int ebase, char* ws,
+                       cudaStream_t st, int num_sms) {
   static_assert(NT == 1 || NT == 2, "routed decode: one or two MMA column groups");
   const DecodeWs L = decode_ws(T, topk, g.experts, g.cols, g.rows);
   const int npairs = T * topk;
@@ -1404,7 +1422,11 @@ static int decode_impl(const WDev& g, const WDev& u, const WDev& d, const Values
   uint16_t* hp = reinterpret_cast<uint16_t*>(ws + L.hperm);
   const int ar = act_rows_smem(NT, T, g.cols);  // x rows in shared memory, else transposed by the prep kernel
   const int pblocks = std::max(1, std::min(num_sms, (int)(((int64_t)T * (g.cols / 16) + 63) / 64)));
-  if (launch_prep(pblocks, st, x, ar ? 0 : T, g.cols, xp, nullptr, 0, ids, npairs, g.experts, status)) return -4;
+  // a shard skips the ids of other shards silently, so it checks none
+  const bool shard = yf != nullptr;
+  if (launch_prep(pblocks, st, x, ar ? 0 : T, g.cols, xp, nullptr, 0, ids, shard ? 0 : npairs, g.experts, status))
+    return -4;
+  a.ebase = ebase;
   a.w0 = g;
   a.w1 = u;
   a.V = V;
@@ -1427,19 +1449,20 @@ static int decode_impl(const WDev& g, const WDev& u, const WDev& d, const Values
   b.w1 = d;
   b.act = hp;
   b.out16 = y;
+  b.yf = yf;
   b.act_rows = act_rows_smem(NT, npairs, d.cols);
   return b.act_rows ? launch_tiles<MODE_DOWN, FD, FD, NT, true>(md, md, b, L.c3.tiles, st, num_sms, true)
                     : launch_tiles<MODE_DOWN, FD, FD, NT, false>(md, md, b, L.c3.tiles, st, num_sms, true);
 }
 
 int launch_moe_decode(const WDev& g, int fg, const WDev& u, int fu, const WDev& d, int fd, const Values& V,
-                      const uint16_t* x, int T, const int32_t* ids, const float* p, int topk, uint16_t* y, char* ws,
-                      cudaStream_t st, int num_sms) {
+                      const uint16_t* x, int T, const int32_t* ids, const float* p, int topk, uint16_t* y, float* yf,
+                      int ebase, char* ws, cudaStream_t st, int num_sms) {
   const int NT = routed_nt(T * topk, g.experts);
   const int key = fg * 4 + fu * 2 + fd;
 #define IQK_DEC(G, U, D, N)                  \
   if (key == G * 4 + U * 2 + D && NT == N) \
-    return decode_impl<G, U, D, N>(g, u, d, V, x, T, ids, p, topk, y, ws, st, num_sms);
+    return decode_impl<G, U, D, N>(g, u, d, V, x, T, ids, p, topk, y, yf, ebase, ws, st, num_sms);
 #define IQK_DEC_N(G, U, D) IQK_DEC(G, U, D, 1) IQK_DEC(G, U, D, 2)
   IQK_DEC_N(0, 0, 0) IQK_DEC_N(0, 0, 1) IQK_DEC_N(0, 1, 0) IQK_DEC_N(0, 1, 1)
   IQK_DEC_N(1, 0, 0) IQK_DEC_N(1, 0, 1) IQK_DEC_N(1, 1, 0) IQK_DEC_N(1, 1, 1)

@@ -82,9 +82,12 @@ int make_qs_map(CUtensorMap* map, const WDev& w, int nb);
 int launch_gemv(const WDev& w, int fmt, int expert, const Values& V, const uint16_t* x, int T,
                 float* y, char* ws, cudaStream_t st, int num_sms);
 
+// yf non-null: an expert-parallel shard holding experts [ebase, ebase + E)
+// writes its float32 partial to yf (y unused) and skips other ids silently.
 int launch_moe_decode(const WDev& g, int fg, const WDev& u, int fu, const WDev& d, int fd,
                       const Values& V, const uint16_t* x, int T, const int32_t* ids, const float* p,
-                      int topk, uint16_t* y, char* ws, cudaStream_t st, int num_sms);
+                      int topk, uint16_t* y, float* yf, int ebase, char* ws, cudaStream_t st, int num_sms);
+int launch_to_bf16(const float* in, uint16_t* out, int64_t n, cudaStream_t st, int num_sms);
 
 // Routed single projection (switch linear), per (token, slot) pair, fp32.
 struct SwitchWs {

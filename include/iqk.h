@@ -252,6 +252,32 @@ int iqk_moe_prefill(const iqk_weights* gate, const iqk_weights* up, const iqk_we
                     void* workspace, size_t ws_bytes, void* stream);
 
 /*
+ * iqk_moe_decode_shard -- one rank's part of an expert-parallel
+ * iqk_moe_decode (the routed block's experts partitioned over ranks; each
+ * rank holds the streams of experts [expert_base, expert_base + E) in
+ * gate/up/down, E = their `experts`). Arguments as iqk_moe_decode, with the
+ * GLOBAL expert ids in `ids`. Pairs whose id lies outside the rank's window
+ * are skipped silently (no status bit: they belong to another rank), so a
+ * shard checks no ids. Output:
+ *   y_partial: device float32 [T][hidden], written completely:
+ *     y_partial[t] = sum over slots j with ids[t][j] in the window of
+ *                    p[t][j] * down_e( bf16_rn( silu(gate_e x_t) * up_e x_t ) )
+ * The sum of every rank's y_partial (a collective, e.g. an all-reduce over
+ * NCCL), rounded with iqk_f32_to_bf16, is the routed block's y; summation
+ * order across ranks is the collective's. Workspace as iqk_moe_decode.
+ */
+int iqk_moe_decode_shard(const iqk_weights* gate, const iqk_weights* up, const iqk_weights* down,
+                         const float* values /* host [8] */, const uint16_t* x, int32_t T,
+                         const int32_t* ids, const float* p, int32_t topk, int32_t expert_base,
+                         float* y_partial, void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * iqk_f32_to_bf16 -- out[i] = bf16_rn(in[i]) (nearest even) for i < n;
+ * device pointers. The last step of an expert-parallel decode.
+ */
+int iqk_f32_to_bf16(const float* in, uint16_t* out, int64_t n, void* stream);
+
+/*
  * iqk_moe_status -- synchronises `stream`, then reads the status word a
  * decode/prefill/switch call left in `workspace`: IQK_OK; IQK_ETIMEOUT if a
  * bounded device wait expired; IQK_EINVAL if any expert id was outside

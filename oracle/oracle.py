@@ -26,6 +26,8 @@ What it computes, and where each step is defined:
   expert ... each expert's weights read once" requires (section "Surface").
 * ``floor_xor``: the deleted-decode address floor's checksum (section
   "Pricing": identical loads, decode removed, an integer accumulator).
+* ``moe_shard``: one expert-parallel rank's part of ``moe`` (the slots
+  routed to its experts), so that the parts of a partition sum to ``moe``.
 * ``dequant_floor``: the dequantizer's own floor signature (same section):
   per qs word, the XOR of the stream fields its 16 weights are decoded from,
   written where the dequantizer writes those weights.
@@ -333,3 +335,14 @@ def dequant_floor(w, e: int, bf16: bool = False) -> np.ndarray:
     m = q ^ s ^ h ^ (x << np.uint32(8)) ^ (dv << np.uint32(16))
     n = 8 if bf16 else 16
     return (m[:, :, None] ^ np.arange(n, dtype=np.uint32)[None, None, :]).reshape(rows, wpr * n)
+
+
+def moe_shard(gate, up, down, values, x_bits, ids, p, lo: int, hi: int):
+    """One rank's part of the routed block when its experts are partitioned
+    over ranks (expert parallelism): the block's weighted sum over slots,
+    restricted to the slots routed to experts [lo, hi); every other slot
+    weighs 0. The parts of a partition of the experts add up to ``moe``'s
+    float64 y (the sum over slots regrouped by owner). Same dict as ``moe``."""
+    ids = np.atleast_2d(ids)
+    p = np.where((ids >= lo) & (ids < hi), np.atleast_2d(p), 0.0)
+    return moe(gate, up, down, values, x_bits, ids, p)

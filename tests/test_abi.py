@@ -90,6 +90,17 @@ def test_moe_shape_checks():
     assert L.iqk_moe_prefill(*args(d, T=70000)) == B.IQK_EUNSUPPORTED
     assert L.iqk_moe_workspace_bytes(0, 65, 6, 4, 256, 512) == 0
     assert L.iqk_moe_workspace_bytes(0, 1, 6, 4, 256, 512) > 0
+    # the expert-parallel shard: same checks, plus a non-negative expert base
+    sargs = lambda dd, T=1, k=6, base=0, ws=None: (ctypes.byref(g), ctypes.byref(u), ctypes.byref(dd), v, 4096, T,
+                                                   4096, 4096, k, base, 4096, ws, 0, None)
+    assert L.iqk_moe_decode_shard(*sargs(d_bad)) == B.IQK_EINVAL
+    assert L.iqk_moe_decode_shard(*sargs(d, base=-1)) == B.IQK_EINVAL
+    assert L.iqk_moe_decode_shard(*sargs(d, T=65)) == B.IQK_EUNSUPPORTED
+    assert L.iqk_moe_decode_shard(*sargs(d, T=0)) == B.IQK_OK
+    assert L.iqk_moe_decode_shard(*sargs(d)) == B.IQK_EWORKSPACE
+    assert L.iqk_f32_to_bf16(None, None, 0, None) == B.IQK_OK
+    assert L.iqk_f32_to_bf16(None, 4096, 8, None) == B.IQK_EINVAL
+    assert L.iqk_f32_to_bf16(4096, 4096, -1, None) == B.IQK_EINVAL
 
 
 def test_switch_linear_mode_checks():
