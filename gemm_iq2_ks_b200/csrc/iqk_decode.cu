@@ -1,5 +1,7 @@
 // Decode-side kernels: single-expert GEMV, routed gate/up + SwiGLU, routed
-// down + weighted combine, and the deleted-decode address floor.
+// down + weighted combine (whole block or one expert-parallel shard), the
+// routed single projection (switch linear), and the deleted-decode address
+// floor.
 //
 // mlx-iqk 0.1.1 PKG-INFO: "a call with few token-expert pairs runs the fused
 // decode GEMV" (section "Surface"); reconstruction d*float(scale_index)*
@@ -12,10 +14,12 @@
 // (no multicast) while the lanes copy the item's scale slice with cp.async
 // onto the same mbarrier; the warp decodes the tile against a per-CTA table
 // of bf16(scale_index * value) entries with byte-permutes and reduces with
-// m16n8k16 tensor-core MMAs (tokens or pairs as the MMA's N). The slices of
-// a tile meet in the workspace; the last item to finish a tile (device-scope
-// counter) sums them in slice order, so results do not depend on arrival
-// order.
+// m16n8k16 tensor-core MMAs (tokens or pairs as the MMA's N). In the tile
+// kernel (routed calls) a CTA takes a group of items and sums their slices in
+// shared memory in warp order; in the stream kernel (GEMV, floor) the slices
+// of a tile meet in the workspace and the last item to finish a tile
+// (device-scope counter) sums them in slice order. Either way results do not
+// depend on arrival order.
 #include <algorithm>
 
 #include "iqk_device.cuh"
@@ -1037,7 +1041,7 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, kDecodeMinBlocks(NT)) k_til
       const int u = (int)A.div_tiles.div((uint32_t)tg);
       const int tile = tg - u * tiles;
       const int p0 = rt.ustart[u];
-      const int ncols = min(rt.ustart[u + 1] - p0, NC);  // more columns: reported as overflow
+      const int ncols = min(rt.ustart[u + 1] - p0, NC);  // runs never exceed NC; the bound guards the slot reads
       if (!waited) {  // h may still be read by the previous call's down kernel
         griddep_wait();
         waited = true;
