@@ -35,9 +35,10 @@ METRIC = "MoE decode µs/token & weight GB/s vs HBM floor; prefill bf16 TFLOP/s"
 RING = 420  # calls per captured graph (10 permutation cycles of 42 calls)
 
 
-# DRAM bytes (read + write) of the two tile kernels of one config-2 decode
-# call, from one ncu capture of `bench.py --profile decode --experts 24`
-# (profiles/decode_config2_tile_kernels.md); per call, not per resident expert.
+# DRAM bytes (read + write) of the two tile kernels of one headline decode
+# call (IQ2_KS, 256 experts, top-6, one token), from one ncu capture of
+# `bench.py --profile decode --experts 24` (its summary is kept under
+# profiles/); per call, not per resident expert.
 DECODE_CALL_TRAFFIC = 41_575_424
 
 
@@ -273,7 +274,7 @@ def floor_graph(torch, bench, stream, n):
 
 
 def prefill_leg(torch, B, weights, values, device, stream, peaks, calls=4, reps=3):
-    """Config 4: 2048 tokens routed top-6 over 256 experts, one prefill call =
+    """The prefill workload: 2048 tokens routed top-6 over 256 experts, one call =
     route + grouped gate/up GEMM + SwiGLU + grouped down GEMM + combine."""
     T = 2048
     rng = S.rng_for(4)
@@ -302,7 +303,7 @@ def prefill_leg(torch, B, weights, values, device, stream, peaks, calls=4, reps=
     tf = flops / per_call / 1e12
     status = B.iqk_moe_status(ws)
     del g, dw
-    return {"workload": "routed-expert prefill, IQ2_KS, 2048 tokens, 256 experts top-6 (config 4)",
+    return {"workload": "routed-expert prefill, IQ2_KS, 2048 tokens, 256 experts top-6",
             "us_per_call": per_call * 1e6, "tflops": tf, "flop_per_call": flops,
             "roofline": {"bound": "tensor", "achieved": tf, "peak": peaks["bf16"], "unit": "TFLOP/s",
                          "frac": tf / peaks["bf16"], "frac_of_sustained": tf / peaks["bf16_sustained"],
@@ -310,9 +311,9 @@ def prefill_leg(torch, B, weights, values, device, stream, peaks, calls=4, reps=
             "weight_gbs": sum(w.nbytes() for w in weights) / per_call / 1e9, "status": status}
 
 
-def gemv_leg(torch, B, cfg, device, stream, calls=200):
-    """Configs 0 and 1: one matrix, one activation row (the inputs stay L2-resident)."""
-    w, x, values = S.matrix_case(cfg)
+def gemv_leg(torch, B, case, device, stream, calls=200):
+    """A single-matrix workload: one matrix, one activation row (the inputs stay L2-resident)."""
+    w, x, values = S.matrix_case(case)
     dw = B.Weights.from_host(w, device)
     xd = torch.from_numpy(x.view(np.int16)).to(device).view(torch.bfloat16)
     y = torch.empty((xd.shape[0], w.rows), dtype=torch.float32, device=device)
@@ -507,7 +508,7 @@ def decode_weights_per_token():
 
 def config_block(extra=None):
     c = {"workload": "routed-expert decode, IQ2_KS, 1 token/call, 256 experts top-6, gate/up 2048x4096, "
-                     "down 4096x2048 (config 2)",
+                     "down 4096x2048",
          "global_batch": 1, "experts": S.EXPERTS, "topk": S.TOPK, "hidden": S.HIDDEN, "inter": S.INTER,
          "format": "iq2_ks", "parallelism": "replicas",
          "l2": "inputs larger than L2: consecutive calls' experts come from a chain of random "
@@ -615,8 +616,8 @@ def main():
         torch.cuda.synchronize()
         return 0
 
-    # ---------------- headline: config 2 decode
-    log("generating config 2 weights")
+    # ---------------- headline: IQ2_KS routed decode, one token per call
+    log("generating the headline decode weights")
     rng = S.rng_for(2 + 1000 * rank)
     w_ks = S.moe_weights(rng, "iq2_ks", S.EXPERTS, S.HIDDEN, S.INTER)
     values = S.value_table("int", 2)
@@ -665,7 +666,7 @@ def main():
     log(f"floor: {floor_us:.2f} us/call")
     details = {}
     if not args.no_details and rank == 0:
-        # config 3 (IQ2_K): T = 1, 4, 16
+        # IQ2_K routed decode at T = 1, 4, 16
         rng3 = S.rng_for(3)
         w_k = S.moe_weights(rng3, "iq2_k", S.EXPERTS, S.HIDDEN, S.INTER)
         for T in (1, 4, 16):
@@ -677,10 +678,10 @@ def main():
             tt3 = cuda_time(torch, stream, lambda: run_steps(gr, 2 * RING))
             per_call = tt3 / (2 * RING)
             by = db.weight_bytes(2 * RING) / (2 * RING)
-            details[f"config3_T{T}"] = {"us_per_call": per_call * 1e6, "us_per_token": per_call / T * 1e6,
-                                        "weight_gbs": by / per_call / 1e9,
-                                        "hbm_frac": by / per_call / 1e9 / peaks["hbm_gbs"],
-                                        "mean_distinct_experts": float(db.distinct.mean())}
+            details[f"decode_iq2_k_T{T}"] = {"us_per_call": per_call * 1e6, "us_per_token": per_call / T * 1e6,
+                                             "weight_gbs": by / per_call / 1e9,
+                                             "hbm_frac": by / per_call / 1e9 / peaks["hbm_gbs"],
+                                             "mean_distinct_experts": float(db.distinct.mean())}
             del db, gr
         if not args.no_price:
             log("pricing against own floors")
@@ -689,11 +690,11 @@ def main():
                                              device, stream, peaks)
         del w_k
         torch.cuda.empty_cache()
-        log("config 4 prefill")
-        details["config4_prefill"] = prefill_leg(torch, B, w_ks, values, device, stream, peaks)
+        log("prefill")
+        details["prefill_iq2_ks_2048"] = prefill_leg(torch, B, w_ks, values, device, stream, peaks)
         torch.cuda.empty_cache()
-        for cfg in (0, 1):
-            details[f"config{cfg}_gemv"] = gemv_leg(torch, B, cfg, device, stream)
+        for case in S.MATRIX_CASES:
+            details[case] = gemv_leg(torch, B, case, device, stream)
 
     launches = 3 * K
     line = {
@@ -716,7 +717,7 @@ def main():
         log("cpu baseline (oracle)")
         sec, ntok = oracle_decode_seconds(w_ks, values, args.cpu_budget)
         line["cpu_baseline"] = {"value": sec * 1e6, "unit": "us/token", "cores": 1, "kind": "oracle",
-                                "sample": f"{ntok} whole single-token decode calls of config 2 "
+                                "sample": f"{ntok} whole single-token headline decode calls "
                                           f"(fresh routing each), one thread"}
     if dist:
         dist.barrier()

@@ -180,28 +180,35 @@ def routing_ring(rng: np.random.Generator, calls: int, experts: int, topk: int):
     return ids, p
 
 
-# The five workloads (geometry: 256 experts, top-6, gate/up [2048,4096], down [4096,2048]).
+# The five workloads (routed geometry: 256 experts, top-6, gate/up
+# [2048,4096], down [4096,2048]), by name; `seed` seeds each one's inputs.
 HIDDEN, INTER, EXPERTS, TOPK = 4096, 2048, 256, 6
 
-CONFIGS = {
-    0: dict(kind="matrix", fmt="iq2_ks", rows=256, cols=512, tokens=1, seed=0),
-    1: dict(kind="matrix", fmt="iq2_k", rows=2048, cols=4096, tokens=1, seed=1),
-    2: dict(kind="decode", fmt="iq2_ks", experts=EXPERTS, hidden=HIDDEN, inter=INTER, topk=TOPK,
-            tokens=(1,), seed=2),
-    3: dict(kind="decode", fmt="iq2_k", experts=EXPERTS, hidden=HIDDEN, inter=INTER, topk=TOPK,
-            tokens=(1, 4, 16), seed=3),
-    4: dict(kind="prefill", fmt="iq2_ks", experts=EXPERTS, hidden=HIDDEN, inter=INTER, topk=TOPK,
-            tokens=(2048,), seed=4),
+WORKLOADS = {
+    "gemv_iq2_ks_256x512": dict(kind="matrix", fmt="iq2_ks", rows=256, cols=512, tokens=1, seed=0),
+    "gemv_iq2_k_2048x4096": dict(kind="matrix", fmt="iq2_k", rows=2048, cols=4096, tokens=1, seed=1),
+    "decode_iq2_ks_e256_top6": dict(kind="decode", fmt="iq2_ks", experts=EXPERTS, hidden=HIDDEN, inter=INTER,
+                                    topk=TOPK, tokens=(1,), seed=2),
+    "decode_iq2_k_e256_top6": dict(kind="decode", fmt="iq2_k", experts=EXPERTS, hidden=HIDDEN, inter=INTER,
+                                   topk=TOPK, tokens=(1, 4, 16), seed=3),
+    "prefill_iq2_ks_e256_top6_2048": dict(kind="prefill", fmt="iq2_ks", experts=EXPERTS, hidden=HIDDEN,
+                                          inter=INTER, topk=TOPK, tokens=(2048,), seed=4),
 }
+MATRIX_CASES = ("gemv_iq2_ks_256x512", "gemv_iq2_k_2048x4096")
+
+
+def seed_of(name: str) -> int:
+    return WORKLOADS[name]["seed"]
 
 
 def rng_for(seed: int) -> np.random.Generator:
     return np.random.Generator(np.random.PCG64(seed))
 
 
-def matrix_case(cfg: int, value_kind: str = "int"):
-    """Config 0/1: one matrix, one activation row and a value table."""
-    c = CONFIGS[cfg]
+def matrix_case(name: str, value_kind: str = "int"):
+    """A single-matrix workload (MATRIX_CASES): one matrix, one activation
+    row and a value table."""
+    c = WORKLOADS[name]
     rng = rng_for(c["seed"])
     w = random_streams(rng, c["fmt"], 1, c["rows"], c["cols"])
     x = random_bf16(rng, (c["tokens"], c["cols"]))

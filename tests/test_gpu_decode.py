@@ -28,11 +28,11 @@ def bits_equal(a, b):
 
 # ------------------------------------------------------------------ dequant
 
-@pytest.mark.parametrize("cfg", [0, 1])
+@pytest.mark.parametrize("case", S.MATRIX_CASES)
 @pytest.mark.parametrize("table", ["int", "f16"])
-def test_dequant_bitexact_configs(B, cfg, table):
-    w, _, _ = S.matrix_case(cfg)
-    values = S.value_table(table, cfg)
+def test_dequant_bitexact_matrix_cases(B, case, table):
+    w, _, _ = S.matrix_case(case)
+    values = S.value_table(table, S.seed_of(case))
     dw = B.Weights.from_host(w)
     got = B.iqk_dequant(dw, 0, values).cpu().numpy()
     assert bits_equal(got, O.dequant_expert(w, 0, values))
@@ -67,10 +67,10 @@ def test_dequant_edge_fields_multi_expert(B, fmt):
         assert bits_equal(got, O.dequant_expert(st, e, values)), e
 
 
-@pytest.mark.parametrize("cfg", [0, 1])
-def test_dequant_bf16_is_rounded_fp32(B, cfg):
-    w, _, _ = S.matrix_case(cfg)
-    values = S.value_table("f16", cfg)
+@pytest.mark.parametrize("case", S.MATRIX_CASES)
+def test_dequant_bf16_is_rounded_fp32(B, case):
+    w, _, _ = S.matrix_case(case)
+    values = S.value_table("f16", S.seed_of(case))
     dw = B.Weights.from_host(w)
     got = B.iqk_dequant_bf16(dw, 0, values).view(torch.int16).cpu().numpy().view(np.uint16)
     assert np.array_equal(got, O.bf16_round(O.dequant_expert(w, 0, values)))
@@ -78,16 +78,16 @@ def test_dequant_bf16_is_rounded_fp32(B, cfg):
 
 # --------------------------------------------------------------------- gemv
 
-@pytest.mark.parametrize("cfg", [0, 1])
+@pytest.mark.parametrize("case", S.MATRIX_CASES)
 @pytest.mark.parametrize("T", [1, 3, 8])
-def test_gemv_configs(B, cfg, T):
-    w, x, values = S.matrix_case(cfg)
+def test_gemv_matrix_cases(B, case, T):
+    w, x, values = S.matrix_case(case)
     rng = S.rng_for(100 + T)
     x = np.concatenate([x, S.random_bf16(rng, (T - 1, w.cols))]) if T > 1 else x
     dw = B.Weights.from_host(w)
     y = B.iqk_gemv(dw, 0, values, to_dev_bf16(x)).cpu().numpy()
     y_ref, Sabs = O.gemv(O.dequant_expert(w, 0, values), x)
-    check_fp32(y, y_ref, Sabs, f"gemv cfg{cfg} T={T}")
+    check_fp32(y, y_ref, Sabs, f"gemv {case} T={T}")
 
 
 @pytest.mark.parametrize("fmt", ["iq2_ks", "iq2_k"])
@@ -182,7 +182,7 @@ def full_k(B):
     return S.moe_weights(rng, "iq2_k", S.EXPERTS, S.HIDDEN, S.INTER)
 
 
-def test_moe_decode_full_config2(B, full_ks):
+def test_moe_decode_full_iq2_ks_e256_top6(B, full_ks):
     gate, up, down = full_ks
     rng = S.rng_for(20)
     x = S.random_bf16(rng, (1, S.HIDDEN))
@@ -190,11 +190,11 @@ def test_moe_decode_full_config2(B, full_ks):
     values = S.value_table("int", 2)
     y = _run_decode(B, gate, up, down, values, x, ids, p)
     ref = O.moe(gate, up, down, values, x, ids, p)
-    check_moe(y, ref, "config 2")
+    check_moe(y, ref, "IQ2_KS decode, 256 experts, top-6, 1 token")
 
 
 @pytest.mark.parametrize("T", [1, 4, 16])
-def test_moe_decode_full_config3(B, full_k, T):
+def test_moe_decode_full_iq2_k_e256_top6(B, full_k, T):
     gate, up, down = full_k
     rng = S.rng_for(30 + T)
     x = S.random_bf16(rng, (T, S.HIDDEN))
@@ -202,7 +202,7 @@ def test_moe_decode_full_config3(B, full_k, T):
     values = S.value_table("f16", 3)
     y = _run_decode(B, gate, up, down, values, x, ids, p)
     ref = O.moe(gate, up, down, values, x, ids, p)
-    check_moe(y, ref, f"config 3 T={T}")
+    check_moe(y, ref, f"IQ2_K decode, 256 experts, top-6, T={T}")
 
 
 # ------------------------------------------------------------------- route

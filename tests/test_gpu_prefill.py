@@ -96,8 +96,8 @@ def test_prefill_bad_ids(B):
     check_moe(from_dev_bf16(y), ref, "prefill bad ids")
 
 
-def test_prefill_full_config4_sampled(B):
-    """Config 4 at full size (2048 tokens, 256 experts, top-6, IQ2_KS);
+def test_prefill_full_iq2_ks_e256_top6_2048_sampled(B):
+    """The prefill workload at full size (2048 tokens, 256 experts, top-6, IQ2_KS);
     sampled tokens checked against the oracle one by one, every output finite."""
     rng = S.rng_for(4)
     gate, up, down = S.moe_weights(rng, "iq2_ks", S.EXPERTS, S.HIDDEN, S.INTER)
@@ -109,4 +109,4 @@ def test_prefill_full_config4_sampled(B):
     assert np.all(np.isfinite(yf))
     sample = np.random.default_rng(0).choice(2048, size=12, replace=False)
     ref = O.moe(gate, up, down, values, x, ids, p, tokens=sample)
-    check_moe(y[sample], ref, "config 4 sampled tokens")
+    check_moe(y[sample], ref, "prefill 2048 tokens, sampled")

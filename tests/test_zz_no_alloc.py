@@ -27,9 +27,9 @@ def test_static_scratch_limit_is_refused_on_the_host():
 
 
 @pytest.mark.gpu
-@pytest.mark.parametrize("cfg,T", [(0, 1), (1, 1), (1, 3)])
-def test_static_matches_workspace_gemv_twice(cfg, T):
-    w, x, values = S.matrix_case(cfg)
+@pytest.mark.parametrize("case,T", [(S.MATRIX_CASES[0], 1), (S.MATRIX_CASES[1], 1), (S.MATRIX_CASES[1], 3)])
+def test_static_matches_workspace_gemv_twice(case, T):
+    w, x, values = S.matrix_case(case)
     if T > 1:
         x = np.concatenate([x, S.random_bf16(S.rng_for(300 + T), (T - 1, w.cols))])
     dw = B.Weights.from_host(w)
@@ -38,5 +38,5 @@ def test_static_matches_workspace_gemv_twice(cfg, T):
     _, Sabs = O.gemv(O.dequant_expert(w, 0, values), x)
     for k in range(2):  # two calls in a row reuse the same scratch
         y_st = B.iqk_gemv_static(dw, 0, values, xd).cpu().numpy()
-        check_fp32(y_st, y_ws, Sabs, f"static gemv cfg{cfg} T={T} call {k}")
+        check_fp32(y_st, y_ws, Sabs, f"static gemv {case} T={T} call {k}")
         assert np.max(np.abs(y_st - y_ws) / np.maximum(Sabs, 1e-30)) <= TOL
