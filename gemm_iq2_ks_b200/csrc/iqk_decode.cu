@@ -568,6 +568,12 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, kDecodeMinBlocks(NT)) k_str
     fence_mbar_init();
   }
   __syncthreads();
+  // Only the kernel parameters are read before the dependency wait: x, the
+  // expert list and the weights may be written by the preceding kernel, which
+  // lets its dependents launch early. Dependents of this kernel may launch at
+  // once because they wait the same way.
+  griddep_launch();
+  griddep_wait();
   const int D = MODE == MODE_FLOOR ? A.nexp : 1;  // matrices streamed
   const int rows = A.w0.rows;
   const int tiles = (rows + kTile - 1) / kTile;
@@ -599,14 +605,6 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, kDecodeMinBlocks(NT)) k_str
     }
   };
   for (int s = 0; s < kStages; s++) issue(s);
-  // Dependents may launch now: the next kernel of a call waits before it
-  // writes, and the first kernel of the next call (prep or zeroing) too.
-  griddep_launch();
-  // Results of the preceding kernel in the stream (the prep kernel's counters
-  // and transposed activations) are read only after griddepcontrol.wait. The
-  // raw activation rows are inputs of the call, so a BSM launch copies them
-  // first and defers the wait to its first epilogue.
-  bool waited = false;
   if constexpr (BSM) {  // the call's activation rows, slot-transposed and padded, once per CTA
     const int gpr = K / 16;  // 16-element groups per row
     const int groups = A.act_rows * gpr;
@@ -628,9 +626,6 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, kDecodeMinBlocks(NT)) k_str
       dst[1] = make_uint4(o[4], o[5], o[6], o[7]);
     }
     __syncthreads();
-  } else if (MODE != MODE_FLOOR) {  // the floor reads no activations: it waits before its first atomic
-    griddep_wait();
-    waited = true;
   }
   const uint16_t* act_base = BSM ? act_s : A.act;
   constexpr int SEG = BSM ? 80 : 64;    // elements between the segments of lanes t and t + 1
@@ -653,7 +648,6 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, kDecodeMinBlocks(NT)) k_str
     const bool kfmt = F0 == FMT_K;
     const int st = it % kStages;
     if (!mbar_wait_bounded(&bar[st], (uint32_t)((it / kStages) & 1))) {
-      if (!waited) griddep_wait();
       if (lane == 0) atomicOr(A.status ? A.status : &g_floor_status, 2);
       // let this warp's copies still in flight land before the CTA exits
       for (int k = 1; k < kStages; k++)
@@ -720,10 +714,6 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, kDecodeMinBlocks(NT)) k_str
     }
     __syncwarp();
     issue(it + kStages);  // refill the stage just consumed
-    if (!waited) {
-      griddep_wait();
-      waited = true;
-    }
 
     const int rg = tile * kTile + g, rh = rg + 8;
     if (MODE == MODE_FLOOR) {
@@ -779,7 +769,6 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, kDecodeMinBlocks(NT)) k_str
         }
     }
   }
-  if (!waited) griddep_wait();  // this grid completes only after the one it depends on
 }
 
 // ------------------------------------------------------------- tile kernel
@@ -822,7 +811,20 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, kDecodeMinBlocks(NT)) k_til
   // floats per warp slot: (mat, column, row) gate/up; (column, row) switch; (token, row) down
   const int slot_f = MODE == MODE_GATEUP ? 2 * NC * kTile : MODE == MODE_SWITCH ? NC * kTile : A.T * kTile;
   uint8_t* route_p = reinterpret_cast<uint8_t*>(red + (size_t)kDecodeWarps * slot_f);
-  // gate/up: request the first activation groups ahead of the weight stream
+  // Only the kernel parameters are read before the dependency wait. Every
+  // input of the call (x, ids, p, h, the expert list) may be written by the
+  // preceding kernel, which lets its dependents launch early, so it is read
+  // after griddepcontrol.wait; dependents of this kernel may launch at once
+  // because they wait the same way.
+  build_lut<F0>(lut0, A.V);
+  if (MODE == MODE_GATEUP) build_lut<F1>(lut1, A.V);
+  if (lane == 0) {
+    for (int s = 0; s < kStages; s++) mbar_init(&bar[s], 1);
+    fence_mbar_init();
+  }
+  griddep_launch();
+  griddep_wait();
+  // gate/up and switch: request the first activation groups ahead of the weight stream
   uint4 pre0 = make_uint4(0u, 0u, 0u, 0u), pre1 = pre0, pre2 = pre0, pre3 = pre0;
   const int act_groups = BSM ? A.act_rows * (K / 16) : 0;
   if (BSM && MODE != MODE_DOWN) {
@@ -835,12 +837,6 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, kDecodeMinBlocks(NT)) k_til
       pre2 = ld_nc_u4(A.xraw + (size_t)g1 * 16);
       pre3 = ld_nc_u4(A.xraw + (size_t)g1 * 16 + 8);
     }
-  }
-  build_lut<F0>(lut0, A.V);
-  if (MODE == MODE_GATEUP) build_lut<F1>(lut1, A.V);
-  if (lane == 0) {
-    for (int s = 0; s < kStages; s++) mbar_init(&bar[s], 1);
-    fence_mbar_init();
   }
   const RouteView rt = carve_route(route_p, npairs);
   build_route(A.ids, npairs, A.w0.experts, rt, NC, A.ebase);  // ends with __syncthreads; runs of <= NC pairs
@@ -896,17 +892,6 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, kDecodeMinBlocks(NT)) k_til
     issued = q + 1;
   };
   for (int q = 0; q < kStages; q++) issue(q);
-  // gate/up lets its down kernel launch; the last kernel of a call lets the
-  // next call's prep (which waits before writing) and first kernel start
-  // their weight loads early
-  griddep_launch();
-  // The raw activation rows are inputs of the call and can be read before the
-  // dependency wait; h (DOWN) is the preceding kernel's result.
-  bool waited = false;
-  if (MODE == MODE_DOWN || !BSM) {
-    griddep_wait();
-    waited = true;
-  }
   if constexpr (BSM) {  // activation rows, slot-transposed and padded, once per CTA
     const int gpr = K / 16;
     for (int k = 0;; k++) {
@@ -938,10 +923,6 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, kDecodeMinBlocks(NT)) k_til
     __syncthreads();
   }
   if (MODE == MODE_SWITCH && rt.scalars[1] < npairs) {  // out-of-range ids: zero rows
-    if (!waited) {  // y may still be written by the previous call
-      griddep_wait();
-      waited = true;
-    }
     for (int pr = 0; pr < npairs; pr++) {
       if (rt.ids[pr] >= 0) continue;
       for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < rows; i += gridDim.x * blockDim.x)
@@ -990,10 +971,6 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, kDecodeMinBlocks(NT)) k_til
       const int st = q % kStages;
       if (!failed && !mbar_wait_bounded(&bar[st], (uint32_t)((q / kStages) & 1))) {
         failed = true;  // keep taking part in the CTA barriers; stop loading
-        if (!waited) {
-          griddep_wait();
-          waited = true;
-        }
         if (lane == 0) atomicOr(A.status, 2);
       }
       if (!failed) {
@@ -1042,10 +1019,6 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, kDecodeMinBlocks(NT)) k_til
       const int tile = tg - u * tiles;
       const int p0 = rt.ustart[u];
       const int ncols = min(rt.ustart[u + 1] - p0, NC);  // runs never exceed NC; the bound guards the slot reads
-      if (!waited) {  // h may still be read by the previous call's down kernel
-        griddep_wait();
-        waited = true;
-      }
       for (int o = threadIdx.x; o < ncols * kTile; o += blockDim.x) {
         const int col = o / kTile, row = o - col * kTile;
         const int f = tile * kTile + row;
@@ -1066,10 +1039,6 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, kDecodeMinBlocks(NT)) k_til
       const int p0 = rt.ustart[u];
       const int ncols = min(rt.ustart[u + 1] - p0, NC);
       const int per = ncols * kTile;
-      if (!waited) {  // y may still be written by the previous call
-        griddep_wait();
-        waited = true;
-      }
       for (int o = threadIdx.x; o < tpg * per; o += blockDim.x) {
         const int sub = o / per, rem = o - sub * per;
         const int col = rem / kTile, row = rem - col * kTile;
@@ -1095,7 +1064,6 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, kDecodeMinBlocks(NT)) k_til
   }
   // let copies still in flight land before the CTA exits (only after a timeout)
   for (int qd = consumed; qd < issued; qd++) (void)mbar_wait_bounded(&bar[qd % kStages], (uint32_t)((qd / kStages) & 1));
-  if (!waited) griddep_wait();  // this grid completes only after the one it depends on
 }
 
 // ================================================================== host

@@ -49,16 +49,17 @@
  *   - bf16 and fp16 values are passed as their 16-bit patterns (uint16_t).
  *   - Every stream plane's base address must be 16-byte aligned (the planes
  *     are staged into shared memory by TMA and bulk copies); IQK_EINVAL if not.
- *   - Consecutive calls overlap: the decode, GEMV, switch-linear and floor
- *     paths launch their kernels as programmatic dependents of whatever
- *     precedes them on the stream, and each kernel lets its dependents launch
- *     right after issuing its first loads. Every kernel of this library waits
- *     (griddepcontrol.wait) before it writes anything a preceding kernel may
- *     still read or write, so stream order holds as usual. A caller's own
- *     kernel launched with programmatic stream serialization right after one
- *     of these calls must do the same before reading the call's outputs;
- *     kernels launched without that attribute, copies and events see the
- *     call complete, as always.
+ *   - Consecutive calls overlap their launches: the decode, GEMV,
+ *     switch-linear and floor paths launch their kernels as programmatic
+ *     dependents of whatever precedes them on the stream, and each kernel
+ *     lets its dependents launch as soon as it starts. Every kernel of this
+ *     library waits (griddepcontrol.wait) for its predecessor before it reads
+ *     or writes any memory other than its launch parameters, so stream order
+ *     holds as usual: a call may read the previous call's output. A caller's
+ *     own kernel launched with programmatic stream serialization right after
+ *     one of these calls must likewise wait before touching the call's
+ *     outputs; kernels launched without that attribute, copies and events
+ *     see the call complete, as always.
  */
 #ifndef IQK_H_
 #define IQK_H_

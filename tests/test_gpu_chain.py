@@ -1,0 +1,88 @@
+"""Consecutive calls on one stream, each reading the previous call's output.
+
+Calls launch as programmatic dependents of whatever precedes them, so call
+N+1's kernels may start while call N's last kernel runs. Each kernel waits
+for its predecessor before it reads anything but its parameters; here call
+N+1's x is call N's y, so a kernel reading x too early would see a partial y.
+The kernels are deterministic, so the chained results must equal, bit for
+bit, the same calls with the stream synchronised between them (eagerly and
+replayed from a CUDA graph). The first call is checked against the oracle.
+"""
+import numpy as np
+import pytest
+
+import iqk_synth as S
+from oracle import oracle as O
+from util import check_moe, from_dev_bf16, to_dev_bf16
+
+torch = pytest.importorskip("torch")
+pytestmark = pytest.mark.gpu
+
+LAYERS = 4
+
+
+@pytest.fixture(scope="module")
+def B():
+    from gemm_iq2_ks_b200 import binding
+    binding.lib()
+    return binding
+
+
+@pytest.mark.parametrize("T", [1, 4])
+def test_chained_decode_calls_read_the_previous_output(B, T):
+    rng = S.rng_for(800 + T)
+    E, H, F, k = 32, 1024, 512, 6
+    # small row scales keep four chained layers (quadratic through SwiGLU) finite and non-zero
+    gate, up, down = (S.random_streams(rng, "iq2_ks", E, r, c, dv_range=(3e-4, 5e-4))
+                      for r, c in ((F, H), (F, H), (H, F)))
+    values = S.value_table("dyadic", 8)
+    x0 = S.random_bf16(rng, (T, H))
+    routes = [S.routing(rng, T, E, k) for _ in range(LAYERS)]
+    dg, du, dd = (B.Weights.from_host(w) for w in (gate, up, down))
+    ids = [torch.from_numpy(i).cuda() for i, _ in routes]
+    ps = [torch.from_numpy(p).cuda() for _, p in routes]
+    ws = B.workspace(B.iqk_moe_workspace_bytes(0, T, k, E, H, F))
+    stream = torch.cuda.Stream()
+    xs = [to_dev_bf16(x0)] + [torch.empty((T, H), dtype=torch.bfloat16, device="cuda") for _ in range(LAYERS)]
+
+    def chain(sync):
+        for l in range(LAYERS):
+            B.iqk_moe_decode(dg, du, dd, values, xs[l], ids[l], ps[l], y=xs[l + 1], ws=ws, stream=stream)
+            if sync:
+                stream.synchronize()
+
+    with torch.cuda.stream(stream):
+        chain(sync=True)
+    torch.cuda.synchronize()
+    ref = [t.clone() for t in xs[1:]]
+    # the first call against the oracle
+    check_moe(from_dev_bf16(ref[0]), O.moe(gate, up, down, values, x0, routes[0][0], routes[0][1]), "layer 0")
+    for l in range(LAYERS):  # every layer's output is a real signal (the comparisons below are bitwise)
+        assert (ref[l].float() != 0).any(), f"layer {l} output is all zero"
+
+    for t in xs[1:]:
+        t.zero_()
+    torch.cuda.synchronize()
+    with torch.cuda.stream(stream):
+        chain(sync=False)
+    torch.cuda.synchronize()
+    for l in range(LAYERS):
+        assert torch.equal(xs[l + 1].view(torch.int16), ref[l].view(torch.int16)), f"eager chain, layer {l}"
+
+    for t in xs[1:]:
+        t.zero_()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(stream):
+        with torch.cuda.graph(g, stream=stream):
+            chain(sync=False)
+    for t in xs[1:]:
+        t.zero_()
+    torch.cuda.synchronize()
+    for _ in range(3):
+        with torch.cuda.stream(stream):
+            g.replay()
+    torch.cuda.synchronize()
+    for l in range(LAYERS):
+        assert torch.equal(xs[l + 1].view(torch.int16), ref[l].view(torch.int16)), f"graph chain, layer {l}"
+    del g
