@@ -367,8 +367,9 @@ __global__ void __launch_bounds__(256) k_prep(const uint16_t* __restrict__ x, in
                                               int nzero, const int32_t* __restrict__ ids, int npairs, int E,
                                               int32_t* __restrict__ status) {
   griddep_launch();
-  // Launched as a dependent of the previous call's down kernel: everything
-  // below writes workspace that kernel may still use.
+  // Launched as a dependent of whatever precedes it (the previous call's last
+  // kernel may still be writing this call's x or ids, or reading the
+  // workspace written below): nothing is read or written before the wait.
   griddep_wait();
   const int tid = blockIdx.x * blockDim.x + threadIdx.x;
   const int nth = gridDim.x * blockDim.x;
@@ -1185,7 +1186,7 @@ static cudaLaunchAttribute pdl_attr() {
 
 // The prep kernel as a programmatic dependent of whatever precedes it on the
 // stream (the previous call's last kernel triggers early); it waits before
-// its first write.
+// its first read or write.
 static int launch_prep(int blocks, cudaStream_t st, const uint16_t* x, int T, int cols, uint16_t* xp, int32_t* zero,
                        int nzero, const int32_t* ids, int npairs, int E, int32_t* status) {
   cudaLaunchConfig_t cfg = {};
