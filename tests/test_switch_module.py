@@ -72,3 +72,18 @@ def test_out_of_range_id_reports_through_status():
     y = proj(x, ids)
     assert proj.status() == B.IQK_EINVAL
     assert not y[0, 1].any()
+
+
+def test_call_checks_shapes_before_any_launch():
+    """Host-side refusals of a loaded projection (streams kept on the CPU:
+    nothing reaches the library)."""
+    torch = pytest.importorskip("torch")
+    w = S.random_streams(S.rng_for(3), "iq2_k", 4, 32, 512)
+    proj = B.IqkSwitchLinear("iq2_k", 4, 32, 512, VALS, device="cpu").load_streams(w)
+    ids = torch.zeros((2, 3), dtype=torch.int32)
+    with pytest.raises(ValueError):
+        proj(torch.zeros((2, 512), dtype=torch.float32), ids)      # not bf16
+    with pytest.raises(ValueError):
+        proj(torch.zeros((2, 256), dtype=torch.bfloat16), ids)     # wrong width
+    with pytest.raises(ValueError):
+        proj(torch.zeros((3, 512), dtype=torch.bfloat16), ids)     # leading shapes differ
