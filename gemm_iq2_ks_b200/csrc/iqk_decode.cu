@@ -360,8 +360,10 @@ __device__ __forceinline__ void build_route(const int32_t* __restrict__ ids, int
 }
 
 // ------------------------------------------------------------- prep kernel
-// Slot-transposes the activations (x[t][16w + i + 4j] -> xp[t][16w + 4i + j]),
-// zeroes the tile counters and records out-of-range expert ids.
+// Resets the status word and records out-of-range expert ids, zeroes the
+// stream kernel's tile counters (GEMV) and slot-transposes the activations
+// read through L1 (x[t][16w + i + 4j] -> xp[t][16w + 4i + j]); T = 0 skips
+// the transposition (x staged in shared memory), npairs = 0 the id check.
 __global__ void __launch_bounds__(256) k_prep(const uint16_t* __restrict__ x, int T, int cols,
                                               uint16_t* __restrict__ xp, int32_t* __restrict__ zero,
                                               int nzero, const int32_t* __restrict__ ids, int npairs, int E,
