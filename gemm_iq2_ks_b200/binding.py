@@ -22,11 +22,16 @@ FMT = {"iq2_ks": 0, "iq2_k": 1}
 EXPORTS = (
     "iqk_strerror", "iqk_last_cuda_error", "iqk_version", "iqk_row_bytes",
     "iqk_dequant", "iqk_dequant_bf16", "iqk_dequant_floor", "iqk_gemv_workspace_bytes", "iqk_gemv", "iqk_gemv_static",
-    "iqk_moe_workspace_bytes", "iqk_moe_decode", "iqk_moe_decode_shard", "iqk_f32_to_bf16",
+    "iqk_moe_workspace_bytes", "iqk_moe_workspace_layout", "iqk_moe_decode", "iqk_moe_decode_shard", "iqk_f32_to_bf16",
     "iqk_moe_prefill", "iqk_moe_status",
     "iqk_route_workspace_bytes", "iqk_moe_route", "iqk_floor",
     "iqk_switch_linear_workspace_bytes", "iqk_switch_linear",
 )
+
+
+class IqkWsLayout(ctypes.Structure):
+    _fields_ = [("status", ctypes.c_int64), ("h", ctypes.c_int64), ("h_order", ctypes.c_int64),
+                ("h_rows", ctypes.c_int32), ("reserved", ctypes.c_int32)]
 
 
 class IqkWeights(ctypes.Structure):
@@ -66,6 +71,8 @@ def lib(build_if_missing: bool = True) -> ctypes.CDLL:
             "iqk_gemv": (ctypes.c_int, [W, i32, vp, vp, i32, vp, vp, sz, vp]),
             "iqk_gemv_static": (ctypes.c_int, [W, i32, vp, vp, i32, vp, vp]),
             "iqk_moe_workspace_bytes": (sz, [i32, i32, i32, i32, i32, i32]),
+            "iqk_moe_workspace_layout": (ctypes.c_int, [i32, i32, i32, i32, i32, i32,
+                                                        ctypes.POINTER(IqkWsLayout)]),
             "iqk_moe_decode": (ctypes.c_int, [W, W, W, vp, vp, i32, vp, vp, i32, vp, vp, sz, vp]),
             "iqk_moe_decode_shard": (ctypes.c_int, [W, W, W, vp, vp, i32, vp, vp, i32, i32, vp, vp, sz, vp]),
             "iqk_f32_to_bf16": (ctypes.c_int, [vp, vp, ctypes.c_int64, vp]),
@@ -246,6 +253,13 @@ def iqk_moe_workspace_bytes(mode: int, T: int, topk: int, experts: int, hidden: 
     return lib().iqk_moe_workspace_bytes(mode, T, topk, experts, hidden, inter)
 
 
+def iqk_moe_workspace_layout(mode: int, T: int, topk: int, experts: int, hidden: int, inter: int) -> IqkWsLayout:
+    out = IqkWsLayout()
+    _check(lib().iqk_moe_workspace_layout(mode, T, topk, experts, hidden, inter, ctypes.byref(out)),
+           "iqk_moe_workspace_layout")
+    return out
+
+
 def _moe(fn, mode, gate, up, down, values, x, ids, p, y, ws, stream):
     torch = _torch()
     T, topk = ids.shape
@@ -345,6 +359,10 @@ class IqkSwitchLinear:
     streams raise ValueError before any launch; a shape the kernels do not
     take raises RuntimeError. Ids outside [0, num_experts) give zero rows and
     make ``status()`` report IQK_EINVAL.
+
+    Each (mode, shape, stream) gets its own workspace, so calls on different
+    streams never share scratch; ``status()`` reports the last call made
+    through this instance.
     """
 
     def __init__(self, member: str, num_experts: int, out_features: int, in_features: int, values,
@@ -385,7 +403,8 @@ class IqkSwitchLinear:
         xt = x.reshape(-1, self.in_features).contiguous()
         ids = indices.reshape(-1, k).to(torch.int32).contiguous()
         T = xt.shape[0]
-        key = (mode, T, k)
+        st = torch.cuda.current_stream(x.device) if stream is None else stream
+        key = (mode, T, k, st.cuda_stream)
         ws = self._ws.get(key)
         if ws is None:
             need = iqk_switch_linear_workspace_bytes(mode, T, k, self.num_experts, self.out_features,
@@ -393,11 +412,14 @@ class IqkSwitchLinear:
             if need == 0:
                 raise RuntimeError(f"IqkSwitchLinear: mode {mode} cannot take {T} tokens x {k} slots")
             ws = self._ws[key] = workspace(need, x.device)
-        self._last_ws = ws
-        y = iqk_switch_linear(self.weights, self.values, xt, ids, mode=mode, ws=ws, stream=stream)
+        self._last_ws = (ws, st)
+        y = iqk_switch_linear(self.weights, self.values, xt, ids, mode=mode, ws=ws, stream=st)
         return y.reshape(*lead, k, self.out_features)
 
     def status(self, stream=None) -> int:
         """Status of the last call as iqk_moe_status reports it: IQK_OK,
         IQK_EINVAL (an id was out of range), IQK_EUNSUPPORTED or IQK_ETIMEOUT."""
-        return 0 if self._last_ws is None else iqk_moe_status(self._last_ws, stream)
+        if self._last_ws is None:
+            return 0
+        ws, st = self._last_ws
+        return iqk_moe_status(ws, st if stream is None else stream)

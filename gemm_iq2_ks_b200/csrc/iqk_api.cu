@@ -185,6 +185,25 @@ size_t iqk_moe_workspace_bytes(int32_t mode, int32_t T, int32_t topk, int32_t ex
   return 0;
 }
 
+int iqk_moe_workspace_layout(int32_t mode, int32_t T, int32_t topk, int32_t experts, int32_t hidden,
+                             int32_t inter, iqk_ws_layout* out) {
+  if (!out || iqk_moe_workspace_bytes(mode, T, topk, experts, hidden, inter) == 0) return IQK_EINVAL;
+  memset(out, 0, sizeof(*out));
+  out->h_rows = T * topk;
+  if (mode == 0) {
+    const DecodeWs L = decode_ws(T, topk, experts, hidden, inter);
+    out->status = (int64_t)L.status;
+    out->h = (int64_t)L.hperm;
+    out->h_order = -1;
+  } else {
+    const PrefillWs L = prefill_ws(T, topk, experts, hidden, inter);
+    out->status = (int64_t)L.status;
+    out->h = (int64_t)L.hs;
+    out->h_order = (int64_t)L.perm;
+  }
+  return IQK_OK;
+}
+
 int iqk_moe_decode(const iqk_weights* gate, const iqk_weights* up, const iqk_weights* down, const float* values,
                    const uint16_t* x, int32_t T, const int32_t* ids, const float* p, int32_t topk, uint16_t* y,
                    void* workspace, size_t ws_bytes, void* stream) {

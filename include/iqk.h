@@ -253,6 +253,34 @@ int iqk_moe_prefill(const iqk_weights* gate, const iqk_weights* up, const iqk_we
                     void* workspace, size_t ws_bytes, void* stream);
 
 /*
+ * iqk_moe_workspace_layout -- where a routed-block call (mode 0 decode,
+ * mode 1 prefill; iqk_moe_decode_shard uses the decode layout) keeps its
+ * intermediates inside the caller's workspace, for inspection: the tests
+ * read the SwiGLU output h there to check the gate/up stage on its own.
+ * Arguments as iqk_moe_workspace_bytes. Fills *out and returns IQK_OK, or
+ * IQK_EINVAL (NULL out, a shape the mode cannot take).
+ *   status:  byte offset of the int32 status word (iqk_moe_status);
+ *   h:       byte offset of h, bf16 [h_rows][inter]. A row holds
+ *            bf16_rn(silu(g) * u) of one (token, slot) pair, its inter
+ *            elements slot-transposed inside every 16-element group:
+ *            element 16w + i + 4j of the pair's h sits at 16w + 4i + j.
+ *   h_order: mode 0: -1, row i is pair i = t*topk + j;
+ *            mode 1: byte offset of int32 [T*topk]: row i is pair h_order[i]
+ *            (pairs in expert order, ties in pair order, as iqk_moe_route);
+ *            rows past the number of pairs with a valid id are unused.
+ * The values belong to the last call that completed on the workspace.
+ */
+typedef struct {
+  int64_t status;
+  int64_t h;
+  int64_t h_order;
+  int32_t h_rows;
+  int32_t reserved;
+} iqk_ws_layout;
+int iqk_moe_workspace_layout(int32_t mode, int32_t T, int32_t topk, int32_t experts, int32_t hidden,
+                             int32_t inter, iqk_ws_layout* out);
+
+/*
  * iqk_moe_decode_shard -- one rank's part of an expert-parallel
  * iqk_moe_decode (the routed block's experts partitioned over ranks; each
  * rank holds the streams of experts [expert_base, expert_base + E) in

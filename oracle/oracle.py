@@ -180,17 +180,6 @@ def silu(g: np.ndarray) -> np.ndarray:
         return g / (1.0 + np.exp(-g))
 
 
-class _Cache:
-    def __init__(self, w, values):
-        self.w, self.values, self.m = w, values, {}
-
-    def __call__(self, e):
-        e = int(e)
-        if e not in self.m:
-            self.m[e] = dequant_expert(self.w, e, self.values).astype(np.float64)
-        return self.m[e]
-
-
 def silu_grad(g: np.ndarray) -> np.ndarray:
     with np.errstate(over="ignore"):
         s = 1.0 / (1.0 + np.exp(-g))
@@ -206,49 +195,63 @@ def bf16_spacing(v: np.ndarray) -> np.ndarray:
 def moe(gate, up, down, values, x_bits, ids, p, tokens=None):
     """Routed-expert block for the listed tokens (all by default).
 
-    Returns dict with
-      y_bits  bf16 [n, hidden], the rounded output;
-      y       float64 [n, hidden] before the final rounding;
-      S       sum_j p_j sum_k |Wd_jk h_jk|: the tolerance scale of the down GEMV;
-      S_prop  sum_j p_j sum_k |Wd_jk| (|dh/dg| S_g + |dh/du| S_u)_k: how far y
-              can move when g and u are each off by their own GEMV scale
-              S_g = sum |Wg x|, S_u = sum |Wu x| (first-order propagation
-              through h = silu(g) u);
-      S_round sum_j p_j sum_k |Wd_jk| * spacing_bf16(h_jk): y's reach when h
-              rounds to the neighbouring bfloat16;
-      h_bits  bf16 [n, topk, inter].
+    For every (token t, slot j) pair with expert e = ids[t, j]:
+      g = Wg_e x_t, u = Wu_e x_t (float64), h = bf16_rn(float32(silu(g) * u)),
+    and y_t = sum_j p_tj * (Wd_e h) in float64, output bf16_rn(float32(y_t)).
+    The pairs are visited expert by expert (each expert's three matrices are
+    dequantized once per call); the sum over a token's slots is a plain sum,
+    so its order does not enter the definition.
+
+    Returns a dict with
+      y_bits   bf16 [n, hidden], the rounded output;
+      y        float64 [n, hidden] before the final rounding;
+      S        sum_j |p_j| sum_f |Wd_jf h_jf|: the scale of the down GEMV's
+               stated tolerance;
+      h_bits   bf16 [n, topk, inter];
+      g, u     the gate and up GEMV results [n, topk, inter] (computed in
+               float64, stored as float32);
+      S_g, S_u their scales sum_k |w x| (same storage).
+    Expert ids must lie in [0, experts).
     """
     x_bits = np.atleast_2d(x_bits)
-    ids = np.atleast_2d(ids)
-    p = np.atleast_2d(p)
-    toks = list(range(x_bits.shape[0])) if tokens is None else list(tokens)
-    Wg, Wu, Wd = _Cache(gate, values), _Cache(up, values), _Cache(down, values)
-    topk = ids.shape[1]
+    ids = np.atleast_2d(np.asarray(ids))
+    p = np.atleast_2d(np.asarray(p))
+    toks = np.arange(x_bits.shape[0]) if tokens is None else np.asarray(list(tokens), np.int64)
+    idn = ids[toks].astype(np.int64)
+    if idn.size and (idn.min() < 0 or idn.max() >= gate.experts):
+        raise ValueError("expert id out of range")
+    pn = p[toks].astype(np.float64)
+    xs = bf16_to_float(x_bits[toks]).astype(np.float64)
+    n, topk = idn.shape
     H, F = down.rows, down.cols
-    y = np.zeros((len(toks), H))
-    S = np.zeros((len(toks), H))
-    S_prop = np.zeros((len(toks), H))
-    S_round = np.zeros((len(toks), H))
-    hb = np.zeros((len(toks), topk, F), np.uint16)
-    for n, t in enumerate(toks):
-        x = bf16_to_float(x_bits[t]).astype(np.float64)
-        ax = np.abs(x)
-        for j in range(topk):
-            e = int(ids[t, j])
-            wg, wu = Wg(e), Wu(e)
-            g = wg @ x
-            u = wu @ x
-            hb[n, j] = bf16_round((silu(g) * u).astype(np.float32))
-            h = bf16_to_float(hb[n, j]).astype(np.float64)
-            wd = Wd(e)
-            pj = float(p[t, j])
-            awd = np.abs(wd)
-            y[n] += pj * (wd @ h)
-            S[n] += pj * (awd @ np.abs(h))
-            reach = np.abs(u * silu_grad(g)) * (np.abs(wg) @ ax) + np.abs(silu(g)) * (np.abs(wu) @ ax)
-            S_prop[n] += pj * (awd @ reach)
-            S_round[n] += pj * (awd @ bf16_spacing(h))
-    return dict(y_bits=bf16_round(y.astype(np.float32)), y=y, S=S, S_prop=S_prop, S_round=S_round, h_bits=hb)
+    y = np.zeros((n, H))
+    S = np.zeros((n, H))
+    hb = np.zeros((n, topk, F), np.uint16)
+    g_out = np.zeros((n, topk, F), np.float32)
+    u_out = np.zeros((n, topk, F), np.float32)
+    sg_out = np.zeros((n, topk, F), np.float32)
+    su_out = np.zeros((n, topk, F), np.float32)
+    for e in np.unique(idn):
+        rows_n, slots = np.nonzero(idn == e)
+        X = xs[rows_n]
+        aX = np.abs(X)
+        wg = dequant_expert(gate, int(e), values).astype(np.float64)
+        wu = dequant_expert(up, int(e), values).astype(np.float64)
+        G = X @ wg.T
+        U = X @ wu.T
+        h = bf16_round((silu(G) * U).astype(np.float32))
+        hf = bf16_to_float(h).astype(np.float64)
+        wd = dequant_expert(down, int(e), values).astype(np.float64)
+        pw = pn[rows_n, slots][:, None]
+        np.add.at(y, rows_n, pw * (hf @ wd.T))
+        np.add.at(S, rows_n, np.abs(pw) * (np.abs(hf) @ np.abs(wd).T))
+        hb[rows_n, slots] = h
+        g_out[rows_n, slots] = G
+        u_out[rows_n, slots] = U
+        sg_out[rows_n, slots] = aX @ np.abs(wg).T
+        su_out[rows_n, slots] = aX @ np.abs(wu).T
+    return dict(y_bits=bf16_round(y.astype(np.float32)), y=y, S=S, h_bits=hb, g=g_out, u=u_out,
+                S_g=sg_out, S_u=su_out)
 
 
 # -------------------------------------------------------------- switch linear

@@ -122,3 +122,25 @@ def test_strerror_covers_every_status():
     for rc in range(0, -7, -1):
         assert L.iqk_strerror(rc) not in (b"", b"unknown status")
     assert L.iqk_strerror(-99) == b"unknown status"
+
+
+def test_workspace_layout_inside_the_workspace():
+    """The intermediates' offsets lie inside the workspace the same call
+    needs, aligned, and the layout refuses shapes the mode cannot take."""
+    for mode, T, k, E, H, F in [(0, 1, 6, 256, 4096, 2048), (0, 64, 16, 40, 256, 512), (1, 2048, 6, 256, 4096, 2048),
+                                (1, 5, 3, 8, 256, 256)]:
+        need = B.iqk_moe_workspace_bytes(mode, T, k, E, H, F)
+        L = B.iqk_moe_workspace_layout(mode, T, k, E, H, F)
+        assert L.h_rows == T * k
+        assert L.status == 0
+        assert L.h % 256 == 0 and L.h + L.h_rows * F * 2 <= need
+        if mode == 0:
+            assert L.h_order == -1
+        else:
+            assert L.h_order % 256 == 0 and L.h_order + T * k * 4 <= need
+            assert not (L.h_order < L.h + L.h_rows * F * 2 and L.h < L.h_order + T * k * 4)
+    lib = B.lib()
+    out = B.IqkWsLayout()
+    assert lib.iqk_moe_workspace_layout(0, 65, 6, 4, 256, 512, ctypes.byref(out)) == B.IQK_EINVAL
+    assert lib.iqk_moe_workspace_layout(2, 1, 6, 4, 256, 512, ctypes.byref(out)) == B.IQK_EINVAL
+    assert lib.iqk_moe_workspace_layout(0, 1, 6, 4, 256, 512, None) == B.IQK_EINVAL

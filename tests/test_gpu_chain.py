@@ -13,7 +13,7 @@ import pytest
 
 import iqk_synth as S
 from oracle import oracle as O
-from util import check_moe, from_dev_bf16, to_dev_bf16
+from util import check_block, from_dev_bf16, read_h, run_block, to_dev_bf16
 
 torch = pytest.importorskip("torch")
 pytestmark = pytest.mark.gpu
@@ -55,8 +55,11 @@ def test_chained_decode_calls_read_the_previous_output(B, T):
         chain(sync=True)
     torch.cuda.synchronize()
     ref = [t.clone() for t in xs[1:]]
-    # the first call against the oracle
-    check_moe(from_dev_bf16(ref[0]), O.moe(gate, up, down, values, x0, routes[0][0], routes[0][1]), "layer 0")
+    # the first call against the oracle (its h from a fresh workspace)
+    y0, h0 = run_block(B, gate, up, down, values, x0, routes[0][0], routes[0][1])
+    assert np.array_equal(y0, from_dev_bf16(ref[0]))
+    check_block(y0, h0, O.moe(gate, up, down, values, x0, routes[0][0], routes[0][1]), down, values, routes[0][0],
+                routes[0][1], "layer 0")
     for l in range(LAYERS):  # every layer's output is a real signal (the comparisons below are bitwise)
         assert (ref[l].float() != 0).any(), f"layer {l} output is all zero"
 

@@ -6,7 +6,7 @@ import pytest
 import iqk_synth as S
 from oracle import oracle as O
 from tests.encode import encode, idx_range, sub_size
-from tests.util import check_fp32, check_moe, from_dev_bf16, to_dev_bf16
+from tests.util import check_block, check_fp32, flat_stats, from_dev_bf16, read_h, run_block, to_dev_bf16
 
 pytestmark = pytest.mark.gpu
 
@@ -115,36 +115,30 @@ def _moe_case(seed, fg, fu, fd, E, H, F, T, topk):
     return gate, up, down, x, ids, p
 
 
-def _run_decode(B, gate, up, down, values, x, ids, p, prefill=False):
-    dg, du, dd = (B.Weights.from_host(w) for w in (gate, up, down))
-    fn = B.iqk_moe_prefill if prefill else B.iqk_moe_decode
-    y = fn(dg, du, dd, values, to_dev_bf16(x), torch.from_numpy(ids).cuda(), torch.from_numpy(p).cuda())
-    torch.cuda.synchronize()
-    return from_dev_bf16(y)
+def _check(B, gate, up, down, values, x, ids, p, what, report):
+    y, h = run_block(B, gate, up, down, values, x, ids, p)
+    ref = O.moe(gate, up, down, values, x, ids, p)
+    out = check_block(y, h, ref, down, values, ids, p, what)
+    report(what, flat_stats(out))
+    return out
 
 
 @pytest.mark.parametrize("fmts", [("iq2_ks",) * 3, ("iq2_k",) * 3, ("iq2_ks", "iq2_k", "iq2_ks"),
                                   ("iq2_k", "iq2_ks", "iq2_k")])
 @pytest.mark.parametrize("T", [1, 4, 16])
-def test_moe_decode_small(B, fmts, T):
+def test_moe_decode_small(B, fmts, T, parity_report):
     gate, up, down, x, ids, p = _moe_case(50 + T, *fmts, E=12, H=512, F=768, T=T, topk=6)
-    values = S.value_table("int", 1)
-    y = _run_decode(B, gate, up, down, values, x, ids, p)
-    ref = O.moe(gate, up, down, values, x, ids, p)
-    check_moe(y, ref, f"decode {fmts} T={T}")
+    _check(B, gate, up, down, S.value_table("int", 1), x, ids, p, f"decode {fmts} T={T}", parity_report)
 
 
-def test_moe_decode_topk_edge(B):
+def test_moe_decode_topk_edge(B, parity_report):
     """topk = 1 and topk = 16, T = 64 (the decode limits)."""
     for T, k in [(3, 1), (64, 16)]:
         gate, up, down, x, ids, p = _moe_case(60 + k, "iq2_ks", "iq2_ks", "iq2_k", E=40, H=256, F=256, T=T, topk=k)
-        values = S.value_table("f16", 2)
-        y = _run_decode(B, gate, up, down, values, x, ids, p)
-        ref = O.moe(gate, up, down, values, x, ids, p)
-        check_moe(y, ref, f"decode T={T} topk={k}")
+        _check(B, gate, up, down, S.value_table("f16", 2), x, ids, p, f"decode T={T} topk={k}", parity_report)
 
 
-def test_moe_decode_bad_ids_skipped_and_flagged(B):
+def test_moe_decode_bad_ids_skipped_and_flagged(B, parity_report):
     gate, up, down, x, ids, p = _moe_case(77, "iq2_ks", "iq2_ks", "iq2_ks", E=8, H=256, F=256, T=2, topk=3)
     values = S.value_table("int", 0)
     bad = ids.copy()
@@ -162,7 +156,10 @@ def test_moe_decode_bad_ids_skipped_and_flagged(B):
     fixed[0, 1] = 0
     fixed[1, 2] = 0
     ref = O.moe(gate, up, down, values, x, fixed, pv)
-    check_moe(from_dev_bf16(y), ref, "bad ids")
+    h = read_h(B, ws, 0, 2, 3, 8, 256, 256)
+    valid = (bad >= 0) & (bad < 8)
+    out = check_block(from_dev_bf16(y), h, ref, down, values, fixed, pv, "bad ids", pairs=valid)
+    parity_report("bad ids", flat_stats(out))
     # a clean call resets the status word
     B.iqk_moe_decode(dg, du, dd, values, to_dev_bf16(x), torch.from_numpy(ids).cuda(),
                      torch.from_numpy(p).cuda(), ws=ws)
@@ -182,27 +179,25 @@ def full_k(B):
     return S.moe_weights(rng, "iq2_k", S.EXPERTS, S.HIDDEN, S.INTER)
 
 
-def test_moe_decode_full_iq2_ks_e256_top6(B, full_ks):
+@pytest.mark.parametrize("table", ["int", "f16"])
+def test_moe_decode_full_iq2_ks_e256_top6(B, full_ks, table, parity_report):
     gate, up, down = full_ks
     rng = S.rng_for(20)
     x = S.random_bf16(rng, (1, S.HIDDEN))
     ids, p = S.routing(rng, 1, S.EXPERTS, S.TOPK)
-    values = S.value_table("int", 2)
-    y = _run_decode(B, gate, up, down, values, x, ids, p)
-    ref = O.moe(gate, up, down, values, x, ids, p)
-    check_moe(y, ref, "IQ2_KS decode, 256 experts, top-6, 1 token")
+    _check(B, gate, up, down, S.value_table(table, 2), x, ids, p,
+           f"IQ2_KS decode, 256 experts, top-6, 1 token, {table} table", parity_report)
 
 
 @pytest.mark.parametrize("T", [1, 4, 16])
-def test_moe_decode_full_iq2_k_e256_top6(B, full_k, T):
+@pytest.mark.parametrize("table", ["int", "f16"])
+def test_moe_decode_full_iq2_k_e256_top6(B, full_k, T, table, parity_report):
     gate, up, down = full_k
     rng = S.rng_for(30 + T)
     x = S.random_bf16(rng, (T, S.HIDDEN))
     ids, p = S.routing(rng, T, S.EXPERTS, S.TOPK)
-    values = S.value_table("f16", 3)
-    y = _run_decode(B, gate, up, down, values, x, ids, p)
-    ref = O.moe(gate, up, down, values, x, ids, p)
-    check_moe(y, ref, f"IQ2_K decode, 256 experts, top-6, T={T}")
+    _check(B, gate, up, down, S.value_table(table, 3), x, ids, p,
+           f"IQ2_K decode, 256 experts, top-6, T={T}, {table} table", parity_report)
 
 
 # ------------------------------------------------------------------- route
@@ -251,7 +246,7 @@ def test_dequant_floor_bitexact(B, fmt, rows, cols, bf16):
         assert np.array_equal(out, O.dequant_floor(w, e, bf16=bf16)), (fmt, rows, cols, bf16, e)
 
 
-def test_moe_decode_duplicate_ids(B):
+def test_moe_decode_duplicate_ids(B, parity_report):
     """A token listing one expert twice: both slots are computed as separate
     pairs. One token listing one expert in all twelve slots: more pairs than
     one MMA column group, split into runs, each run a separate pass."""
@@ -259,30 +254,30 @@ def test_moe_decode_duplicate_ids(B):
     ids = ids.copy()
     ids[0, 1] = ids[0, 0]
     ids[1, 3] = ids[1, 2]
-    dg, du, dd = (B.Weights.from_host(w) for w in (gate, up, down))
     vals = S.value_table("int", 3)
     ws = B.workspace(B.iqk_moe_workspace_bytes(0, 2, 4, 12, 512, 768))
-    y = B.iqk_moe_decode(dg, du, dd, vals, to_dev_bf16(x), torch.from_numpy(ids).cuda(),
-                         torch.from_numpy(p).cuda(), ws=ws)
+    _check_ws(B, gate, up, down, vals, x, ids, p, ws, "duplicate ids", parity_report)
     assert B.iqk_moe_status(ws) == B.IQK_OK
-    check_moe(from_dev_bf16(y), O.moe(gate, up, down, vals, x, ids, p), "duplicate ids")
     ids12 = np.full((1, 12), 5, np.int32)
     p12 = np.full((1, 12), 1.0 / 12, np.float32)
     ws12 = B.workspace(B.iqk_moe_workspace_bytes(0, 1, 12, 12, 512, 768))
-    y12 = B.iqk_moe_decode(dg, du, dd, vals, to_dev_bf16(x[:1]), torch.from_numpy(ids12).cuda(),
-                           torch.from_numpy(p12).cuda(), ws=ws12)
+    _check_ws(B, gate, up, down, vals, x[:1], ids12, p12, ws12, "twelve slots, one expert", parity_report)
     assert B.iqk_moe_status(ws12) == B.IQK_OK
-    check_moe(from_dev_bf16(y12), O.moe(gate, up, down, vals, x[:1], ids12, p12), "twelve slots, one expert")
 
 
 @pytest.mark.parametrize("T,topk,E,dup", [(2, 10, 20, True), (33, 6, 12, False), (40, 4, 64, False)])
-def test_moe_decode_runs_of_pairs(B, T, topk, E, dup):
+def test_moe_decode_runs_of_pairs(B, T, topk, E, dup, parity_report):
     """Experts with more pairs than the MMA columns: split into runs (one
     column group when experts average at most 8 pairs, two otherwise)."""
     gate, up, down, x, ids, p = _moe_case(300 + T, "iq2_k", "iq2_ks", "iq2_ks", E=E, H=512, F=256, T=T, topk=topk)
     if dup:  # token 0 puts one expert in every slot: 10 pairs, 2 runs of one column group
         ids = ids.copy()
         ids[0, :] = ids[1, 0]
-    values = S.value_table("f16", 6)
-    y = _run_decode(B, gate, up, down, values, x, ids, p)
-    check_moe(y, O.moe(gate, up, down, values, x, ids, p), f"decode runs T={T} topk={topk} E={E}")
+    _check(B, gate, up, down, S.value_table("f16", 6), x, ids, p, f"decode runs T={T} topk={topk} E={E}",
+           parity_report)
+
+
+def _check_ws(B, gate, up, down, values, x, ids, p, ws, what, report):
+    y, h = run_block(B, gate, up, down, values, x, ids, p, ws=ws)
+    out = check_block(y, h, O.moe(gate, up, down, values, x, ids, p), down, values, ids, p, what)
+    report(what, flat_stats(out))

@@ -1,11 +1,12 @@
 """GPU parity of the tcgen05 prefill path against the CPU oracle (the prefill
-reference is the decode reference applied per token)."""
+reference is the decode reference applied per token). Both stages of the
+block are checked: the SwiGLU output h read back from the workspace, and y."""
 import numpy as np
 import pytest
 
 import iqk_synth as S
 from oracle import oracle as O
-from tests.util import check_moe, from_dev_bf16, to_dev_bf16
+from tests.util import check_block, flat_stats, from_dev_bf16, read_h, run_block, to_dev_bf16
 
 pytestmark = pytest.mark.gpu
 
@@ -35,50 +36,38 @@ def _case(seed, fmts, E, H, F, T, topk, skew=None):
     return gate, up, down, x, ids, p
 
 
-def _prefill(B, gate, up, down, values, x, ids, p, ws=None):
-    dg, du, dd = (B.Weights.from_host(w) for w in (gate, up, down))
-    y = B.iqk_moe_prefill(dg, du, dd, values, to_dev_bf16(x), torch.from_numpy(ids).cuda(),
-                          torch.from_numpy(p).cuda(), ws=ws)
-    torch.cuda.synchronize()
-    return from_dev_bf16(y)
+def _check(B, gate, up, down, values, x, ids, p, what, report, prefill=True):
+    y, h = run_block(B, gate, up, down, values, x, ids, p, prefill=prefill)
+    out = check_block(y, h, O.moe(gate, up, down, values, x, ids, p), down, values, ids, p, what)
+    report(what, flat_stats(out))
+    return y
 
 
 @pytest.mark.parametrize("fmts", [("iq2_ks",) * 3, ("iq2_k",) * 3, ("iq2_ks", "iq2_k", "iq2_k"),
                                   ("iq2_k", "iq2_ks", "iq2_ks")])
 @pytest.mark.parametrize("T", [1, 37, 300])
-def test_prefill_small(B, fmts, T):
+def test_prefill_small(B, fmts, T, parity_report):
     gate, up, down, x, ids, p = _case(200 + T, fmts, E=8, H=512, F=512, T=T, topk=6)
-    values = S.value_table("int", 5)
-    y = _prefill(B, gate, up, down, values, x, ids, p)
-    ref = O.moe(gate, up, down, values, x, ids, p)
-    check_moe(y, ref, f"prefill {fmts} T={T}")
+    _check(B, gate, up, down, S.value_table("int", 5), x, ids, p, f"prefill {fmts} T={T}", parity_report)
 
 
-def test_prefill_many_pairs_per_expert(B):
+def test_prefill_many_pairs_per_expert(B, parity_report):
     """One expert receives every token (> 128 pairs: several N tiles);
     ragged pair counts on the others; f16 table."""
     gate, up, down, x, ids, p = _case(300, ("iq2_ks",) * 3, E=6, H=768, F=512, T=333, topk=2, skew=3)
-    values = S.value_table("f16", 6)
-    y = _prefill(B, gate, up, down, values, x, ids, p)
-    ref = O.moe(gate, up, down, values, x, ids, p)
-    check_moe(y, ref, "prefill skewed")
+    _check(B, gate, up, down, S.value_table("f16", 6), x, ids, p, "prefill skewed", parity_report)
 
 
-def test_prefill_matches_decode_math(B):
+def test_prefill_matches_decode_math(B, parity_report):
     """Decode and prefill compute the same block: both within tolerance of
     the oracle on the same inputs (T=16, 64 experts)."""
     gate, up, down, x, ids, p = _case(301, ("iq2_k",) * 3, E=64, H=1024, F=512, T=16, topk=6)
     values = S.value_table("int", 7)
-    ref = O.moe(gate, up, down, values, x, ids, p)
-    y_pf = _prefill(B, gate, up, down, values, x, ids, p)
-    check_moe(y_pf, ref, "prefill")
-    dg, du, dd = (B.Weights.from_host(w) for w in (gate, up, down))
-    y_dec = B.iqk_moe_decode(dg, du, dd, values, to_dev_bf16(x), torch.from_numpy(ids).cuda(),
-                             torch.from_numpy(p).cuda())
-    check_moe(from_dev_bf16(y_dec), ref, "decode")
+    _check(B, gate, up, down, values, x, ids, p, "prefill", parity_report)
+    _check(B, gate, up, down, values, x, ids, p, "decode", parity_report, prefill=False)
 
 
-def test_prefill_bad_ids(B):
+def test_prefill_bad_ids(B, parity_report):
     gate, up, down, x, ids, p = _case(302, ("iq2_ks",) * 3, E=8, H=256, F=256, T=5, topk=3)
     values = S.value_table("int", 0)
     bad = ids.copy()
@@ -92,21 +81,45 @@ def test_prefill_bad_ids(B):
     pv[2, 1] = 0
     fixed = ids.copy()
     fixed[2, 1] = 0
-    ref = O.moe(gate, up, down, values, x, fixed, pv)
-    check_moe(from_dev_bf16(y), ref, "prefill bad ids")
+    valid = (bad >= 0) & (bad < 8)
+    h = read_h(B, ws, 1, 5, 3, 8, 256, 256, valid_pairs=int(valid.sum()))
+    out = check_block(from_dev_bf16(y), h, O.moe(gate, up, down, values, x, fixed, pv), down, values, fixed, pv,
+                      "prefill bad ids", pairs=valid)
+    parity_report("prefill bad ids", flat_stats(out))
 
 
-def test_prefill_full_iq2_ks_e256_top6_2048_sampled(B):
-    """The prefill workload at full size (2048 tokens, 256 experts, top-6, IQ2_KS);
-    sampled tokens checked against the oracle one by one, every output finite."""
+@pytest.fixture(scope="module")
+def full_prefill(B):
+    """The prefill workload at full size: 2048 tokens, 256 experts, top-6,
+    IQ2_KS (about 48 pairs per expert), int table."""
     rng = S.rng_for(4)
     gate, up, down = S.moe_weights(rng, "iq2_ks", S.EXPERTS, S.HIDDEN, S.INTER)
     x = S.random_bf16(rng, (2048, S.HIDDEN))
     ids, p = S.routing(rng, 2048, S.EXPERTS, S.TOPK)
     values = S.value_table("int", 4)
-    y = _prefill(B, gate, up, down, values, x, ids, p)
-    yf = (y.astype(np.uint32) << 16).view(np.float32)
-    assert np.all(np.isfinite(yf))
-    sample = np.random.default_rng(0).choice(2048, size=12, replace=False)
-    ref = O.moe(gate, up, down, values, x, ids, p, tokens=sample)
-    check_moe(y[sample], ref, "prefill 2048 tokens, sampled")
+    y, h = run_block(B, gate, up, down, values, x, ids, p, prefill=True)
+    return gate, up, down, values, x, ids, p, y, h
+
+
+def test_prefill_full_every_expert_last_tile(B, full_prefill, parity_report):
+    """Tokens chosen so that every expert's last (ragged) N tile of pairs is
+    checked: for each expert, the token of its last pair in expert order."""
+    gate, up, down, values, x, ids, p, y, h = full_prefill
+    flat = ids.reshape(-1)
+    order = np.argsort(flat, kind="stable")
+    last = {}
+    for i in order:
+        last[int(flat[i])] = int(i) // ids.shape[1]
+    toks = np.array(sorted(set(last.values())))
+    ref = O.moe(gate, up, down, values, x, ids, p, tokens=toks)
+    out = check_block(y[toks], h[toks], ref, down, values, ids[toks], p[toks],
+                      f"prefill 2048 tokens, {len(toks)} tokens covering every expert's last tile")
+    parity_report("prefill 2048, last tiles", flat_stats(out))
+
+
+def test_prefill_full_all_tokens(B, full_prefill, parity_report):
+    """Every output and every h of the full prefill workload."""
+    gate, up, down, values, x, ids, p, y, h = full_prefill
+    ref = O.moe(gate, up, down, values, x, ids, p)
+    out = check_block(y, h, ref, down, values, ids, p, "prefill 2048 tokens, all")
+    parity_report("prefill 2048, all tokens", flat_stats(out))

@@ -11,7 +11,7 @@ import pytest
 import iqk_synth as S
 from gemm_iq2_ks_b200 import binding as B
 from oracle import oracle as O
-from util import TOL, check_fp32, to_dev_bf16
+from util import check_fp32, to_dev_bf16
 
 
 def test_static_scratch_limit_is_refused_on_the_host():
@@ -35,8 +35,10 @@ def test_static_matches_workspace_gemv_twice(case, T):
     dw = B.Weights.from_host(w)
     xd = to_dev_bf16(x)
     y_ws = B.iqk_gemv(dw, 0, values, xd).cpu().numpy().astype(np.float64)
-    _, Sabs = O.gemv(O.dequant_expert(w, 0, values), x)
+    y_ref, Sabs = O.gemv(O.dequant_expert(w, 0, values), x)
     for k in range(2):  # two calls in a row reuse the same scratch
         y_st = B.iqk_gemv_static(dw, 0, values, xd).cpu().numpy()
-        check_fp32(y_st, y_ws, Sabs, f"static gemv {case} T={T} call {k}")
-        assert np.max(np.abs(y_st - y_ws) / np.maximum(Sabs, 1e-30)) <= TOL
+        # against the workspace entry point, within the stated tolerance ...
+        check_fp32(y_st, y_ws, Sabs, f"static gemv vs iqk_gemv, {case} T={T} call {k}")
+        # ... and against the oracle
+        check_fp32(y_st, y_ref, Sabs, f"static gemv vs oracle, {case} T={T} call {k}")
