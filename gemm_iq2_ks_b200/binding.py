@@ -23,8 +23,8 @@ EXPORTS = (
     "iqk_strerror", "iqk_last_cuda_error", "iqk_version", "iqk_row_bytes",
     "iqk_dequant", "iqk_dequant_bf16", "iqk_dequant_floor", "iqk_gemv_workspace_bytes", "iqk_gemv", "iqk_gemv_static",
     "iqk_moe_workspace_bytes", "iqk_moe_workspace_layout", "iqk_moe_decode", "iqk_moe_decode_shard", "iqk_f32_to_bf16",
-    "iqk_moe_prefill", "iqk_moe_status",
-    "iqk_route_workspace_bytes", "iqk_moe_route", "iqk_floor",
+    "iqk_moe_prefill", "iqk_moe_prefill_shard", "iqk_moe_combine", "iqk_moe_status",
+    "iqk_route_workspace_bytes", "iqk_moe_route", "iqk_floor", "iqk_floor_status", "iqk_set_wait_limit_ns",
     "iqk_switch_linear_workspace_bytes", "iqk_switch_linear",
 )
 
@@ -77,10 +77,14 @@ def lib(build_if_missing: bool = True) -> ctypes.CDLL:
             "iqk_moe_decode_shard": (ctypes.c_int, [W, W, W, vp, vp, i32, vp, vp, i32, i32, vp, vp, sz, vp]),
             "iqk_f32_to_bf16": (ctypes.c_int, [vp, vp, ctypes.c_int64, vp]),
             "iqk_moe_prefill": (ctypes.c_int, [W, W, W, vp, vp, i32, vp, vp, i32, vp, vp, sz, vp]),
+            "iqk_moe_prefill_shard": (ctypes.c_int, [W, W, W, vp, vp, i32, vp, vp, i32, i32, vp, vp, sz, vp]),
+            "iqk_moe_combine": (ctypes.c_int, [vp, vp, i32, i32, i32, vp, vp]),
             "iqk_moe_status": (ctypes.c_int, [vp, vp]),
             "iqk_route_workspace_bytes": (sz, [i32, i32, i32]),
             "iqk_moe_route": (ctypes.c_int, [vp, i32, i32, i32, vp, vp, vp, vp, sz, vp]),
             "iqk_floor": (ctypes.c_int, [W, vp, i32, vp, vp]),
+            "iqk_floor_status": (ctypes.c_int, [vp]),
+            "iqk_set_wait_limit_ns": (ctypes.c_int, [ctypes.c_uint64, i32]),
             "iqk_switch_linear_workspace_bytes": (sz, [i32, i32, i32, i32, i32, i32]),
             "iqk_switch_linear": (ctypes.c_int, [W, vp, vp, i32, vp, i32, vp, i32, vp, sz, vp]),
         }
@@ -300,6 +304,33 @@ def iqk_moe_decode_shard(gate: Weights, up: Weights, down: Weights, values, x, i
     return y
 
 
+def iqk_moe_prefill_shard(gate: Weights, up: Weights, down: Weights, values, x, ids, p, expert_base: int,
+                          y=None, ws=None, stream=None):
+    """One expert-parallel rank's float32 prefill partial [T, hidden]."""
+    torch = _torch()
+    T, topk = ids.shape
+    y = _empty((T, down.rows), torch.float32, x.device) if y is None else y
+    if ws is None:
+        ws = workspace(iqk_moe_workspace_bytes(1, T, topk, gate.experts, gate.cols, gate.rows), x.device)
+    v = _values(values)
+    _check(lib().iqk_moe_prefill_shard(ctypes.byref(gate.c), ctypes.byref(up.c), ctypes.byref(down.c),
+                                       v.ctypes.data, x.data_ptr(), T, ids.data_ptr(), p.data_ptr(), topk,
+                                       expert_base, y.data_ptr(), ws.data_ptr(), ws.numel(), _stream(stream)),
+           "iqk_moe_prefill_shard")
+    return y
+
+
+def iqk_moe_combine(rows, p, y=None, stream=None):
+    """y[t] = bf16(sum_j p[t, j] rows[t * topk + j]) in slot order."""
+    torch = _torch()
+    T, topk = p.shape
+    H = rows.shape[-1]
+    y = _empty((T, H), torch.bfloat16, rows.device) if y is None else y
+    _check(lib().iqk_moe_combine(rows.data_ptr(), p.data_ptr(), T, topk, H, y.data_ptr(), _stream(stream)),
+           "iqk_moe_combine")
+    return y
+
+
 def iqk_f32_to_bf16(x, out=None, stream=None):
     torch = _torch()
     out = _empty(tuple(x.shape), torch.bfloat16, x.device) if out is None else out
@@ -335,6 +366,14 @@ def iqk_floor(w: Weights, expert_list, out=None, stream=None):
     _check(lib().iqk_floor(ctypes.byref(w.c), expert_list.data_ptr(), n, out.data_ptr(), _stream(stream)),
            "iqk_floor")
     return out
+
+
+def iqk_floor_status(stream=None) -> int:
+    return lib().iqk_floor_status(_stream(stream))
+
+
+def iqk_set_wait_limit_ns(limit_ns: int, expire: bool = False) -> int:
+    return lib().iqk_set_wait_limit_ns(int(limit_ns), int(bool(expire)))
 
 
 # --------------------------------------------------------------- module form

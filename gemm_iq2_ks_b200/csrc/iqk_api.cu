@@ -264,8 +264,39 @@ int iqk_moe_prefill(const iqk_weights* gate, const iqk_weights* up, const iqk_we
   if ((rc = check_ws(workspace, ws_bytes, prefill_ws(T, topk, g.experts, g.cols, g.rows).total))) return rc;
   const int sms = num_sms();
   if (sms < 0) return cuda_fail(cudaGetLastError());
-  return from_launch(launch_moe_prefill(g, gate->fmt, u, up->fmt, d, down->fmt, V, x, T, ids, p, topk, y,
-                                        (char*)workspace, (cudaStream_t)stream, sms));
+  return from_launch(launch_moe_prefill(g, gate->fmt, u, up->fmt, d, down->fmt, V, x, T, ids, p, topk, y, nullptr,
+                                        0, (char*)workspace, (cudaStream_t)stream, sms));
+}
+
+int iqk_moe_prefill_shard(const iqk_weights* gate, const iqk_weights* up, const iqk_weights* down,
+                          const float* values, const uint16_t* x, int32_t T, const int32_t* ids, const float* p,
+                          int32_t topk, int32_t expert_base, float* y_partial, void* workspace, size_t ws_bytes,
+                          void* stream) {
+  WDev g, u, d;
+  Values V;
+  int rc;
+  if ((rc = check_moe(gate, up, down, &g, &u, &d)) || (rc = check_values(values, &V))) return rc;
+  if (!x || !ids || !p || !y_partial || expert_base < 0) return IQK_EINVAL;
+  if (T == 0) return IQK_OK;
+  if (T < 0 || topk < 1 || topk > 16) return IQK_EINVAL;
+  if (T > 65536) return IQK_EUNSUPPORTED;
+  if (!aligned(x, 16) || !aligned(y_partial, 16)) return IQK_EINVAL;
+  if ((rc = check_ws(workspace, ws_bytes, prefill_ws(T, topk, g.experts, g.cols, g.rows).total))) return rc;
+  const int sms = num_sms();
+  if (sms < 0) return cuda_fail(cudaGetLastError());
+  return from_launch(launch_moe_prefill(g, gate->fmt, u, up->fmt, d, down->fmt, V, x, T, ids, p, topk, nullptr,
+                                        y_partial, expert_base, (char*)workspace, (cudaStream_t)stream, sms));
+}
+
+int iqk_moe_combine(const float* rows, const float* p, int32_t T, int32_t topk, int32_t hidden, uint16_t* y,
+                    void* stream) {
+  if (T == 0) return IQK_OK;
+  if (!rows || !p || !y || T < 0 || topk < 1 || topk > 16) return IQK_EINVAL;
+  if (hidden <= 0 || hidden % 4) return IQK_ESHAPE;
+  if (!aligned(rows, 16) || !aligned(y, 8)) return IQK_EINVAL;
+  const int sms = num_sms();
+  if (sms < 0) return cuda_fail(cudaGetLastError());
+  return from_launch(launch_combine(rows, p, T, topk, hidden, y, (cudaStream_t)stream, sms));
 }
 
 int iqk_moe_status(const void* workspace, void* stream) {
@@ -305,6 +336,17 @@ int iqk_floor(const iqk_weights* w, const int32_t* expert_list, int32_t n_expert
   const int sms = num_sms();
   if (sms < 0) return cuda_fail(cudaGetLastError());
   return from_launch(launch_floor(wd, w->fmt, expert_list, n_experts, out, (cudaStream_t)stream, sms));
+}
+
+int iqk_floor_status(void* stream) {
+  int32_t s = 0;
+  if (read_floor_status((cudaStream_t)stream, &s)) return cuda_fail(cudaGetLastError());
+  return (s & 2) ? IQK_ETIMEOUT : IQK_OK;
+}
+
+int iqk_set_wait_limit_ns(uint64_t limit_ns, int32_t expire) {
+  set_wait_limit(limit_ns, expire);
+  return IQK_OK;
 }
 
 }  // extern "C"

@@ -21,17 +21,26 @@
 // (device-scope counter) sums them in slice order. Either way results do not
 // depend on arrival order.
 #include <algorithm>
+#include <atomic>
 
 #include "iqk_device.cuh"
 #include "iqk_internal.h"
 
 // Selector arithmetic of the code lookup: 0 all shifts on the integer-logic
-// pipe (the default: fastest measured on B200 with the unrolled item loop);
-// 1 the high-half selector by multiply-high; 2 as 1, plus slot 2's pre-shift
-// by multiply-high (moves work from the integer-logic pipe to the FMA pipe).
+// pipe; 1 the high-half selector by multiply-high; 2 as 1, plus slot 2's
+// pre-shift by multiply-high; 3 both halves from one wide multiply-add
+// (moves work from the integer-logic pipe to the FMA pipe).
 #ifndef IQK_LOOKUP
 #define IQK_LOOKUP 0
 #endif
+
+// Group reduction of the tile kernel: 1 the last warp to finish its share of
+// a group sums the group's slots (two slot sets, so warps run one group
+// ahead, no CTA barrier); 0 two CTA barriers per group.
+#ifndef IQK_LAST_ARRIVER
+#define IQK_LAST_ARRIVER 1
+#endif
+constexpr int kSlotSets = IQK_LAST_ARRIVER ? 2 : 1;
 
 namespace iqk {
 
@@ -137,7 +146,8 @@ __device__ __forceinline__ void build_lut(uint2* lut, const Values& V) {
   }
 }
 
-// 16-byte activation fragment: from shared memory (BSM) or the read-only path.
+// 16-byte activation fragment: from shared memory (BSM) or from the
+// workspace rows the preceding kernel wrote (a plain load, after the wait).
 template <bool BSM>
 __device__ __forceinline__ uint4 ld_act(const uint16_t* p) {
   if constexpr (BSM) {
@@ -145,7 +155,7 @@ __device__ __forceinline__ uint4 ld_act(const uint16_t* p) {
     asm("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w) : "r"(smem_u32(p)));
     return r;
   } else {
-    return ld_nc_u4(p);
+    return ld_u4(p);
   }
 }
 
@@ -153,6 +163,9 @@ __device__ __forceinline__ Pair2 lookup(uint32_t q, int i, uint32_t t0, uint32_t
 #if IQK_LOOKUP == 0
   (void)k65536;
   return lookup_slot(q, i, t0, t1);
+#elif IQK_LOOKUP == 3
+  (void)k65536;
+  return lookup_slot_wide(q, i, t0, t1);
 #elif IQK_LOOKUP == 1
   return lookup_slot_mh(q, i, t0, t1, k65536);
 #else
@@ -310,7 +323,7 @@ __device__ __forceinline__ RouteView carve_route(uint8_t* p, int n) {
 __device__ __forceinline__ void build_route(const int32_t* __restrict__ ids, int n, int E, RouteView r,
                                             int chunk = 1 << 30, int ebase = 0) {
   for (int p = threadIdx.x; p < n; p += blockDim.x) {
-    const int e = ids[p] - ebase;  // an expert-parallel shard holds experts [ebase, ebase + E)
+    const int e = __ldcg(ids + p) - ebase;  // an expert-parallel shard holds experts [ebase, ebase + E)
     r.ids[p] = (e >= 0 && e < E) ? e : -1;
   }
   __syncthreads();
@@ -368,11 +381,13 @@ __global__ void __launch_bounds__(256) k_prep(const uint16_t* __restrict__ x, in
                                               uint16_t* __restrict__ xp, int32_t* __restrict__ zero,
                                               int nzero, const int32_t* __restrict__ ids, int npairs, int E,
                                               int32_t* __restrict__ status) {
-  griddep_launch();
   // Launched as a dependent of whatever precedes it (the previous call's last
   // kernel may still be writing this call's x or ids, or reading the
   // workspace written below): nothing is read or written before the wait.
+  // Only then may the call's other kernels launch, so they can read the
+  // call's inputs as soon as they start.
   griddep_wait();
+  griddep_launch();
   const int tid = blockIdx.x * blockDim.x + threadIdx.x;
   const int nth = gridDim.x * blockDim.x;
   for (int i = tid; i < nzero; i += nth) zero[i] = 0;
@@ -442,6 +457,8 @@ struct UnitArgs {
   int act_rows;  // BSM: activation rows copied into shared memory
   int tpg;       // tile kernel, SWITCH: tiles per group (items per group = splits * tpg)
   int ebase;     // routed modes: first expert id the weights hold (expert-parallel shard)
+  int expire;    // testing hook: warp 0 of every CTA also waits on a barrier nothing arrives on
+  uint64_t wait_ns;  // bound of every wait on a data barrier (global-timer ns)
   FastDiv div_s, div_tiles;
 };
 
@@ -536,8 +553,8 @@ __device__ __forceinline__ void stage_scales(uint8_t* slot, const WDev& w, int64
   __syncwarp();
 }
 
-// Timeout flag of the floor arm, which has no workspace; read with
-// cudaMemcpyFromSymbol when diagnosing.
+// Timeout flag of the floor arm, which has no workspace: cleared by each
+// floor call's first kernel, read back by iqk_floor_status.
 __device__ int32_t g_floor_status;
 
 template <int MODE, int F0, int F1, int NT, bool BSM>
@@ -559,7 +576,8 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, kDecodeMinBlocks(NT)) k_str
   uint8_t* ring_slots = smem + wid * warp_bytes + (size_t)kStages * stage_words * 4;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kDecodeWarps * warp_bytes);
   uint64_t* bar = bars + wid * kStages;
-  uint2* lut0 = reinterpret_cast<uint2*>(bars + kDecodeWarps * kStages);
+  uint64_t* never_bar = bars + kDecodeWarps * kStages;  // nothing arrives on it (expire hook)
+  uint2* lut0 = reinterpret_cast<uint2*>(never_bar + 2);
   uint2* lut1 = lut0 + 64;
   uint16_t* act_s = reinterpret_cast<uint16_t*>(lut1 + 64);  // BSM activation rows
   // BSM rows keep each lane's 64-element segment in 80 elements (160 bytes),
@@ -568,15 +586,17 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, kDecodeMinBlocks(NT)) k_str
   if (MODE == MODE_GEMV) build_lut<F0>(lut0, A.V);
   if (lane == 0) {
     for (int s = 0; s < kStages; s++) mbar_init(&bar[s], 1);
+    if (wid == 0) mbar_init(never_bar, 1);
     fence_mbar_init();
   }
   __syncthreads();
-  // Only the kernel parameters are read before the dependency wait: x, the
-  // expert list and the weights may be written by the preceding kernel, which
-  // lets its dependents launch early. Dependents of this kernel may launch at
-  // once because they wait the same way.
+  // This kernel starts only after the call's first kernel has seen the
+  // previous work on the stream complete (that kernel waits before it lets
+  // its dependents launch), so the call's inputs (x, the expert list) and the
+  // weight streams are read right away. The workspace and the outputs, which
+  // the first kernel writes, are touched only after the dependency wait.
+  // Dependents of this kernel may launch at once: they wait the same way.
   griddep_launch();
-  griddep_wait();
   const int D = MODE == MODE_FLOOR ? A.nexp : 1;  // matrices streamed
   const int rows = A.w0.rows;
   const int tiles = (rows + kTile - 1) / kTile;
@@ -590,10 +610,12 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, kDecodeMinBlocks(NT)) k_str
     u = (int)A.div_tiles.div((uint32_t)r);
     tile = r - u * tiles;
   };
-  auto expert_of = [&](int u) -> int { return MODE == MODE_FLOOR ? A.elist[u] : A.expert; };
+  auto expert_of = [&](int u) -> int { return MODE == MODE_FLOOR ? __ldcg(A.elist + u) : A.expert; };
+  int issued = 0;  // items this warp has requested
   auto issue = [&](int it) {
     const int id = gw + it * W;
     if (id >= nitems) return;
+    issued = it + 1;
     const int st = it % kStages;
     int u, tile, s;
     item_of(id, u, tile, s);
@@ -615,7 +637,7 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, kDecodeMinBlocks(NT)) k_str
       const int r = gi / gpr, c0 = (gi - r * gpr) * 16;
       uint32_t o[8];
       const uint4* src = reinterpret_cast<const uint4*>(A.xraw + (size_t)gi * 16);
-      const uint4 a = ld_nc_u4(src), b = ld_nc_u4(src + 1);
+      const uint4 a = ld_cg_u4(src), b = ld_cg_u4(src + 1);
       const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
 #pragma unroll
       for (int i2 = 0; i2 < 4; i2++) {
@@ -633,6 +655,13 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, kDecodeMinBlocks(NT)) k_str
   const uint16_t* act_base = BSM ? act_s : A.act;
   constexpr int SEG = BSM ? 80 : 64;    // elements between the segments of lanes t and t + 1
   constexpr int BLKE = BSM ? 320 : 256;  // elements between consecutive 256-weight blocks
+  griddep_wait();  // from here on: the workspace (transposed x, counters, partial sums) and the outputs
+  int32_t* status = A.status ? A.status : &g_floor_status;
+  if (A.expire && wid == 0 && !mbar_wait_ns(never_bar, 0, A.wait_ns)) {  // testing hook: this wait runs out
+    if (lane == 0) atomicOr(status, 2);
+    for (int k = 0; k < issued; k++) (void)mbar_wait_ns(&bar[k % kStages], (uint32_t)((k / kStages) & 1), kDrainWaitNs);
+    return;
+  }
 
   for (int it = 0;; it++) {
     const int id = gw + it * W;
@@ -650,11 +679,11 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, kDecodeMinBlocks(NT)) k_str
     const bool fmt0 = true;
     const bool kfmt = F0 == FMT_K;
     const int st = it % kStages;
-    if (!mbar_wait_bounded(&bar[st], (uint32_t)((it / kStages) & 1))) {
-      if (lane == 0) atomicOr(A.status ? A.status : &g_floor_status, 2);
+    if (!mbar_wait_ns(&bar[st], (uint32_t)((it / kStages) & 1), A.wait_ns)) {
+      if (lane == 0) atomicOr(status, 2);
       // let this warp's copies still in flight land before the CTA exits
-      for (int k = 1; k < kStages; k++)
-        (void)mbar_wait_bounded(&bar[(it + k) % kStages], (uint32_t)(((it + k) / kStages) & 1));
+      for (int k = it; k < issued; k++)
+        (void)mbar_wait_ns(&bar[k % kStages], (uint32_t)((k / kStages) & 1), kDrainWaitNs);
       return;
     }
     const uint32_t* sq = ring_qs + (size_t)st * stage_words;
@@ -806,39 +835,46 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, kDecodeMinBlocks(NT)) k_til
   uint8_t* ring_slots = smem + wid * warp_bytes + (size_t)kStages * stage_words * 4;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kDecodeWarps * warp_bytes);
   uint64_t* bar = bars + wid * kStages;
-  uint2* lut0 = reinterpret_cast<uint2*>(bars + kDecodeWarps * kStages);
+  uint64_t* never_bar = bars + kDecodeWarps * kStages;  // nothing arrives on it (expire hook)
+  uint2* lut0 = reinterpret_cast<uint2*>(never_bar + 2);
   uint2* lut1 = lut0 + 64;
   const int KP = BSM ? K / 64 * 80 : K;  // activation row stride (elements), see k_stream
   uint16_t* act_s = reinterpret_cast<uint16_t*>(lut1 + 64);
-  float* red = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(act_s) + (BSM ? (size_t)A.act_rows * KP * 2 : 0));
+  // group-reduction words: arrivals and completed reductions per slot set
+  int* gsync = reinterpret_cast<int*>(reinterpret_cast<uint8_t*>(act_s) + (BSM ? (size_t)A.act_rows * KP * 2 : 0));
+  float* red = reinterpret_cast<float*>(gsync + 4);
   // floats per warp slot: (mat, column, row) gate/up; (column, row) switch; (token, row) down
   const int slot_f = MODE == MODE_GATEUP ? 2 * NC * kTile : MODE == MODE_SWITCH ? NC * kTile : A.T * kTile;
-  uint8_t* route_p = reinterpret_cast<uint8_t*>(red + (size_t)kDecodeWarps * slot_f);
-  // Only the kernel parameters are read before the dependency wait. Every
-  // input of the call (x, ids, p, h, the expert list) may be written by the
-  // preceding kernel, which lets its dependents launch early, so it is read
-  // after griddepcontrol.wait; dependents of this kernel may launch at once
-  // because they wait the same way.
+  uint8_t* route_p = reinterpret_cast<uint8_t*>(red + (size_t)kSlotSets * kDecodeWarps * slot_f);
+  // This kernel starts only after the call's first kernel has seen the
+  // previous work on the stream complete (that kernel waits before it lets
+  // its dependents launch), so the call's inputs (x, ids, p) and the weight
+  // streams are read right away: the routing is built and the first weight
+  // tiles are requested while the preceding kernel of this call finishes.
+  // What a preceding kernel of the call writes (the status word, transposed
+  // x, h) and the outputs are touched only after the dependency wait.
+  // Dependents of this kernel may launch at once: they wait the same way.
   build_lut<F0>(lut0, A.V);
   if (MODE == MODE_GATEUP) build_lut<F1>(lut1, A.V);
   if (lane == 0) {
     for (int s = 0; s < kStages; s++) mbar_init(&bar[s], 1);
+    if (wid == 0) mbar_init(never_bar, 1);
     fence_mbar_init();
   }
+  if (threadIdx.x < 4) gsync[threadIdx.x] = 0;  // visible to all after build_route's barriers
   griddep_launch();
-  griddep_wait();
   // gate/up and switch: request the first activation groups ahead of the weight stream
   uint4 pre0 = make_uint4(0u, 0u, 0u, 0u), pre1 = pre0, pre2 = pre0, pre3 = pre0;
   const int act_groups = BSM ? A.act_rows * (K / 16) : 0;
   if (BSM && MODE != MODE_DOWN) {
     const int g0 = threadIdx.x, g1 = threadIdx.x + blockDim.x;
     if (g0 < act_groups) {
-      pre0 = ld_nc_u4(A.xraw + (size_t)g0 * 16);
-      pre1 = ld_nc_u4(A.xraw + (size_t)g0 * 16 + 8);
+      pre0 = ld_cg_u4(A.xraw + (size_t)g0 * 16);
+      pre1 = ld_cg_u4(A.xraw + (size_t)g0 * 16 + 8);
     }
     if (g1 < act_groups) {
-      pre2 = ld_nc_u4(A.xraw + (size_t)g1 * 16);
-      pre3 = ld_nc_u4(A.xraw + (size_t)g1 * 16 + 8);
+      pre2 = ld_cg_u4(A.xraw + (size_t)g1 * 16);
+      pre3 = ld_cg_u4(A.xraw + (size_t)g1 * 16 + 8);
     }
   }
   const RouteView rt = carve_route(route_p, npairs);
@@ -895,6 +931,7 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, kDecodeMinBlocks(NT)) k_til
     issued = q + 1;
   };
   for (int q = 0; q < kStages; q++) issue(q);
+  griddep_wait();  // from here on: what the call's preceding kernels wrote, and the outputs
   if constexpr (BSM) {  // activation rows, slot-transposed and padded, once per CTA
     const int gpr = K / 16;
     for (int k = 0;; k++) {
@@ -904,12 +941,12 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, kDecodeMinBlocks(NT)) k_til
       uint32_t o[8];
       if (MODE == MODE_DOWN) {
         const uint4* src = reinterpret_cast<const uint4*>(A.act + (size_t)gi * 16);
-        const uint4 a = ld_nc_u4(src), b = ld_nc_u4(src + 1);
+        const uint4 a = ld_u4(src), b = ld_u4(src + 1);
         o[0] = a.x; o[1] = a.y; o[2] = a.z; o[3] = a.w; o[4] = b.x; o[5] = b.y; o[6] = b.z; o[7] = b.w;
       } else {
         const uint4* src = reinterpret_cast<const uint4*>(A.xraw + (size_t)gi * 16);
-        const uint4 a = k == 0 ? pre0 : k == 1 ? pre2 : ld_nc_u4(src);
-        const uint4 b = k == 0 ? pre1 : k == 1 ? pre3 : ld_nc_u4(src + 1);
+        const uint4 a = k == 0 ? pre0 : k == 1 ? pre2 : ld_cg_u4(src);
+        const uint4 b = k == 0 ? pre1 : k == 1 ? pre3 : ld_cg_u4(src + 1);
         const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
 #pragma unroll
         for (int i2 = 0; i2 < 4; i2++) {
@@ -942,11 +979,36 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, kDecodeMinBlocks(NT)) k_til
   const uint16_t* act_base = BSM ? act_s : A.act;
   constexpr int SEG = BSM ? 80 : 64;
   constexpr int BLKE = BSM ? 320 : 256;
-  float* my = red + (size_t)wid * slot_f;
   bool failed = false;
+  if (A.expire && wid == 0 && !mbar_wait_ns(never_bar, 0, A.wait_ns)) {  // testing hook: this wait runs out
+    failed = true;  // keep taking part in the group reductions; stop loading
+    if (lane == 0) atomicOr(A.status, 2);
+  }
+  // warps with items in a group: 0 .. P-1 (cnt_w > 0 exactly for them)
+  const int P = n_it < kDecodeWarps ? n_it : kDecodeWarps;
   int consumed = 0;
   int q = 0;
   for (int r = 0; r < rounds; r++) {
+    const int set = IQK_LAST_ARRIVER ? (r & 1) : 0;
+    float* my = red + ((size_t)set * kDecodeWarps + wid) * slot_f;
+    if (IQK_LAST_ARRIVER) {
+      if (cnt_w == 0) continue;  // no item of this warp in any group
+      // the set was last used by group r - 2: wait until it has been reduced
+      if (r >= 2) {
+        volatile int* done = gsync + 2 + set;
+        if (*done < (r >> 1)) {
+          const uint64_t t0 = globaltimer_ns();
+          while (*done < (r >> 1)) {
+            if (globaltimer_ns() - t0 >= A.wait_ns) {
+              if (!failed && lane == 0) atomicOr(A.status, 2);
+              failed = true;
+              break;
+            }
+          }
+        }
+        __threadfence_block();
+      }
+    }
     for (int i = lane; i < slot_f; i += 32) my[i] = 0.f;
     __syncwarp();
     for (int k = 0; k < cnt_w; k++, q++) {
@@ -972,8 +1034,8 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, kDecodeMinBlocks(NT)) k_til
 #pragma unroll
         for (int qq = 0; qq < 4; qq++) acc[n][qq] = 0.f;
       const int st = q % kStages;
-      if (!failed && !mbar_wait_bounded(&bar[st], (uint32_t)((q / kStages) & 1))) {
-        failed = true;  // keep taking part in the CTA barriers; stop loading
+      if (!failed && !mbar_wait_ns(&bar[st], (uint32_t)((q / kStages) & 1), A.wait_ns)) {
+        failed = true;  // keep taking part in the group reductions; stop loading
         if (lane == 0) atomicOr(A.status, 2);
       }
       if (!failed) {
@@ -1008,28 +1070,44 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, kDecodeMinBlocks(NT)) k_til
             for (int qq = 0; qq < 4; qq++) {
               if (8 * n + 2 * t + (qq & 1) != c) continue;
               const int pair = rt.sorted[p0 + c];
-              my[(pair / A.topk) * kTile + g + 8 * (qq >> 1)] += __ldg(A.p + pair) * acc[n][qq];
+              my[(pair / A.topk) * kTile + g + 8 * (qq >> 1)] += __ldcg(A.p + pair) * acc[n][qq];
             }
           __syncwarp();
         }
       }
       __syncwarp();
     }
-    __syncthreads();  // every warp's slot of this group is complete
+    // The group's reduction, by all threads after a CTA barrier, or by the
+    // last warp to add its slot (the slots summed in warp order either way).
+    int rt0 = threadIdx.x, rstep = blockDim.x;
+    if (IQK_LAST_ARRIVER) {
+      int last = 0;
+      if (lane == 0) {
+        __threadfence_block();
+        last = atomicAdd(gsync + set, 1) == P - 1;
+      }
+      if (!__shfl_sync(0xffffffffu, last, 0)) continue;
+      __threadfence_block();
+      rt0 = lane;
+      rstep = 32;
+    } else {
+      __syncthreads();  // every warp's slot of this group is complete
+    }
+    const float* rb = red + (size_t)set * kDecodeWarps * slot_f;
     const int tg = (int)blockIdx.x + r * (int)gridDim.x;
     if (MODE == MODE_GATEUP) {
       const int u = (int)A.div_tiles.div((uint32_t)tg);
       const int tile = tg - u * tiles;
       const int p0 = rt.ustart[u];
       const int ncols = min(rt.ustart[u + 1] - p0, NC);  // runs never exceed NC; the bound guards the slot reads
-      for (int o = threadIdx.x; o < ncols * kTile; o += blockDim.x) {
+      for (int o = rt0; o < ncols * kTile; o += rstep) {
         const int col = o / kTile, row = o - col * kTile;
         const int f = tile * kTile + row;
         if (f >= rows) continue;
         float gv = 0.f, uv = 0.f;
-        for (int w = 0; w < kDecodeWarps; w++) {
-          gv += red[(size_t)w * slot_f + col * kTile + row];
-          uv += red[(size_t)w * slot_f + (NC + col) * kTile + row];
+        for (int w = 0; w < P; w++) {
+          gv += rb[(size_t)w * slot_f + col * kTile + row];
+          uv += rb[(size_t)w * slot_f + (NC + col) * kTile + row];
         }
         const float h = gv / (1.0f + __expf(-gv)) * uv;
         A.out16[(size_t)rt.sorted[p0 + col] * rows + perm16(f)] = f32_to_bf16_bits(h);
@@ -1042,34 +1120,58 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, kDecodeMinBlocks(NT)) k_til
       const int p0 = rt.ustart[u];
       const int ncols = min(rt.ustart[u + 1] - p0, NC);
       const int per = ncols * kTile;
-      for (int o = threadIdx.x; o < tpg * per; o += blockDim.x) {
+      for (int o = rt0; o < tpg * per; o += rstep) {
         const int sub = o / per, rem = o - sub * per;
         const int col = rem / kTile, row = rem - col * kTile;
         const int f = (t0 + sub) * kTile + row;
         if (t0 + sub >= tiles || f >= rows) continue;
-        const int w0 = tpg > 1 ? sub * S : 0, w1 = tpg > 1 ? w0 + S : kDecodeWarps;
+        const int w0 = tpg > 1 ? sub * S : 0, w1 = tpg > 1 ? w0 + S : P;
         float v = 0.f;
-        for (int w = w0; w < w1; w++) v += red[(size_t)w * slot_f + col * kTile + row];
+        for (int w = w0; w < w1; w++) v += rb[(size_t)w * slot_f + col * kTile + row];
         A.yf[(size_t)rt.sorted[p0 + col] * rows + f] = v;
       }
     } else {
-      for (int o = threadIdx.x; o < A.T * kTile; o += blockDim.x) {
+      for (int o = rt0; o < A.T * kTile; o += rstep) {
         const int tok = o / kTile, row = o - tok * kTile;
         const int f = tg * kTile + row;
         if (f >= rows) continue;
         float y = 0.f;
-        for (int w = 0; w < kDecodeWarps; w++) y += red[(size_t)w * slot_f + tok * kTile + row];
+        for (int w = 0; w < P; w++) y += rb[(size_t)w * slot_f + tok * kTile + row];
         if (A.yf) A.yf[(size_t)tok * rows + f] = y;  // an expert-parallel partial, summed across ranks
         else A.out16[(size_t)tok * rows + f] = f32_to_bf16_bits(y);
       }
     }
-    __syncthreads();  // slots free for the next group
+    if (IQK_LAST_ARRIVER) {
+      __syncwarp();  // every lane's reads of the set are done
+      if (lane == 0) {
+        gsync[set] = 0;
+        __threadfence_block();
+        *(volatile int*)(gsync + 2 + set) = (r >> 1) + 1;
+      }
+    } else {
+      __syncthreads();  // slots free for the next group
+    }
   }
   // let copies still in flight land before the CTA exits (only after a timeout)
-  for (int qd = consumed; qd < issued; qd++) (void)mbar_wait_bounded(&bar[qd % kStages], (uint32_t)((qd / kStages) & 1));
+  for (int qd = consumed; qd < issued; qd++) (void)mbar_wait_ns(&bar[qd % kStages], (uint32_t)((qd / kStages) & 1), kDrainWaitNs);
 }
 
 // ================================================================== host
+
+// Bound of the data-barrier waits and the expire hook, copied into every
+// decode-side launch (iqk_set_wait_limit_ns).
+static std::atomic<uint64_t> g_wait_ns{kDefaultWaitNs};
+static std::atomic<int> g_expire{0};
+
+void set_wait_limit(uint64_t ns, int expire) {
+  g_wait_ns.store(ns ? ns : kDefaultWaitNs);
+  g_expire.store(expire ? 1 : 0);
+}
+
+int read_floor_status(cudaStream_t st, int32_t* out) {
+  if (cudaStreamSynchronize(st) != cudaSuccess) return -4;
+  return cudaMemcpyFromSymbol(out, g_floor_status, sizeof(int32_t)) == cudaSuccess ? 0 : -4;
+}
 
 EncodeTiledFn encode_tiled_fn() {
   static EncodeTiledFn fn = nullptr;
@@ -1103,7 +1205,7 @@ template <int F0, int F1>
 static size_t stream_smem(int cols, int act_rows) {
   const int bpi = item_blocks(cols);
   const size_t warp = (size_t)kStages * ((size_t)kTile * bpi * 16 * 4 + slot_bytes2<F0, F1>(bpi));
-  return kDecodeWarps * warp + (size_t)kDecodeWarps * kStages * 8 + 2 * 64 * 8 +
+  return kDecodeWarps * warp + (size_t)kDecodeWarps * kStages * 8 + 16 + 2 * 64 * 8 +
          (size_t)act_rows * (cols / 64 * 80) * 2;
 }
 
@@ -1111,9 +1213,9 @@ template <int MODE, int F0, int F1, int NT>
 static size_t tiles_smem(int cols, int T, int npairs, int act_rows) {
   const int bpi = item_blocks(cols);
   const size_t warp = (size_t)kStages * ((size_t)kTile * bpi * 16 * 4 + slot_bytes2<F0, F1>(bpi));
-  const size_t red =
-      (size_t)kDecodeWarps * (MODE == MODE_GATEUP ? 2 * 8 * NT * kTile : MODE == MODE_SWITCH ? 8 * NT * kTile : T * kTile) * 4;
-  return kDecodeWarps * warp + (size_t)kDecodeWarps * kStages * 8 + 2 * 64 * 8 + (size_t)act_rows * (cols / 64 * 80) * 2 +
+  const size_t red = 16 + (size_t)kSlotSets * kDecodeWarps *
+                              (MODE == MODE_GATEUP ? 2 * 8 * NT * kTile : MODE == MODE_SWITCH ? 8 * NT * kTile : T * kTile) * 4;
+  return kDecodeWarps * warp + (size_t)kDecodeWarps * kStages * 8 + 16 + 2 * 64 * 8 + (size_t)act_rows * (cols / 64 * 80) * 2 +
          red + route_smem_bytes(npairs);
 }
 
@@ -1201,11 +1303,13 @@ static int launch_prep(int blocks, cudaStream_t st, const uint16_t* x, int T, in
   return cudaLaunchKernelEx(&cfg, k_prep, x, T, cols, xp, zero, nzero, ids, npairs, E, status) == cudaSuccess ? 0 : -4;
 }
 
-// Zeroes n words after the preceding kernel completes (programmatic
-// dependent, like the prep kernel).
+// Zeroes n words and the floor's timeout flag after the preceding kernel
+// completes (programmatic dependent, like the prep kernel; its dependents
+// launch only after that wait).
 __global__ void __launch_bounds__(256) k_zero(uint32_t* __restrict__ out, size_t n) {
-  griddep_launch();
   griddep_wait();
+  griddep_launch();
+  if (blockIdx.x == 0 && threadIdx.x == 0) g_floor_status = 0;
   for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x) out[i] = 0u;
 }
 
@@ -1246,6 +1350,8 @@ static int launch_stream(const CUtensorMap& m0, const CUtensorMap& m1, const Uni
   auto kern = k_stream<MODE, F0, F1, NT, BSM>;
   // the item-index dividers follow this launch's own geometry
   UnitArgs args = a;
+  args.wait_ns = g_wait_ns.load();
+  args.expire = g_expire.load();
   args.div_s = FastDiv::of((uint32_t)a.splits);
   args.div_tiles = FastDiv::of((uint32_t)((a.w0.rows + kTile - 1) / kTile));
   const size_t smem = stream_smem<F0, F1>(a.w0.cols, BSM ? a.act_rows : 0);
@@ -1268,6 +1374,8 @@ static int launch_tiles(const CUtensorMap& m0, const CUtensorMap& m1, const Unit
                         int num_sms, bool pdl) {
   auto kern = k_tiles<MODE, F0, F1, NT, BSM>;
   UnitArgs args = a;
+  args.wait_ns = g_wait_ns.load();
+  args.expire = g_expire.load();
   args.div_s = FastDiv::of((uint32_t)a.splits);
   const int tiles = (a.w0.rows + kTile - 1) / kTile;
   args.div_tiles = FastDiv::of((uint32_t)(MODE == MODE_SWITCH ? (tiles + a.tpg - 1) / a.tpg : tiles));

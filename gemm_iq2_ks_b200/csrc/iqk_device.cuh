@@ -105,6 +105,29 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
   return false;
 }
 
+__device__ __forceinline__ uint64_t globaltimer_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+// Bounded wait on an mbarrier phase, the bound in nanoseconds of the GPU's
+// global timer. Returns false once `limit_ns` has passed without the phase
+// completing.
+__device__ __forceinline__ bool mbar_wait_ns(uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (;;) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (globaltimer_ns() - t0 >= limit_ns) return false;
+  }
+}
+
+// Bound of the waits that let a warp's copies still in flight land after one
+// of its waits expired (the copies complete on their own; this only guards
+// against a wedged copy engine).
+constexpr uint64_t kDrainWaitNs = 2000000000ull;
+
 // 2-D tiled TMA load (no multicast) into shared memory, completion on `bar`.
 __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int32_t x, int32_t y,
                                             uint64_t* bar) {
@@ -157,6 +180,26 @@ __device__ __forceinline__ Pair2 lookup_slot(uint32_t q, int i, uint32_t t0, uin
   return r;
 }
 
+// Same, with both selector halves from one 32 x 32 -> 64-bit multiply-add:
+// with V = u * 0x22, u * 0x00220022 = V + V * 2^16, whose low word holds V's
+// low half in bits 0..15 and whose high word is V's high half exactly (the
+// middle sum stays below 2^32 because every byte of V is at most 0x66). The
+// 64-bit addend puts 0x1010 on both halves. This replaces the integer-logic
+// pipe's 16-bit shift with work on the FMA pipe.
+__device__ __forceinline__ Pair2 lookup_slot_wide(uint32_t q, int i, uint32_t t0, uint32_t t1) {
+  const uint32_t u = (q >> (2 * i)) & 0x03030303u;
+  uint32_t lo, hi;
+  asm("{\n\t.reg .u64 w;\n\t"
+      "mad.wide.u32 w, %2, 0x00220022, 0x0000101000001010;\n\t"
+      "mov.b64 {%0, %1}, w;\n\t}"
+      : "=r"(lo), "=r"(hi)
+      : "r"(u));
+  Pair2 r;
+  r.lo = prmt(t0, t1, lo);
+  r.hi = prmt(t0, t1, hi);
+  return r;
+}
+
 // Same, with the high selector's 16-bit shift done as a multiply-high by
 // `k65536` (= 65536, held in a register the compiler cannot fold), which runs
 // on the FMA pipe instead of the integer-logic pipe the permutes use.
@@ -190,6 +233,22 @@ __device__ __forceinline__ Pair2 lookup_slot_mh2(uint32_t q, uint32_t t0, uint32
 __device__ __forceinline__ uint32_t opaque_u32(uint32_t v) {
   uint32_t r;
   asm volatile("mov.u32 %0, %1;" : "=r"(r) : "r"(v));
+  return r;
+}
+
+// 16 bytes through L2 only (no L1 allocation): call inputs read before a
+// kernel's dependency wait.
+__device__ __forceinline__ uint4 ld_cg_u4(const void* p) {
+  uint4 r;
+  asm volatile("ld.global.cg.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w) : "l"(p));
+  return r;
+}
+
+// 16 bytes by a plain global load: data a preceding kernel of the same call
+// wrote, read after the dependency wait (the wait orders those writes first).
+__device__ __forceinline__ uint4 ld_u4(const void* p) {
+  uint4 r;
+  asm volatile("ld.global.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w) : "l"(p));
   return r;
 }
 

@@ -103,6 +103,14 @@ int launch_switch_gemm(const WDev& w, int fmt, const Values& V, const uint16_t* 
 
 int launch_floor(const WDev& w, int fmt, const int32_t* experts, int n, uint32_t* out, cudaStream_t st,
                  int num_sms);
+// The floor's timeout flag (cleared by every floor call), after syncing `st`.
+int read_floor_status(cudaStream_t st, int32_t* out);
+
+// Bound of the decode-side kernels' data-barrier waits in ns (0: the
+// default), and the expire hook (warp 0 of every CTA also waits on a barrier
+// nothing arrives on), applied to launches made from now on.
+constexpr uint64_t kDefaultWaitNs = 2000000000ull;
+void set_wait_limit(uint64_t ns, int expire);
 
 // ----------------------------------------------------------------- prefill
 struct PrefillWs {
@@ -112,15 +120,22 @@ struct PrefillWs {
 PrefillWs prefill_ws(int T, int topk, int experts, int hidden, int inter);
 
 // Grouping step. `cc` is scratch of route_scratch_ints(T*topk, experts) ints.
+// ebase / silent: an expert-parallel shard groups only ids in [ebase, ebase +
+// experts), as ids - ebase, and skips the others without flagging them.
 int launch_route(const int32_t* ids, int T, int topk, int experts, int32_t* counts, int32_t* offsets,
-                 int32_t* perm, int32_t* status, int32_t* cc, cudaStream_t st);
+                 int32_t* perm, int32_t* status, int32_t* cc, cudaStream_t st, int ebase = 0, bool silent = false);
 inline size_t route_scratch_ints(int npairs, int experts) {
   return (size_t)((npairs + 1023) / 1024) * experts;
 }
 
+// yf non-null: an expert-parallel shard holding experts [ebase, ebase + E)
+// writes its float32 partial to yf (y unused) and skips other ids silently.
 int launch_moe_prefill(const WDev& g, int fg, const WDev& u, int fu, const WDev& d, int fd,
                        const Values& V, const uint16_t* x, int T, const int32_t* ids, const float* p,
-                       int topk, uint16_t* y, char* ws, cudaStream_t st, int num_sms);
+                       int topk, uint16_t* y, float* yf, int ebase, char* ws, cudaStream_t st, int num_sms);
+// y[t] = bf16_rn(sum over slots j in order of p[t][j] * rows[t * topk + j]).
+int launch_combine(const float* rows, const float* p, int T, int topk, int H, uint16_t* y, cudaStream_t st,
+                   int num_sms);
 
 // Driver entry point for cuTensorMapEncodeTiled (resolved once).
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,

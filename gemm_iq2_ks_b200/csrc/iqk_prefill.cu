@@ -451,16 +451,17 @@ __global__ void __launch_bounds__(256) k_pf_gather(const uint16_t* __restrict__ 
   }
 }
 
-// y[t][o] = bf16(sum over slots j in order of outp[inv[t*topk + j]][o]).
+// y[t][o] = bf16(sum over slots j in order of p[t][j] * outp[inv[t*topk + j]][o])
+// (inv == nullptr: row t*topk + j); float32 into yf instead when yf is set.
 __global__ void __launch_bounds__(256) k_pf_combine(const float* __restrict__ outp, const int32_t* __restrict__ inv,
                                                     const float* __restrict__ p, int T, int topk, int H,
-                                                    uint16_t* __restrict__ y) {
+                                                    uint16_t* __restrict__ y, float* __restrict__ yf) {
   const int64_t n = (int64_t)T * (H / 4);
   for (int64_t g = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; g < n; g += (int64_t)gridDim.x * blockDim.x) {
     const int t = (int)(g / (H / 4)), o4 = (int)(g % (H / 4));
     float4 s = make_float4(0.f, 0.f, 0.f, 0.f);
     for (int j = 0; j < topk; j++) {
-      const int pos = inv[t * topk + j];
+      const int pos = inv ? inv[t * topk + j] : t * topk + j;
       if (pos < 0) continue;
       const float pw = __ldg(p + t * topk + j);
       const float4 v = __ldg(reinterpret_cast<const float4*>(outp + (size_t)pos * H) + o4);
@@ -469,11 +470,23 @@ __global__ void __launch_bounds__(256) k_pf_combine(const float* __restrict__ ou
       s.z += pw * v.z;
       s.w += pw * v.w;
     }
-    uint2 out;
-    out.x = pack_bf16x2(s.x, s.y);
-    out.y = pack_bf16x2(s.z, s.w);
-    reinterpret_cast<uint2*>(y + (size_t)t * H)[o4] = out;
+    if (yf) {
+      reinterpret_cast<float4*>(yf + (size_t)t * H)[o4] = s;
+    } else {
+      uint2 out;
+      out.x = pack_bf16x2(s.x, s.y);
+      out.y = pack_bf16x2(s.z, s.w);
+      reinterpret_cast<uint2*>(y + (size_t)t * H)[o4] = out;
+    }
   }
+}
+
+int launch_combine(const float* rows, const float* p, int T, int topk, int H, uint16_t* y, cudaStream_t st,
+                   int num_sms) {
+  const int64_t n = (int64_t)T * (H / 4);
+  const int blocks = (int)std::min<int64_t>((n + 255) / 256, (int64_t)num_sms * 16);
+  k_pf_combine<<<std::max(blocks, 1), 256, 0, st>>>(rows, nullptr, p, T, topk, H, y, nullptr);
+  return cudaGetLastError() == cudaSuccess ? 0 : -4;
 }
 
 PrefillWs prefill_ws(int T, int topk, int experts, int hidden, int inter) {
@@ -555,8 +568,8 @@ static int dispatch_gemm(int f0, int f1, const CUtensorMap& m0, const CUtensorMa
 }
 
 int launch_moe_prefill(const WDev& g, int fg, const WDev& u, int fu, const WDev& d, int fd, const Values& V,
-                       const uint16_t* x, int T, const int32_t* ids, const float* p, int topk, uint16_t* y, char* ws,
-                       cudaStream_t st, int num_sms) {
+                       const uint16_t* x, int T, const int32_t* ids, const float* p, int topk, uint16_t* y, float* yf,
+                       int ebase, char* ws, cudaStream_t st, int num_sms) {
   const int H = g.cols, F = g.rows, E = g.experts;
   const PrefillWs L = prefill_ws(T, topk, E, H, F);
   const int P = T * topk;
@@ -571,7 +584,7 @@ int launch_moe_prefill(const WDev& g, int fg, const WDev& u, int fu, const WDev&
   float* outp = reinterpret_cast<float*>(ws + L.outp);
 
   if (cudaMemsetAsync(inv, 0xFF, (size_t)P * 4, st) != cudaSuccess) return -4;
-  int rc = launch_route(ids, T, topk, E, counts, offsets, perm, status, cc, st);
+  int rc = launch_route(ids, T, topk, E, counts, offsets, perm, status, cc, st, ebase, yf != nullptr);
   if (rc) return rc;
   {
     const int64_t n = (int64_t)P * (H / 16);
@@ -607,7 +620,7 @@ int launch_moe_prefill(const WDev& g, int fg, const WDev& u, int fu, const WDev&
   {
     const int64_t n = (int64_t)T * (H / 4);
     const int blocks = (int)std::min<int64_t>((n + 255) / 256, (int64_t)num_sms * 16);
-    k_pf_combine<<<std::max(blocks, 1), 256, 0, st>>>(outp, inv, p, T, topk, H, y);
+    k_pf_combine<<<std::max(blocks, 1), 256, 0, st>>>(outp, inv, p, T, topk, H, y, yf);
   }
   return cudaGetLastError() == cudaSuccess ? 0 : -4;
 }

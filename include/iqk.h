@@ -301,6 +301,34 @@ int iqk_moe_decode_shard(const iqk_weights* gate, const iqk_weights* up, const i
                          float* y_partial, void* workspace, size_t ws_bytes, void* stream);
 
 /*
+ * iqk_moe_prefill_shard -- one rank's part of an expert-parallel prefill, the
+ * prefill counterpart of iqk_moe_decode_shard: the rank holds experts
+ * [expert_base, expert_base + E) in gate/up/down; ids are global; pairs
+ * outside the window are skipped silently. Output
+ *   y_partial: device float32 [T][hidden], 16-byte aligned, written completely:
+ *     y_partial[t] = sum over slots j in order with ids[t][j] in the window of
+ *                    p[t][j] * down_e( bf16_rn( silu(gate_e x_t) * up_e x_t ) )
+ * With topk = 1 and p = 1 every row is one pair's float32 down output, the
+ * form an all-to-all dispatch / combine ships back to the pair's token
+ * (iqk_moe_combine). Workspace and limits as iqk_moe_prefill.
+ */
+int iqk_moe_prefill_shard(const iqk_weights* gate, const iqk_weights* up, const iqk_weights* down,
+                          const float* values /* host [8] */, const uint16_t* x, int32_t T,
+                          const int32_t* ids, const float* p, int32_t topk, int32_t expert_base,
+                          float* y_partial, void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * iqk_moe_combine -- the routed block's weighted combine on its own:
+ *   y[t] = bf16_rn( sum over slots j in order of p[t][j] * rows[t*topk + j] )
+ * rows: device float32 [T*topk][hidden] (one pair's down output per row, in
+ * pair order), 16-byte aligned; p: device float32 [T][topk]; y: device bf16
+ * [T][hidden]; hidden a multiple of 4. The same arithmetic, in the same
+ * order, as the combine of iqk_moe_prefill.
+ */
+int iqk_moe_combine(const float* rows, const float* p, int32_t T, int32_t topk, int32_t hidden, uint16_t* y,
+                    void* stream);
+
+/*
  * iqk_f32_to_bf16 -- out[i] = bf16_rn(in[i]) (nearest even) for i < n;
  * device pointers. The last step of an expert-parallel decode.
  */
@@ -343,6 +371,29 @@ int iqk_moe_route(const int32_t* ids, int32_t T, int32_t topk, int32_t experts, 
  */
 int iqk_floor(const iqk_weights* w, const int32_t* expert_list, int32_t n_experts, uint32_t* out,
               void* stream);
+
+/*
+ * iqk_floor_status -- synchronises `stream`, then reports whether a bounded
+ * wait of the last iqk_floor call expired: IQK_OK or IQK_ETIMEOUT (that
+ * call's checksums are then incomplete). The flag is process-wide per device
+ * and cleared by every iqk_floor call; read it before the next one.
+ */
+int iqk_floor_status(void* stream);
+
+/*
+ * iqk_set_wait_limit_ns -- the bound of the device-side waits of the decode,
+ * GEMV, switch-linear (decode mode) and floor kernels launched from now on,
+ * in nanoseconds of the GPU's global timer (0 restores the default, 2 s).
+ * A wait that runs out sets the call's status to IQK_ETIMEOUT
+ * (iqk_moe_status, iqk_floor_status); the kernel then lets its copies in
+ * flight land (bounded separately, 2 s) and finishes without further loads,
+ * and the call's outputs are incomplete.
+ * expire != 0 is a testing hook: warp 0 of every CTA of those kernels then
+ * also waits once on a barrier nothing arrives on, so the bound runs out on
+ * purpose and the timeout path can be exercised; pass 0 for normal work.
+ * Process-wide; not synchronised with launches in flight on other threads.
+ */
+int iqk_set_wait_limit_ns(uint64_t limit_ns, int32_t expire);
 
 #ifdef __cplusplus
 }

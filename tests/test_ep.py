@@ -92,3 +92,78 @@ def _rank(rank, world, port):
 
 def test_two_gloo_ranks_all_reduce_their_parts_to_the_block():
     torch.multiprocessing.spawn(_rank, args=(2, _free_port()), nprocs=2, join=True)
+
+
+def _prefill_rank(rank, world, port, E):
+    """One gloo rank of the expert-parallel prefill: its own tokens, the
+    dispatch / combine of the module, the expert step computed by the oracle
+    (one pair per row), the result checked against the oracle's block."""
+    import torch.distributed as dist
+    sys.path.insert(0, ROOT)
+    from tests.util import check_y
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        rng = S.rng_for(90)
+        H, F, k = 256, 256, 4
+        gate = S.random_streams(rng, "iq2_ks", E, F, H)
+        up = S.random_streams(rng, "iq2_k", E, F, H)
+        down = S.random_streams(rng, "iq2_ks", E, H, F)
+        vals = S.value_table("f16", 3)
+        r2 = S.rng_for(91 + rank)
+        T = 5 + 4 * rank  # ranks hold different token counts
+        x = S.random_bf16(r2, (T, H))
+        ids, p = S.routing(r2, T, E, k)
+        lo, hi = ep.shard_range(E, world, rank)
+        seen = []
+
+        def compute(rows, rid):
+            bits = rows.view(torch.int16).numpy().view(np.uint16)
+            rid = rid.numpy()
+            seen.append(rid.copy())
+            if len(rid) == 0:
+                return torch.empty((0, H), dtype=torch.float32)
+            out = O.moe(gate, up, down, vals, bits, rid[:, None], np.ones((len(rid), 1), np.float32))
+            return torch.from_numpy(out["y"].astype(np.float32))
+
+        def combine(rows, pw):
+            r = rows.numpy().reshape(T, k, H)
+            acc = np.zeros((T, H), np.float32)
+            for j in range(k):  # slot order, float32, as the device combine
+                acc = acc + pw.numpy()[:, j:j + 1] * r[:, j]
+            return O.bf16_round(acc)
+
+        mod = ep.ExpertParallelPrefill(gate, up, down, vals, compute=compute, combine=combine)
+        y = mod(torch.from_numpy(x.view(np.int16)).view(torch.bfloat16), torch.from_numpy(ids), torch.from_numpy(p))
+        got = np.concatenate(seen) if seen else np.zeros(0, np.int32)
+        assert np.all((got >= lo) & (got < hi)), "a pair reached a rank that does not own its expert"
+        # every pair routed to this rank's experts, from every rank's tokens, arrived here
+        owned = [ep.shard_range(E, world, r) for r in range(world)]
+        routed = torch.tensor([int(np.sum((ids >= a) & (ids < b))) for a, b in owned])
+        dist.all_reduce(routed)
+        assert len(got) == int(routed[rank])
+        check_y(y, O.moe(gate, up, down, vals, x, ids, p), None, f"rank {rank}")
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world", [2, 3])
+def test_gloo_ranks_dispatch_and_combine_the_prefill(world):
+    """All-to-all dispatch of every (token, slot) pair to its expert's owner
+    and the combine back, over gloo ranks with different token counts."""
+    torch.multiprocessing.spawn(_prefill_rank, args=(world, _free_port(), 10), nprocs=world, join=True)
+
+
+def test_prefill_plan_groups_pairs_by_owner():
+    mod = ep.ExpertParallelPrefill.__new__(ep.ExpertParallelPrefill)
+    mod.torch, mod.world, mod.experts = torch, 3, 10
+    mod.bounds = [ep.shard_range(10, 3, r) for r in range(3)]
+    mod._starts = torch.tensor([lo for lo, _ in mod.bounds])
+    ids = torch.tensor([[9, 0, 4], [3, 3, 7], [5, 1, 8]], dtype=torch.int32)
+    order, counts = mod.plan(ids)
+    owner = [next(r for r, (lo, hi) in enumerate(mod.bounds) if lo <= e < hi) for e in ids.reshape(-1).tolist()]
+    assert counts.tolist() == [owner.count(r) for r in range(3)]
+    assert order.tolist() == sorted(range(9), key=lambda i: (owner[i], i))
+    with pytest.raises(ValueError):
+        mod.plan(torch.tensor([[10]], dtype=torch.int32))

@@ -101,3 +101,75 @@ def test_module_with_one_rank_equals_the_single_gpu_decode(B):
         torch.cuda.synchronize()
     finally:
         dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("T,world", [(37, 2), (300, 3)])
+def test_prefill_shards_sum_to_the_block(B, T, world, parity_report):
+    """iqk_moe_prefill_shard: each rank's float32 partial against the
+    oracle's part (h from the shard's workspace), the partials summed and
+    rounded against the whole block."""
+    gate, up, down, vals, x, ids, p = _case(760 + T, T)
+    xd, idd, pd = to_dev_bf16(x), torch.from_numpy(ids).cuda(), torch.from_numpy(p).cuda()
+    H, F, k = gate.cols, gate.rows, ids.shape[1]
+    total = torch.zeros((T, down.rows), dtype=torch.float32, device="cuda")
+    h_all = np.full((T, k, F), np.nan)
+    for r in range(world):
+        lo, hi = ep.shard_range(gate.experts, world, r)
+        wsr = [B.Weights.from_host(ep.shard_streams(w, lo, hi)) for w in (gate, up, down)]
+        ws = B.workspace(B.iqk_moe_workspace_bytes(1, T, k, hi - lo, H, F))
+        part = B.iqk_moe_prefill_shard(*wsr, vals, xd, idd, pd, lo, ws=ws)
+        torch.cuda.synchronize()
+        assert B.iqk_moe_status(ws) == B.IQK_OK  # other ranks' ids are not errors
+        mine = (ids >= lo) & (ids < hi)
+        h = read_h(B, ws, 1, T, k, hi - lo, H, F, valid_pairs=int(mine.sum()))
+        h_all[mine] = h[mine]
+        out = check_block(part.cpu().numpy(), h, O.moe_shard(gate, up, down, vals, x, ids, p, lo, hi), down, vals,
+                          ids, np.where(mine, p, 0), f"prefill shard {r}/{world} T={T}", pairs=mine, y_f32=True)
+        parity_report(f"prefill shard {r}/{world} T={T}", flat_stats(out))
+        total += part
+    y = from_dev_bf16(B.iqk_f32_to_bf16(total))
+    out = check_block(y, h_all, O.moe(gate, up, down, vals, x, ids, p), down, vals, ids, p,
+                      f"sum of {world} prefill shards T={T}")
+    parity_report(f"sum of {world} prefill shards T={T}", flat_stats(out))
+
+
+def test_combine_is_the_slot_order_weighted_sum(B):
+    """iqk_moe_combine: y[t] = bf16(sum over slots in order of p * row), within
+    one bf16 spacing of the exact sum (the rounding of float32 partial sums)."""
+    rng = np.random.default_rng(5)
+    T, k, H = 33, 6, 512
+    rows = rng.standard_normal((T * k, H)).astype(np.float32)
+    p = rng.random((T, k)).astype(np.float32)
+    y = from_dev_bf16(B.iqk_moe_combine(torch.from_numpy(rows).cuda(), torch.from_numpy(p).cuda()))
+    exact = np.einsum("tj,tjh->th", p.astype(np.float64), rows.reshape(T, k, H).astype(np.float64))
+    got = (y.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    spac = 2.0 ** (np.floor(np.log2(np.maximum(np.abs(exact), 2.0 ** -126))) - 7)
+    assert np.all(np.abs(got - exact) <= spac + 1e-6 * np.abs(rows).max())
+
+
+def test_prefill_module_with_one_rank_equals_the_single_gpu_prefill(B, parity_report):
+    """The all-to-all prefill with one rank (no group, then a one-rank NCCL
+    group): every pair is dispatched to itself, computed as one float32 row
+    and combined; against the oracle, and compared with iqk_moe_prefill."""
+    import torch.distributed as dist
+    gate, up, down, vals, x, ids, p = _case(730, 40)
+    xd, idd, pd = to_dev_bf16(x), torch.from_numpy(ids).cuda(), torch.from_numpy(p).cuda()
+    dg, du, dd = (B.Weights.from_host(w) for w in (gate, up, down))
+    ref_dev = from_dev_bf16(B.iqk_moe_prefill(dg, du, dd, vals, xd, idd, pd))
+    ref = O.moe(gate, up, down, vals, x, ids, p)
+    mod = ep.ExpertParallelPrefill(gate, up, down, vals)
+    y = from_dev_bf16(mod(xd, idd, pd))
+    out = check_block(y, None, ref, down, vals, ids, p, "one-rank prefill module")
+    parity_report("one-rank prefill module", dict(flat_stats(out), equal_to_single_gpu=bool(np.array_equal(y, ref_dev))))
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(_free_port())
+    import datetime
+    dist.init_process_group("nccl", rank=0, world_size=1, device_id=torch.device("cuda:0"),
+                            timeout=datetime.timedelta(seconds=60))
+    try:
+        mod1 = ep.ExpertParallelPrefill(gate, up, down, vals)
+        y1 = from_dev_bf16(mod1(xd, idd, pd))
+        torch.cuda.synchronize()
+        assert np.array_equal(y1, y)
+    finally:
+        dist.destroy_process_group()

@@ -1,12 +1,13 @@
 """Pricing against the deleted-decode floor (mlx-iqk 0.1.1 PKG-INFO, section
-"Pricing"): validation first, then the timed arms and the declared gates.
+"Pricing"): the validation half. Every arm the benchmark times is checked
+against the oracle here: the routed projection decode within the stated
+tolerance, the dequantizer and both floors' integer signatures bit for bit
+(every load reached the output).
 
 Per member (IQ2_KS, IQ2_K) and projection (gate/up [2048 x 4096], down
-[4096 x 2048]), 256 experts resident: the routed projection decode and the
-dequantizer, each against its own floor. Before any timing, every arm's output
-is checked against the oracle (the floors' integer signatures bit for bit,
-which shows that every load reached the output). Then the gates: the declared
-ratio bar, the floor-rate band and no kernel faster than its own floor.
+[4096 x 2048]), 256 experts resident. The timed half -- the declared ratio
+bar, the floor-rate band and no kernel faster than its own floor -- runs in
+bench.py (details.pricing), so that a slow box cannot turn a parity run red.
 """
 import numpy as np
 import pytest
@@ -48,24 +49,15 @@ def _validate(cell):
 
 
 @pytest.mark.parametrize("fmt", ["iq2_ks", "iq2_k"])
-def test_pricing_cells_validate_then_meet_the_declared_gates(B, fmt):
+def test_pricing_arms_validate(B, fmt):
     import bench as BE
-    peaks = BE.measured_peaks()
     rng = S.rng_for(77)
     values = S.value_table("int" if fmt == "iq2_ks" else "f16", 5)
     device, stream = torch.device("cuda:0"), torch.cuda.Stream()
-    cells = []
-    for proj, (rows, cols) in (("gate/up", (S.INTER, S.HIDDEN)), ("down", (S.HIDDEN, S.INTER))):
+    for seed, (rows, cols) in enumerate(((S.INTER, S.HIDDEN), (S.HIDDEN, S.INTER))):
         w = S.random_streams(rng, fmt, S.EXPERTS, rows, cols)
-        cell = BE.PriceCell(torch, B, w, values, device, stream, seed=len(cells) + 3, calls=84)
+        cell = BE.PriceCell(torch, B, w, values, device, stream, seed=seed + 3, calls=84)
         _validate(cell)
-        t = cell.time(reps=3)
-        cells.append({"member": fmt, "projection": proj,
-                      "decode_over_floor": t["decode"] / t["floor"],
-                      "dequant_over_floor": t["dequant"] / t["dequant_floor"],
-                      "floor_gbs": cell.decode_bytes / (t["floor"] * 1e-6) / 1e9,
-                      "dequant_floor_gbs": cell.dequant_bytes / (t["dequant_floor"] * 1e-6) / 1e9})
+        assert B.iqk_floor_status(stream) == B.IQK_OK
         del cell, w
         torch.cuda.empty_cache()
-    fails = BE.price_gates(cells, peaks["hbm_gbs"])
-    assert not fails, "\n".join(fails) + f"\n{cells}"
