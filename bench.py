@@ -735,6 +735,8 @@ def main():
         with torch.cuda.stream(stream):
             for _ in range(rolls):
                 graphs[0].replay()
+            if K % RING:  # the timed remainder graph's first launch (its upload) stays out of the timed region
+                graphs[1][K % RING].replay()
 
     with ClockSampler(torch.cuda.get_device_properties(device)) as clk:
         roll()

@@ -27,20 +27,18 @@
 #include "iqk_internal.h"
 
 // Selector arithmetic of the code lookup: 0 all shifts on the integer-logic
-// pipe; 1 the high-half selector by multiply-high; 2 as 1, plus slot 2's
-// pre-shift by multiply-high; 3 both halves from one wide multiply-add
-// (moves work from the integer-logic pipe to the FMA pipe).
+// pipe (the default: fastest measured on B200 with the unrolled item loop);
+// 1 the high-half selector by multiply-high; 2 as 1, plus slot 2's pre-shift
+// by multiply-high (moves work from the integer-logic pipe to the FMA pipe).
 #ifndef IQK_LOOKUP
 #define IQK_LOOKUP 0
 #endif
 
-// Group reduction of the tile kernel: 1 the last warp to finish its share of
-// a group sums the group's slots (two slot sets, so warps run one group
-// ahead, no CTA barrier); 0 two CTA barriers per group.
-#ifndef IQK_LAST_ARRIVER
-#define IQK_LAST_ARRIVER 1
+// 1: the item's 256-weight blocks unrolled at compile time (item widths of 2
+// and 4 blocks); 0: a loop over the blocks (smaller code).
+#ifndef IQK_UNROLL_BLOCKS
+#define IQK_UNROLL_BLOCKS 1
 #endif
-constexpr int kSlotSets = IQK_LAST_ARRIVER ? 2 : 1;
 
 namespace iqk {
 
@@ -163,9 +161,6 @@ __device__ __forceinline__ Pair2 lookup(uint32_t q, int i, uint32_t t0, uint32_t
 #if IQK_LOOKUP == 0
   (void)k65536;
   return lookup_slot(q, i, t0, t1);
-#elif IQK_LOOKUP == 3
-  (void)k65536;
-  return lookup_slot_wide(q, i, t0, t1);
 #elif IQK_LOOKUP == 1
   return lookup_slot_mh(q, i, t0, t1, k65536);
 #else
@@ -294,14 +289,17 @@ struct RouteView {
   int32_t* uexp;     // [n] expert id of u
   uint8_t* first;    // [n] scratch
   int32_t* scalars;  // [0] = D, [1] = valid pairs
+  float* pw;         // [n] routing weights (down kernel)
 };
 
 __host__ __device__ inline size_t route_smem_bytes(int n) {
-  return (size_t)n * 4 + (size_t)n * 2 + (size_t)(n + 1) * 2 + (size_t)n * 4 + (size_t)n + 16 + 64;
+  return (size_t)n * 4 + (size_t)n * 2 + (size_t)(n + 1) * 2 + (size_t)n * 4 + (size_t)n + 16 + 64 + (size_t)n * 4;
 }
 
 __device__ __forceinline__ RouteView carve_route(uint8_t* p, int n) {
   RouteView r;
+  r.pw = reinterpret_cast<float*>(p);
+  p += (size_t)n * 4;
   r.ids = reinterpret_cast<int32_t*>(p);
   p += (size_t)n * 4;
   r.uexp = reinterpret_cast<int32_t*>(p);
@@ -737,9 +735,9 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, kDecodeMinBlocks(NT)) k_str
       // IQ2_KS row scales of rows g and g + 8, applied after the slice's MMAs
       const float dg = kfmt ? 0.f : d_smem_ks(slot, bpi, g), dh = kfmt ? 0.f : d_smem_ks(slot, bpi, g + 8);
       // unrolled over the item's blocks where registers allow (one or two column groups)
-      if (NT <= 2 && bpi == 4)
+      if (IQK_UNROLL_BLOCKS && NT <= 2 && bpi == 4)
         item_mma<F0, F1, NT, BSM, 4>(sq, slot, bpi, o, ldw, bsrc, fmt0, kfmt, lut0, lut1, dg, dh, g, t, k65536, acc);
-      else if (NT <= 2 && bpi == 2)
+      else if (IQK_UNROLL_BLOCKS && NT <= 2 && bpi == 2)
         item_mma<F0, F1, NT, BSM, 2>(sq, slot, bpi, o, ldw, bsrc, fmt0, kfmt, lut0, lut1, dg, dh, g, t, k65536, acc);
       else
         item_mma<F0, F1, NT, BSM>(sq, slot, bpi, o, ldw, bsrc, fmt0, kfmt, lut0, lut1, dg, dh, g, t, k65536, acc);
@@ -840,12 +838,10 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, kDecodeMinBlocks(NT)) k_til
   uint2* lut1 = lut0 + 64;
   const int KP = BSM ? K / 64 * 80 : K;  // activation row stride (elements), see k_stream
   uint16_t* act_s = reinterpret_cast<uint16_t*>(lut1 + 64);
-  // group-reduction words: arrivals and completed reductions per slot set
-  int* gsync = reinterpret_cast<int*>(reinterpret_cast<uint8_t*>(act_s) + (BSM ? (size_t)A.act_rows * KP * 2 : 0));
-  float* red = reinterpret_cast<float*>(gsync + 4);
+  float* red = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(act_s) + (BSM ? (size_t)A.act_rows * KP * 2 : 0));
   // floats per warp slot: (mat, column, row) gate/up; (column, row) switch; (token, row) down
   const int slot_f = MODE == MODE_GATEUP ? 2 * NC * kTile : MODE == MODE_SWITCH ? NC * kTile : A.T * kTile;
-  uint8_t* route_p = reinterpret_cast<uint8_t*>(red + (size_t)kSlotSets * kDecodeWarps * slot_f);
+  uint8_t* route_p = reinterpret_cast<uint8_t*>(red + (size_t)kDecodeWarps * slot_f);
   // This kernel starts only after the call's first kernel has seen the
   // previous work on the stream complete (that kernel waits before it lets
   // its dependents launch), so the call's inputs (x, ids, p) and the weight
@@ -861,7 +857,6 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, kDecodeMinBlocks(NT)) k_til
     if (wid == 0) mbar_init(never_bar, 1);
     fence_mbar_init();
   }
-  if (threadIdx.x < 4) gsync[threadIdx.x] = 0;  // visible to all after build_route's barriers
   griddep_launch();
   // gate/up and switch: request the first activation groups ahead of the weight stream
   uint4 pre0 = make_uint4(0u, 0u, 0u, 0u), pre1 = pre0, pre2 = pre0, pre3 = pre0;
@@ -878,6 +873,8 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, kDecodeMinBlocks(NT)) k_til
     }
   }
   const RouteView rt = carve_route(route_p, npairs);
+  if (MODE == MODE_DOWN)  // the routing weights, read once per pair and item below
+    for (int i = threadIdx.x; i < npairs; i += blockDim.x) rt.pw[i] = __ldcg(A.p + i);
   build_route(A.ids, npairs, A.w0.experts, rt, NC, A.ebase);  // ends with __syncthreads; runs of <= NC pairs
   const int D = rt.scalars[0];
   const int rows = A.w0.rows;
@@ -979,36 +976,15 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, kDecodeMinBlocks(NT)) k_til
   const uint16_t* act_base = BSM ? act_s : A.act;
   constexpr int SEG = BSM ? 80 : 64;
   constexpr int BLKE = BSM ? 320 : 256;
+  float* my = red + (size_t)wid * slot_f;
   bool failed = false;
   if (A.expire && wid == 0 && !mbar_wait_ns(never_bar, 0, A.wait_ns)) {  // testing hook: this wait runs out
-    failed = true;  // keep taking part in the group reductions; stop loading
+    failed = true;  // keep taking part in the CTA barriers; stop loading
     if (lane == 0) atomicOr(A.status, 2);
   }
-  // warps with items in a group: 0 .. P-1 (cnt_w > 0 exactly for them)
-  const int P = n_it < kDecodeWarps ? n_it : kDecodeWarps;
   int consumed = 0;
   int q = 0;
   for (int r = 0; r < rounds; r++) {
-    const int set = IQK_LAST_ARRIVER ? (r & 1) : 0;
-    float* my = red + ((size_t)set * kDecodeWarps + wid) * slot_f;
-    if (IQK_LAST_ARRIVER) {
-      if (cnt_w == 0) continue;  // no item of this warp in any group
-      // the set was last used by group r - 2: wait until it has been reduced
-      if (r >= 2) {
-        volatile int* done = gsync + 2 + set;
-        if (*done < (r >> 1)) {
-          const uint64_t t0 = globaltimer_ns();
-          while (*done < (r >> 1)) {
-            if (globaltimer_ns() - t0 >= A.wait_ns) {
-              if (!failed && lane == 0) atomicOr(A.status, 2);
-              failed = true;
-              break;
-            }
-          }
-        }
-        __threadfence_block();
-      }
-    }
     for (int i = lane; i < slot_f; i += 32) my[i] = 0.f;
     __syncwarp();
     for (int k = 0; k < cnt_w; k++, q++) {
@@ -1035,7 +1011,7 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, kDecodeMinBlocks(NT)) k_til
         for (int qq = 0; qq < 4; qq++) acc[n][qq] = 0.f;
       const int st = q % kStages;
       if (!failed && !mbar_wait_ns(&bar[st], (uint32_t)((q / kStages) & 1), A.wait_ns)) {
-        failed = true;  // keep taking part in the group reductions; stop loading
+        failed = true;  // keep taking part in the CTA barriers; stop loading
         if (lane == 0) atomicOr(A.status, 2);
       }
       if (!failed) {
@@ -1044,9 +1020,9 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, kDecodeMinBlocks(NT)) k_til
         const uint8_t* slot = ring_slots + (size_t)st * slot_b;
         const int o = A.async_sc ? (s * bpi) & 3 : 0;
         const float dg = kfmt ? 0.f : d_smem_ks(slot, bpi, g), dh = kfmt ? 0.f : d_smem_ks(slot, bpi, g + 8);
-        if (bpi == 4)
+        if (IQK_UNROLL_BLOCKS && bpi == 4)
           item_mma<F0, F1, NT, BSM, 4>(sq, slot, bpi, o, ldw, bsrc, fmt0, kfmt, lut0, lut1, dg, dh, g, t, k65536, acc);
-        else if (bpi == 2)
+        else if (IQK_UNROLL_BLOCKS && bpi == 2)
           item_mma<F0, F1, NT, BSM, 2>(sq, slot, bpi, o, ldw, bsrc, fmt0, kfmt, lut0, lut1, dg, dh, g, t, k65536, acc);
         else
           item_mma<F0, F1, NT, BSM>(sq, slot, bpi, o, ldw, bsrc, fmt0, kfmt, lut0, lut1, dg, dh, g, t, k65536, acc);
@@ -1070,46 +1046,30 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, kDecodeMinBlocks(NT)) k_til
             for (int qq = 0; qq < 4; qq++) {
               if (8 * n + 2 * t + (qq & 1) != c) continue;
               const int pair = rt.sorted[p0 + c];
-              my[(pair / A.topk) * kTile + g + 8 * (qq >> 1)] += __ldcg(A.p + pair) * acc[n][qq];
+              my[(pair / A.topk) * kTile + g + 8 * (qq >> 1)] += rt.pw[pair] * acc[n][qq];
             }
           __syncwarp();
         }
       }
       __syncwarp();
     }
-    // The group's reduction, by all threads after a CTA barrier, or by the
-    // last warp to add its slot (the slots summed in warp order either way).
-    int rt0 = threadIdx.x, rstep = blockDim.x;
-    if (IQK_LAST_ARRIVER) {
-      int last = 0;
-      if (lane == 0) {
-        __threadfence_block();
-        last = atomicAdd(gsync + set, 1) == P - 1;
-      }
-      if (!__shfl_sync(0xffffffffu, last, 0)) continue;
-      __threadfence_block();
-      rt0 = lane;
-      rstep = 32;
-    } else {
-      __syncthreads();  // every warp's slot of this group is complete
-    }
-    const float* rb = red + (size_t)set * kDecodeWarps * slot_f;
+    __syncthreads();  // every warp's slot of this group is complete
     const int tg = (int)blockIdx.x + r * (int)gridDim.x;
     if (MODE == MODE_GATEUP) {
       const int u = (int)A.div_tiles.div((uint32_t)tg);
       const int tile = tg - u * tiles;
       const int p0 = rt.ustart[u];
       const int ncols = min(rt.ustart[u + 1] - p0, NC);  // runs never exceed NC; the bound guards the slot reads
-      for (int o = rt0; o < ncols * kTile; o += rstep) {
+      for (int o = threadIdx.x; o < ncols * kTile; o += blockDim.x) {
         const int col = o / kTile, row = o - col * kTile;
         const int f = tile * kTile + row;
         if (f >= rows) continue;
         float gv = 0.f, uv = 0.f;
-        for (int w = 0; w < P; w++) {
-          gv += rb[(size_t)w * slot_f + col * kTile + row];
-          uv += rb[(size_t)w * slot_f + (NC + col) * kTile + row];
+        for (int w = 0; w < kDecodeWarps; w++) {
+          gv += red[(size_t)w * slot_f + col * kTile + row];
+          uv += red[(size_t)w * slot_f + (NC + col) * kTile + row];
         }
-        const float h = gv / (1.0f + __expf(-gv)) * uv;
+        const float h = silu_f32(gv) * uv;
         A.out16[(size_t)rt.sorted[p0 + col] * rows + perm16(f)] = f32_to_bf16_bits(h);
       }
     } else if (MODE == MODE_SWITCH) {
@@ -1120,37 +1080,28 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, kDecodeMinBlocks(NT)) k_til
       const int p0 = rt.ustart[u];
       const int ncols = min(rt.ustart[u + 1] - p0, NC);
       const int per = ncols * kTile;
-      for (int o = rt0; o < tpg * per; o += rstep) {
+      for (int o = threadIdx.x; o < tpg * per; o += blockDim.x) {
         const int sub = o / per, rem = o - sub * per;
         const int col = rem / kTile, row = rem - col * kTile;
         const int f = (t0 + sub) * kTile + row;
         if (t0 + sub >= tiles || f >= rows) continue;
-        const int w0 = tpg > 1 ? sub * S : 0, w1 = tpg > 1 ? w0 + S : P;
+        const int w0 = tpg > 1 ? sub * S : 0, w1 = tpg > 1 ? w0 + S : kDecodeWarps;
         float v = 0.f;
-        for (int w = w0; w < w1; w++) v += rb[(size_t)w * slot_f + col * kTile + row];
+        for (int w = w0; w < w1; w++) v += red[(size_t)w * slot_f + col * kTile + row];
         A.yf[(size_t)rt.sorted[p0 + col] * rows + f] = v;
       }
     } else {
-      for (int o = rt0; o < A.T * kTile; o += rstep) {
+      for (int o = threadIdx.x; o < A.T * kTile; o += blockDim.x) {
         const int tok = o / kTile, row = o - tok * kTile;
         const int f = tg * kTile + row;
         if (f >= rows) continue;
         float y = 0.f;
-        for (int w = 0; w < P; w++) y += rb[(size_t)w * slot_f + tok * kTile + row];
+        for (int w = 0; w < kDecodeWarps; w++) y += red[(size_t)w * slot_f + tok * kTile + row];
         if (A.yf) A.yf[(size_t)tok * rows + f] = y;  // an expert-parallel partial, summed across ranks
         else A.out16[(size_t)tok * rows + f] = f32_to_bf16_bits(y);
       }
     }
-    if (IQK_LAST_ARRIVER) {
-      __syncwarp();  // every lane's reads of the set are done
-      if (lane == 0) {
-        gsync[set] = 0;
-        __threadfence_block();
-        *(volatile int*)(gsync + 2 + set) = (r >> 1) + 1;
-      }
-    } else {
-      __syncthreads();  // slots free for the next group
-    }
+    __syncthreads();  // slots free for the next group
   }
   // let copies still in flight land before the CTA exits (only after a timeout)
   for (int qd = consumed; qd < issued; qd++) (void)mbar_wait_ns(&bar[qd % kStages], (uint32_t)((qd / kStages) & 1), kDrainWaitNs);
@@ -1213,8 +1164,8 @@ template <int MODE, int F0, int F1, int NT>
 static size_t tiles_smem(int cols, int T, int npairs, int act_rows) {
   const int bpi = item_blocks(cols);
   const size_t warp = (size_t)kStages * ((size_t)kTile * bpi * 16 * 4 + slot_bytes2<F0, F1>(bpi));
-  const size_t red = 16 + (size_t)kSlotSets * kDecodeWarps *
-                              (MODE == MODE_GATEUP ? 2 * 8 * NT * kTile : MODE == MODE_SWITCH ? 8 * NT * kTile : T * kTile) * 4;
+  const size_t red =
+      (size_t)kDecodeWarps * (MODE == MODE_GATEUP ? 2 * 8 * NT * kTile : MODE == MODE_SWITCH ? 8 * NT * kTile : T * kTile) * 4;
   return kDecodeWarps * warp + (size_t)kDecodeWarps * kStages * 8 + 16 + 2 * 64 * 8 + (size_t)act_rows * (cols / 64 * 80) * 2 +
          red + route_smem_bytes(npairs);
 }

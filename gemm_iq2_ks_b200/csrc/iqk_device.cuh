@@ -149,6 +149,16 @@ __device__ __forceinline__ uint2 ld_nc_u2(const void* p) {
   return r;
 }
 
+// silu(g) = g / (1 + e^-g), evaluated as g * sigmoid(g) from e = exp(-|g|),
+// which never overflows: sigmoid(g) = 1 / (1 + e) for g >= 0 and e / (1 + e)
+// below. The plain quotient overflows e^-g to infinity below g = -88 and
+// returns 0 where silu(g) is still a normal float (about -90 * e^-90).
+__device__ __forceinline__ float silu_f32(float g) {
+  const float e = expf(-fabsf(g));
+  const float r = 1.0f / (1.0f + e);
+  return g * (g >= 0.f ? r : e * r);
+}
+
 // bf16 helpers (bit patterns)
 __device__ __forceinline__ float bf16_bits_to_f32(uint16_t b) { return __uint_as_float((uint32_t)b << 16); }
 __device__ __forceinline__ uint16_t f32_to_bf16_bits(float f) {
@@ -177,26 +187,6 @@ __device__ __forceinline__ Pair2 lookup_slot(uint32_t q, int i, uint32_t t0, uin
   Pair2 r;
   r.lo = prmt(t0, t1, s);
   r.hi = prmt(t0, t1, s >> 16);
-  return r;
-}
-
-// Same, with both selector halves from one 32 x 32 -> 64-bit multiply-add:
-// with V = u * 0x22, u * 0x00220022 = V + V * 2^16, whose low word holds V's
-// low half in bits 0..15 and whose high word is V's high half exactly (the
-// middle sum stays below 2^32 because every byte of V is at most 0x66). The
-// 64-bit addend puts 0x1010 on both halves. This replaces the integer-logic
-// pipe's 16-bit shift with work on the FMA pipe.
-__device__ __forceinline__ Pair2 lookup_slot_wide(uint32_t q, int i, uint32_t t0, uint32_t t1) {
-  const uint32_t u = (q >> (2 * i)) & 0x03030303u;
-  uint32_t lo, hi;
-  asm("{\n\t.reg .u64 w;\n\t"
-      "mad.wide.u32 w, %2, 0x00220022, 0x0000101000001010;\n\t"
-      "mov.b64 {%0, %1}, w;\n\t}"
-      : "=r"(lo), "=r"(hi)
-      : "r"(u));
-  Pair2 r;
-  r.lo = prmt(t0, t1, lo);
-  r.hi = prmt(t0, t1, hi);
   return r;
 }
 

@@ -388,7 +388,7 @@ __global__ void __launch_bounds__(PF_THREADS, 2) k_pf_gemm(const __grid_constant
               const int n = c0 + i;
               if (n < ncols) {
                 const float gv = g8[i] * dg, uv = u8[i] * du;
-                const float h = gv / (1.0f + __expf(-gv)) * uv;
+                const float h = silu_f32(gv) * uv;
                 A.hs[(size_t)(off + n0 + n) * Fdim + perm16(f)] = f32_to_bf16_bits(h);
               }
             }

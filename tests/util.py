@@ -87,8 +87,11 @@ def h_interval(ref):
     c = np.stack([s_lo * (u - du), s_lo * (u + du), s_hi * (u - du), s_hi * (u + du)])
     lo, hi = c.min(axis=0), c.max(axis=0)
     # the kernel evaluates silu and the product in float32 with its own exp:
-    # allow a relative 2^-20 on top (float32 keeps 24 bits)
-    slack = 2.0 ** -20 * np.maximum(np.abs(lo), np.abs(hi)) + 1e-37
+    # a relative 2^-20 on top (float32 keeps 24 bits), and an absolute floor
+    # for e^g below float32's normal range (2^-126), where silu(g) = g e^g /
+    # (1 + e^g) can lose up to |g| 2^-126 before the product with u
+    slack = (2.0 ** -20 * np.maximum(np.abs(lo), np.abs(hi))
+             + 2.0 ** -126 * np.maximum(1.0, np.abs(g) + dg) * (np.abs(u) + du) + 2.0 ** -149)
     return lo - slack, hi + slack
 
 
