@@ -39,7 +39,7 @@ RING = 420  # calls per captured graph (10 permutation cycles of 42 calls)
 # call (IQ2_KS, 256 experts, top-6, one token), from one ncu capture of
 # `bench.py --profile decode --experts 24` (its summary is kept under
 # profiles/); per call, not per resident expert.
-DECODE_CALL_TRAFFIC = 41_575_424
+DECODE_CALL_TRAFFIC = 41_570_304  # 27,659,776 (gate/up) + 13,910,528 (down)
 
 
 def env_int(k, d):

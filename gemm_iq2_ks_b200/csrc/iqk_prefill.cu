@@ -148,18 +148,18 @@ __device__ __forceinline__ bool pf_produce(const WDev& W, int64_t grow, int nch,
   const uint32_t tlane = tmem + ((uint32_t)(32 * q) << 16) + TM_A + (tile ? 32u : 0u);
   uint32_t ra[32], rb[32];
   int pend_sa = -1;  // stage of the chunk whose store is in flight
-  // decode chunk c into regs; returns the A stage it goes to, or -1 after a failed wait
-  auto decode = [&](int c, uint32_t (&regs)[32]) -> int {
+  // Decode chunk c into regs (registers only: the A stage is claimed after
+  // the decode, just before the tensor-memory store, so the decode overlaps
+  // the MMAs still reading that stage). Returns false after a failed wait.
+  auto decode = [&](int c, uint32_t (&regs)[32]) -> bool {
     const int s = qi % PF_SQ;
     if ((c & 3) == 0) {
       if (c > 0) {
         sc = scn;
         if ((c >> 2) + 1 < nb) scn = load_blk<FMT>(W, grow, (c >> 2) + 1);
       }
-      if (!pf_wait(&qs_full[s], (qi / PF_SQ) & 1, abort_flag, status)) return -1;
+      if (!pf_wait(&qs_full[s], (qi / PF_SQ) & 1, abort_flag, status)) return false;
     }
-    const int sa = ai % PF_SA;
-    if (!pf_wait(&a_free[sa], ((ai / PF_SA) & 1) ^ 1, abort_flag, status)) return -1;
     // qs tiles arrive with the 64-byte swizzle: 16-byte chunk j of row r sits at chunk j ^ ((r >> 1) & 3)
     const uint4 qw = *reinterpret_cast<const uint4*>(qbuf + (size_t)s * (PF_Q_BYTES / 4) + (tile ? 128 * 16 : 0) +
                                                      r * 16 + 4 * ((c & 3) ^ ((r >> 1) & 3)));
@@ -179,6 +179,12 @@ __device__ __forceinline__ bool pf_produce(const WDev& W, int64_t grow, int nch,
       if (lane == 0) mbar_arrive(&qs_empty[s]);
       qi++;
     }
+    return true;
+  };
+  // the next A stage, once the MMAs that read it last have completed; -1 after a failed wait
+  auto claim = [&]() -> int {
+    const int sa = ai % PF_SA;
+    if (!pf_wait(&a_free[sa], ((ai / PF_SA) & 1) ^ 1, abort_flag, status)) return -1;
     ai++;
     return sa;
   };
@@ -190,20 +196,27 @@ __device__ __forceinline__ bool pf_produce(const WDev& W, int64_t grow, int nch,
     if (lane == 0) mbar_arrive(&a_ready[pend_sa]);
   };
   for (int c = 0; c < nch; c += 2) {
-    int sa = decode(c, ra);
-    if (sa < 0) {
+    int sa;
+    if (!decode(c, ra)) {
       tmem_wait_st();
       return false;
     }
     publish();
+    if ((sa = claim()) < 0) {
+      tmem_wait_st();
+      return false;
+    }
     tmem_st32(tlane + 64u * sa, ra);
     pend_sa = sa;
-    sa = decode(c + 1, rb);
-    if (sa < 0) {
+    if (!decode(c + 1, rb)) {
       tmem_wait_st();
       return false;
     }
     publish();
+    if ((sa = claim()) < 0) {
+      tmem_wait_st();
+      return false;
+    }
     tmem_st32(tlane + 64u * sa, rb);
     pend_sa = sa;
   }
