@@ -34,24 +34,15 @@
 #define IQK_LOOKUP 0
 #endif
 
-// 1: the item's 256-weight blocks unrolled at compile time (item widths of 2
-// and 4 blocks); 0: a loop over the blocks (smaller code).
-#ifndef IQK_UNROLL_BLOCKS
-#define IQK_UNROLL_BLOCKS 1
-#endif
-
 namespace iqk {
 
 // Blocks per item: four for rows of at least 16 blocks, two for shorter rows
 // with a multiple of four blocks (more items to spread over the warps), else
 // two or one. With a multiple of four blocks per row every scale slice lies
 // on the boundaries cp.async needs.
-#ifndef IQK_MAX_ITEM_BLOCKS
-#define IQK_MAX_ITEM_BLOCKS 4
-#endif
 int item_blocks(int cols) {
   const int nbk = cols / 256;
-  if (nbk % 4 == 0) return nbk >= 16 && IQK_MAX_ITEM_BLOCKS >= 4 ? 4 : 2;
+  if (nbk % 4 == 0) return nbk >= 16 ? 4 : 2;
   return nbk % 2 == 0 ? 2 : 1;
 }
 static bool async_scales(int cols) { return (cols / 256) % 4 == 0; }
@@ -177,47 +168,11 @@ __device__ __forceinline__ Pair2 lookup(uint32_t q, int i, uint32_t t0, uint32_t
 // Each of the block's four qs words feeds its own accumulator set, so
 // consecutive MMAs do not wait on each other; half a block's activation
 // fragments are requested ahead of their MMAs.
-#ifndef IQK_MMA_ORDER
-#define IQK_MMA_ORDER 0
-#endif
 template <int FMT, int NT, bool BSM>
 __device__ __forceinline__ void block_mma(const uint32_t* __restrict__ sq, int ldw, int bcol, const uint16_t* const (&src)[NT],
                                           const uint32_t (&cg)[4], const uint32_t (&ch)[4],
                                           const uint2* __restrict__ lut, float (&part)[4][NT][4], int g, int t,
                                           uint32_t k65536) {
-#if IQK_MMA_ORDER == 1
-  // slot-outer order: the four words' MMAs of one slot are independent, so
-  // consecutive MMAs never wait on each other's accumulators
-  uint4 bf[NT][8];
-#pragma unroll
-  for (int n = 0; n < NT; n++)
-#pragma unroll
-    for (int f = 0; f < 8; f++) bf[n][f] = ld_act<BSM>(src[n] + 8 * f);
-  const uint4 qg = *reinterpret_cast<const uint4*>(sq + g * ldw + bcol + 4 * t);
-  const uint4 qh = *reinterpret_cast<const uint4*>(sq + (g + 8) * ldw + bcol + 4 * t);
-  uint2 tg[4], th[4];
-#pragma unroll
-  for (int m = 0; m < 4; m++) {
-    tg[m] = lut[cg[m]];
-    th[m] = lut[ch[m]];
-  }
-#pragma unroll
-  for (int i = 0; i < 4; i++) {
-#pragma unroll
-    for (int m = 0; m < 4; m++) {
-      const uint32_t wg = m == 0 ? qg.x : m == 1 ? qg.y : m == 2 ? qg.z : qg.w;
-      const uint32_t wh = m == 0 ? qh.x : m == 1 ? qh.y : m == 2 ? qh.z : qh.w;
-      const Pair2 pg = lookup(wg, i, tg[m].x, tg[m].y, k65536);
-      const Pair2 ph = lookup(wh, i, th[m].x, th[m].y, k65536);
-#pragma unroll
-      for (int n = 0; n < NT; n++) {
-        const uint4 b4 = bf[n][4 * (m >> 1) + 2 * (m & 1) + (i >> 1)];
-        const uint32_t b0 = (i & 1) ? b4.z : b4.x, b1 = (i & 1) ? b4.w : b4.y;
-        mma_bf16_4(part[m][n][0], part[m][n][1], part[m][n][2], part[m][n][3], pg.lo, ph.lo, pg.hi, ph.hi, b0, b1);
-      }
-    }
-  }
-#else
   // activation fragments of slots (m, i): 8 bytes each, 32 consecutive bytes per word m
   uint4 bf[NT][4];
 #pragma unroll
@@ -250,7 +205,6 @@ __device__ __forceinline__ void block_mma(const uint32_t* __restrict__ sq, int l
       }
     }
   }
-#endif
 }
 
 // One item (16 rows x bpi blocks) of a matrix in format F0 (fmt0) or F1:
@@ -775,9 +729,9 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, kDecodeMinBlocks(NT)) k_str
       // IQ2_KS row scales of rows g and g + 8, applied after the slice's MMAs
       const float dg = kfmt ? 0.f : d_smem_ks(slot, bpi, g), dh = kfmt ? 0.f : d_smem_ks(slot, bpi, g + 8);
       // unrolled over the item's blocks where registers allow (one or two column groups)
-      if (IQK_UNROLL_BLOCKS && NT <= 2 && bpi == 4)
+      if (NT <= 2 && bpi == 4)
         item_mma<F0, F1, NT, BSM, 4>(sq, slot, bpi, o, ldw, bsrc, fmt0, kfmt, lut0, lut1, dg, dh, g, t, k65536, acc);
-      else if (IQK_UNROLL_BLOCKS && NT <= 2 && bpi == 2)
+      else if (NT <= 2 && bpi == 2)
         item_mma<F0, F1, NT, BSM, 2>(sq, slot, bpi, o, ldw, bsrc, fmt0, kfmt, lut0, lut1, dg, dh, g, t, k65536, acc);
       else
         item_mma<F0, F1, NT, BSM>(sq, slot, bpi, o, ldw, bsrc, fmt0, kfmt, lut0, lut1, dg, dh, g, t, k65536, acc);
@@ -1060,9 +1014,9 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, kDecodeMinBlocks(NT)) k_til
         const uint8_t* slot = ring_slots + (size_t)st * slot_b;
         const int o = A.async_sc ? (s * bpi) & 3 : 0;
         const float dg = kfmt ? 0.f : d_smem_ks(slot, bpi, g), dh = kfmt ? 0.f : d_smem_ks(slot, bpi, g + 8);
-        if (IQK_UNROLL_BLOCKS && bpi == 4)
+        if (bpi == 4)
           item_mma<F0, F1, NT, BSM, 4>(sq, slot, bpi, o, ldw, bsrc, fmt0, kfmt, lut0, lut1, dg, dh, g, t, k65536, acc);
-        else if (IQK_UNROLL_BLOCKS && bpi == 2)
+        else if (bpi == 2)
           item_mma<F0, F1, NT, BSM, 2>(sq, slot, bpi, o, ldw, bsrc, fmt0, kfmt, lut0, lut1, dg, dh, g, t, k65536, acc);
         else
           item_mma<F0, F1, NT, BSM>(sq, slot, bpi, o, ldw, bsrc, fmt0, kfmt, lut0, lut1, dg, dh, g, t, k65536, acc);

@@ -39,13 +39,8 @@ constexpr int kDecodeWarps = IQK_DECODE_WARPS;  // warps per decode CTA, each wi
 constexpr int kStages = IQK_DECODE_STAGES;      // ring stages per warp, one item each
 // Resident CTAs per SM the decode kernels are compiled for (16 warps per SM
 // with one or two MMA column groups, 8 with more).
-#ifndef IQK_DECODE_MIN_BLOCKS
-#define IQK_DECODE_MIN_BLOCKS 0
-#endif
 constexpr int kDecodeMinBlocks(int nt) {
-  return IQK_DECODE_MIN_BLOCKS > 0 && nt <= 2
-             ? IQK_DECODE_MIN_BLOCKS
-             : nt >= 4 ? (8 / kDecodeWarps > 0 ? 8 / kDecodeWarps : 1) : (16 / kDecodeWarps > 0 ? 16 / kDecodeWarps : 1);
+  return nt >= 4 ? (8 / kDecodeWarps > 0 ? 8 / kDecodeWarps : 1) : (16 / kDecodeWarps > 0 ? 16 / kDecodeWarps : 1);
 }
 constexpr int kMaxPairs = 1024;  // routed decode and switch: T * topk
 
