@@ -312,10 +312,13 @@ __device__ __forceinline__ RouteView carve_route(uint8_t* p, int n) {
 // into runs of at most `chunk` (each run its own entry u, so a tile kernel's
 // MMA columns always suffice; such an expert's weights are then read once per
 // run).
-__device__ __forceinline__ void build_route(const int32_t* __restrict__ ids, int n, int E, RouteView r,
+// `my_id`: ids[threadIdx.x], loaded by the caller ahead of time (when
+// threadIdx.x < n).
+__device__ __forceinline__ void build_route(const int32_t* __restrict__ ids, int my_id, int n, int E, RouteView r,
                                             int chunk = 1 << 30, int ebase = 0) {
   for (int p = threadIdx.x; p < n; p += blockDim.x) {
-    const int e = __ldcg(ids + p) - ebase;  // an expert-parallel shard holds experts [ebase, ebase + E)
+    // an expert-parallel shard holds experts [ebase, ebase + E)
+    const int e = (p == (int)threadIdx.x ? my_id : __ldcg(ids + p)) - ebase;
     r.ids[p] = (e >= 0 && e < E) ? e : -1;
   }
   __syncthreads();
@@ -360,6 +363,45 @@ __device__ __forceinline__ void build_route(const int32_t* __restrict__ ids, int
     for (int q = 0; q < nv; q++) D += r.first[q] != 0;
     r.scalars[0] = D;
     r.ustart[D] = (int16_t)nv;
+  }
+  __syncthreads();
+}
+
+// The same list for at most 32 pairs, built by warp 0 alone (lane p holds
+// pair p): stable ranks by ballot and shuffle, run starts by ballot; one CTA
+// barrier at the end.
+__device__ __forceinline__ void build_route_warp(int my_id, int n, int E, RouteView r, int chunk, int ebase) {
+  if (threadIdx.x < 32) {
+    const int lane = threadIdx.x;
+    const int e0 = lane < n ? my_id - ebase : -1;
+    const int ev = (lane < n && e0 >= 0 && e0 < E) ? e0 : -1;
+    if (lane < n) r.ids[lane] = ev;
+    int rank = 0;
+#pragma unroll 4
+    for (int q = 0; q < 32; q++) {
+      const int eq = __shfl_sync(0xffffffffu, ev, q);
+      rank += (eq >= 0) && (eq < ev || (eq == ev && q < lane));
+    }
+    const int nv = __popc(__ballot_sync(0xffffffffu, ev >= 0));
+    if (ev >= 0) r.sorted[rank] = (int16_t)lane;
+    __syncwarp();
+    // position k of the expert order: its expert, and whether a run starts there
+    const int ek = lane < nv ? r.ids[r.sorted[lane]] : -1;
+    const int eprev = __shfl_up_sync(0xffffffffu, ek, 1);
+    const unsigned bound = __ballot_sync(0xffffffffu, lane < nv && (lane == 0 || eprev != ek));
+    const int start = 31 - __clz(bound & (0xffffffffu >> (31 - lane)));  // this expert's first position
+    const unsigned runs = __ballot_sync(0xffffffffu, lane < nv && (lane - start) % chunk == 0);
+    if ((runs >> lane) & 1u) {
+      const int u = __popc(runs & ((1u << lane) - 1u));
+      r.uexp[u] = ek;
+      r.ustart[u] = (int16_t)lane;
+    }
+    if (lane == 0) {
+      const int D = __popc(runs);
+      r.scalars[0] = D;
+      r.scalars[1] = nv;
+      r.ustart[D] = (int16_t)nv;
+    }
   }
   __syncthreads();
 }
@@ -449,6 +491,8 @@ struct UnitArgs {
   int act_rows;  // BSM: activation rows copied into shared memory
   int tpg;       // tile kernel, SWITCH: tiles per group (items per group = splits * tpg)
   int ebase;     // routed modes: first expert id the weights hold (expert-parallel shard)
+  int first;     // tile kernel launched as the call's first kernel (no prep kernel before it)
+  int check_ids; // first: record out-of-range ids in the status word
   int expire;    // testing hook: warp 0 of every CTA also waits on a barrier nothing arrives on
   uint64_t wait_ns;  // bound of every wait on a data barrier (global-timer ns)
   FastDiv div_s, div_tiles;
@@ -575,6 +619,7 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, kDecodeMinBlocks(NT)) k_str
   // BSM rows keep each lane's 64-element segment in 80 elements (160 bytes),
   // so the four segments a warp reads at once start in different bank groups
   const int KP = BSM ? K / 64 * 80 : K;  // activation row stride (elements)
+  if (threadIdx.x == 0) prefetch_tensormap(&m0);
   if (MODE == MODE_GEMV) build_lut<F0>(lut0, A.V);
   if (lane == 0) {
     for (int s = 0; s < kStages; s++) mbar_init(&bar[s], 1);
@@ -844,14 +889,23 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, kDecodeMinBlocks(NT)) k_til
   // What a preceding kernel of the call writes (the status word, transposed
   // x, h) and the outputs are touched only after the dependency wait.
   // Dependents of this kernel may launch at once: they wait the same way.
-  build_lut<F0>(lut0, A.V);
-  if (MODE == MODE_GATEUP) build_lut<F1>(lut1, A.V);
+  // As the call's first kernel (A.first) it waits for everything before it
+  // first, like the prep kernel it replaces, and only then lets the call's
+  // other kernels launch.
+  if (threadIdx.x == 0) {
+    prefetch_tensormap(&m0);
+    if (MODE == MODE_GATEUP) prefetch_tensormap(&m1);
+  }
   if (lane == 0) {
     for (int s = 0; s < kStages; s++) mbar_init(&bar[s], 1);
     if (wid == 0) mbar_init(never_bar, 1);
     fence_mbar_init();
   }
+  if (A.first) griddep_wait();
   griddep_launch();
+  // the call's inputs first (ids, routing weights, x), then the tables while they arrive
+  const int my_id = (int)threadIdx.x < npairs ? __ldcg(A.ids + threadIdx.x) : 0;
+  const float my_p = (MODE == MODE_DOWN && (int)threadIdx.x < npairs) ? __ldcg(A.p + threadIdx.x) : 0.f;
   // gate/up and switch: request the first activation groups ahead of the weight stream
   uint4 pre0 = make_uint4(0u, 0u, 0u, 0u), pre1 = pre0, pre2 = pre0, pre3 = pre0;
   const int act_groups = BSM ? A.act_rows * (K / 16) : 0;
@@ -866,10 +920,14 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, kDecodeMinBlocks(NT)) k_til
       pre3 = ld_cg_u4(A.xraw + (size_t)g1 * 16 + 8);
     }
   }
+  build_lut<F0>(lut0, A.V);
+  if (MODE == MODE_GATEUP) build_lut<F1>(lut1, A.V);
   const RouteView rt = carve_route(route_p, npairs);
   if (MODE == MODE_DOWN)  // the routing weights, read once per pair and item below
-    for (int i = threadIdx.x; i < npairs; i += blockDim.x) rt.pw[i] = __ldcg(A.p + i);
-  build_route(A.ids, npairs, A.w0.experts, rt, NC, A.ebase);  // ends with __syncthreads; runs of <= NC pairs
+    for (int i = threadIdx.x; i < npairs; i += blockDim.x) rt.pw[i] = i == (int)threadIdx.x ? my_p : __ldcg(A.p + i);
+  // ends with __syncthreads; runs of <= NC pairs
+  if (npairs <= 32) build_route_warp(my_id, npairs, A.w0.experts, rt, NC, A.ebase);
+  else build_route(A.ids, my_id, npairs, A.w0.experts, rt, NC, A.ebase);
   const int D = rt.scalars[0];
   const int rows = A.w0.rows;
   const int tiles = (rows + kTile - 1) / kTile;
@@ -922,7 +980,13 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, kDecodeMinBlocks(NT)) k_til
     issued = q + 1;
   };
   for (int q = 0; q < kStages; q++) issue(q);
-  griddep_wait();  // from here on: what the call's preceding kernels wrote, and the outputs
+  if (!A.first) griddep_wait();  // from here on: what the call's preceding kernels wrote, and the outputs
+  // The first kernel resets the call's status word (and records ids outside
+  // [0, E)). Every other write to it is a timeout bit, set at least one wait
+  // bound after this kernel's CTAs have passed their dependency wait, so
+  // after this reset.
+  if (A.first && blockIdx.x == 0 && threadIdx.x == 0)
+    *reinterpret_cast<volatile int32_t*>(A.status) = (A.check_ids && rt.scalars[1] < npairs) ? 1 : 0;
   if constexpr (BSM) {  // activation rows, slot-transposed and padded, once per CTA
     const int gpr = K / 16;
     for (int k = 0;; k++) {
@@ -1452,8 +1516,12 @@ static int decode_impl(const WDev& g, const WDev& u, const WDev& d, const Values
   const int pblocks = std::max(1, std::min(num_sms, (int)(((int64_t)T * (g.cols / 16) + 63) / 64)));
   // a shard skips the ids of other shards silently, so it checks none
   const bool shard = yf != nullptr;
-  if (launch_prep(pblocks, st, x, ar ? 0 : T, g.cols, xp, nullptr, 0, ids, shard ? 0 : npairs, g.experts, status))
+  // With x staged in shared memory there is nothing to transpose: the gate/up
+  // kernel is the call's first kernel and resets the status word itself.
+  if (!ar && launch_prep(pblocks, st, x, T, g.cols, xp, nullptr, 0, ids, shard ? 0 : npairs, g.experts, status))
     return -4;
+  a.first = ar ? 1 : 0;
+  a.check_ids = shard ? 0 : 1;
   a.ebase = ebase;
   a.w0 = g;
   a.w1 = u;
@@ -1472,6 +1540,7 @@ static int decode_impl(const WDev& g, const WDev& u, const WDev& d, const Values
                     : launch_tiles<MODE_GATEUP, FG, FU, NT, false>(mg, mu, a, groups, st, num_sms, true);
   if (rc) return rc;
   UnitArgs b = a;
+  b.first = 0;
   split_args(b, d.cols);
   b.w0 = d;
   b.w1 = d;
@@ -1528,7 +1597,10 @@ static int switch_impl(const WDev& w, const Values& V, const uint16_t* x, int T,
   const int tiles = (w.rows + kTile - 1) / kTile;
   const int ar = act_rows_smem(NT, T, w.cols);  // x rows in shared memory, else transposed by the prep kernel
   const int pblocks = std::max(1, std::min(num_sms, (int)(((int64_t)T * (w.cols / 16) + 63) / 64)));
-  if (launch_prep(pblocks, st, x, ar ? 0 : T, w.cols, xp, nullptr, 0, ids, npairs, w.experts, status)) return -4;
+  // as in the routed decode: with x in shared memory the tile kernel is the call's first kernel
+  if (!ar && launch_prep(pblocks, st, x, T, w.cols, xp, nullptr, 0, ids, npairs, w.experts, status)) return -4;
+  a.first = ar ? 1 : 0;
+  a.check_ids = 1;
   a.w0 = w;
   a.w1 = w;
   a.V = V;
