@@ -411,15 +411,14 @@ extern "C" int iqk_switch_linear(const iqk_weights* w, const float* values, cons
 // ------------------------------------------------------- no-allocation GEMV
 // iqk_gemv_static runs the same launches as iqk_gemv, with its scratch in a
 // file-scope device array instead of a caller-provided workspace. The array
-// lives in every device context that loads the library; its address is
-// looked up once per device (cudaGetSymbolAddress) on the first call there.
-// That first call should happen before any stream capture that records the
-// call. What must start at zero (the tile counters) is zeroed by the call's
-// own first kernel. Calls that overlap in time on one device share the array
-// and race; the caller serialises them (one stream, or events).
+// lives in every device context that loads the library; every call looks up
+// its address in the current context (cudaGetSymbolAddress), so nothing is
+// kept across a device reset. What must start at zero (the tile counters) is
+// zeroed by the call's own first kernel. Calls that overlap in time on one
+// device share the array and race; the caller serialises them (one stream,
+// or events).
 namespace {
 static __device__ __align__(256) unsigned char g_gemv_scratch[IQK_GEMV_STATIC_SCRATCH_BYTES];
-char* g_gemv_scratch_ptr[64] = {nullptr};
 }  // namespace
 
 extern "C" int iqk_gemv_static(const iqk_weights* w, int32_t expert, const float* values, const uint16_t* x,
@@ -432,18 +431,11 @@ extern "C" int iqk_gemv_static(const iqk_weights* w, int32_t expert, const float
   if (!aligned(x, 16) || !aligned(y, 4)) return IQK_EINVAL;
   if (T < 1 || T > 64) return IQK_EUNSUPPORTED;
   if (gemv_ws(T, wd.rows, wd.cols).total > IQK_GEMV_STATIC_SCRATCH_BYTES) return IQK_EWORKSPACE;
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
+  void* scratch = nullptr;
+  const cudaError_t e = cudaGetSymbolAddress(&scratch, g_gemv_scratch);
   if (e != cudaSuccess) return cuda_fail(e);
-  if (dev < 0 || dev >= 64) return IQK_EUNSUPPORTED;
-  if (!g_gemv_scratch_ptr[dev]) {
-    void* p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_gemv_scratch);
-    if (e != cudaSuccess) return cuda_fail(e);
-    g_gemv_scratch_ptr[dev] = static_cast<char*>(p);
-  }
   const int sms = num_sms();
   if (sms < 0) return cuda_fail(cudaGetLastError());
   return from_launch(
-      launch_gemv(wd, w->fmt, expert, V, x, T, y, g_gemv_scratch_ptr[dev], (cudaStream_t)stream, sms));
+      launch_gemv(wd, w->fmt, expert, V, x, T, y, static_cast<char*>(scratch), (cudaStream_t)stream, sms));
 }

@@ -377,8 +377,7 @@ __device__ __forceinline__ void build_route_warp(int my_id, int n, int E, RouteV
     const int ev = (lane < n && e0 >= 0 && e0 < E) ? e0 : -1;
     if (lane < n) r.ids[lane] = ev;
     int rank = 0;
-#pragma unroll 4
-    for (int q = 0; q < 32; q++) {
+    for (int q = 0; q < n; q++) {  // lanes past n hold no pair
       const int eq = __shfl_sync(0xffffffffu, ev, q);
       rank += (eq >= 0) && (eq < ev || (eq == ev && q < lane));
     }
@@ -694,7 +693,7 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, kDecodeMinBlocks(NT)) k_str
   constexpr int BLKE = BSM ? 320 : 256;  // elements between consecutive 256-weight blocks
   griddep_wait();  // from here on: the workspace (transposed x, counters, partial sums) and the outputs
   int32_t* status = A.status ? A.status : &g_floor_status;
-  if (A.expire && wid == 0 && !mbar_wait_ns(never_bar, 0, A.wait_ns)) {  // testing hook: this wait runs out
+  if (A.expire && wid == 0 && !__all_sync(0xffffffffu, mbar_wait_ns(never_bar, 0, A.wait_ns))) {  // testing hook
     if (lane == 0) atomicOr(status, 2);
     for (int k = 0; k < issued; k++) (void)mbar_wait_ns(&bar[k % kStages], (uint32_t)((k / kStages) & 1), kDrainWaitNs);
     return;
@@ -716,7 +715,8 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, kDecodeMinBlocks(NT)) k_str
     const bool fmt0 = true;
     const bool kfmt = F0 == FMT_K;
     const int st = it % kStages;
-    if (!mbar_wait_ns(&bar[st], (uint32_t)((it / kStages) & 1), A.wait_ns)) {
+    // warp-uniform: a lane that saw the data at the bound must not run on alone
+    if (!__all_sync(0xffffffffu, mbar_wait_ns(&bar[st], (uint32_t)((it / kStages) & 1), A.wait_ns))) {
       if (lane == 0) atomicOr(status, 2);
       // let this warp's copies still in flight land before the CTA exits
       for (int k = it; k < issued; k++)

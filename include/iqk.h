@@ -206,10 +206,10 @@ int iqk_switch_linear(const iqk_weights* w, const float* values /* host [8] */, 
  * cannot allocate device memory at the call site (a plain C host linking only
  * this library, or a code path that must not enter an allocator).
  * A shape whose scratch (iqk_gemv_workspace_bytes) exceeds the array returns
- * IQK_EWORKSPACE; the first call on a device looks the array up with
- * cudaGetSymbolAddress, so make it before capturing a stream that records the
- * call. Calls overlapping in time on one device share the array and race:
- * serialise them. Arguments and accuracy as iqk_gemv.
+ * IQK_EWORKSPACE. Every call looks the array's address up in the current
+ * device context (cudaGetSymbolAddress). Calls overlapping in time on one
+ * device share the array and race: serialise them. Arguments and accuracy as
+ * iqk_gemv.
  */
 #define IQK_GEMV_STATIC_SCRATCH_BYTES (4u << 20)
 int iqk_gemv_static(const iqk_weights* w, int32_t expert, const float* values /* host [8] */,
