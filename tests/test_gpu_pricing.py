@@ -43,9 +43,9 @@ def _validate(cell):
     for i, e in enumerate(cell.elist[c].cpu().numpy()):
         assert np.array_equal(fo[i], O.floor_xor(w, int(e))), "floor arm signature"
     e = cell.deq_e[c]
-    assert np.array_equal(cell.dq.cpu().numpy().view(np.uint32),
+    assert np.array_equal(cell.dq[c % 4].cpu().numpy().view(np.uint32),
                           O.dequant_expert(w, e, cell.values).view(np.uint32)), "dequant arm"
-    assert np.array_equal(cell.dqf.cpu().numpy().view(np.uint32), O.dequant_floor(w, e)), "dequant floor signature"
+    assert np.array_equal(cell.dqf[c % 4].cpu().numpy().view(np.uint32), O.dequant_floor(w, e)), "dequant floor signature"
 
 
 @pytest.mark.parametrize("fmt", ["iq2_ks", "iq2_k"])

@@ -5,7 +5,7 @@ import bench as BE
 
 def _cell(**kw):
     c = {"member": "IQ2_KS", "projection": "gate/up", "decode_over_floor": 1.5, "dequant_over_floor": 1.05,
-         "floor_gbs": 2000.0, "dequant_floor_gbs": 5000.0}
+         "floor_gbs": 5000.0, "dequant_floor_gbs": 5000.0}
     c.update(kw)
     return c
 
