@@ -123,9 +123,13 @@ class ClockSampler:
 
 def cuda_time(torch, stream, fn):
     """Device seconds of fn's work: fn runs with `stream` current (graph
-    replays launch on the current stream) between two events on it."""
+    replays launch on the current stream) between two events on it. A short
+    device-side delay (about 0.5 ms of spinning) goes ahead of the first
+    event, so that the host has enqueued fn's launches by the time that event
+    fires: the interval is device time only, not host launch latency."""
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with torch.cuda.stream(stream):
+        torch.cuda._sleep(1_000_000)
         a.record(stream)
         fn()
         b.record(stream)
@@ -312,7 +316,7 @@ def prefill_leg(torch, B, weights, values, device, stream, peaks, calls=4, reps=
             "weight_gbs": sum(w.nbytes() for w in weights) / per_call / 1e9, "status": status}
 
 
-def gemv_leg(torch, B, case, device, stream, calls=200, cold_copies=64):
+def gemv_leg(torch, B, case, device, stream, calls=200, cold_copies=128):
     """A single-matrix workload: one matrix, one activation row. Warm: the
     same matrix every call (L2-resident). Cold: calls rotate over
     ``cold_copies`` distinct matrices of the same shape and distribution
