@@ -148,12 +148,6 @@ __device__ __forceinline__ void griddep_launch() {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
-__device__ __forceinline__ uint2 ld_nc_u2(const void* p) {
-  uint2 r;
-  asm volatile("ld.global.nc.v2.u32 {%0,%1}, [%2];" : "=r"(r.x), "=r"(r.y) : "l"(p));
-  return r;
-}
-
 // silu(g) = g / (1 + e^-g), evaluated as g * sigmoid(g) from e = exp(-|g|),
 // which never overflows: sigmoid(g) = 1 / (1 + e) for g >= 0 and e / (1 + e)
 // below. The plain quotient overflows e^-g to infinity below g = -88 and
@@ -244,12 +238,6 @@ __device__ __forceinline__ uint4 ld_cg_u4(const void* p) {
 __device__ __forceinline__ uint4 ld_u4(const void* p) {
   uint4 r;
   asm volatile("ld.global.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w) : "l"(p));
-  return r;
-}
-
-__device__ __forceinline__ uint4 ld_nc_u4(const void* p) {
-  uint4 r;
-  asm volatile("ld.global.nc.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w) : "l"(p));
   return r;
 }
 
