@@ -25,7 +25,7 @@ EXPORTS = (
     "iqk_moe_workspace_bytes", "iqk_moe_workspace_layout", "iqk_moe_decode", "iqk_moe_decode_shard", "iqk_f32_to_bf16",
     "iqk_moe_prefill", "iqk_moe_prefill_shard", "iqk_moe_combine", "iqk_moe_status",
     "iqk_route_workspace_bytes", "iqk_moe_route", "iqk_floor", "iqk_floor_status", "iqk_set_wait_limit_ns",
-    "iqk_switch_linear_workspace_bytes", "iqk_switch_linear",
+    "iqk_switch_linear_workspace_bytes", "iqk_switch_linear", "iqk_slots_bytes", "iqk_pack_slots",
 )
 
 
@@ -37,7 +37,8 @@ class IqkWsLayout(ctypes.Structure):
 class IqkWeights(ctypes.Structure):
     _fields_ = [("fmt", ctypes.c_int32), ("experts", ctypes.c_int32), ("rows", ctypes.c_int32),
                 ("cols", ctypes.c_int32), ("qs", ctypes.c_void_p), ("scl", ctypes.c_void_p),
-                ("sch", ctypes.c_void_p), ("sex", ctypes.c_void_p), ("dv", ctypes.c_void_p)]
+                ("sch", ctypes.c_void_p), ("sex", ctypes.c_void_p), ("dv", ctypes.c_void_p),
+                ("slots", ctypes.c_void_p)]
 
 
 _lib = None
@@ -87,6 +88,8 @@ def lib(build_if_missing: bool = True) -> ctypes.CDLL:
             "iqk_set_wait_limit_ns": (ctypes.c_int, [ctypes.c_uint64, i32]),
             "iqk_switch_linear_workspace_bytes": (sz, [i32, i32, i32, i32, i32, i32]),
             "iqk_switch_linear": (ctypes.c_int, [W, vp, vp, i32, vp, i32, vp, i32, vp, sz, vp]),
+            "iqk_slots_bytes": (sz, [W]),
+            "iqk_pack_slots": (ctypes.c_int, [W, vp, sz, vp]),
         }
         for name, (res, args) in sig.items():
             f = getattr(L, name)
@@ -134,14 +137,18 @@ def _ptr(t) -> Optional[int]:
 class Weights:
     """Device-resident stacked streams of one weight tensor (torch CUDA tensors)."""
 
-    def __init__(self, fmt: str, experts: int, rows: int, cols: int, qs, scl, sch, sex, dv):
+    def __init__(self, fmt: str, experts: int, rows: int, cols: int, qs, scl, sch, sex, dv, slots=None):
         self.fmt, self.experts, self.rows, self.cols = fmt, experts, rows, cols
         self.qs, self.scl, self.sch, self.sex, self.dv = qs, scl, sch, sex, dv
-        self._c = IqkWeights(FMT[fmt], experts, rows, cols, _ptr(qs), _ptr(scl), _ptr(sch), _ptr(sex), _ptr(dv))
+        self.slots = slots
+        self._c = IqkWeights(FMT[fmt], experts, rows, cols, _ptr(qs), _ptr(scl), _ptr(sch), _ptr(sex), _ptr(dv),
+                             _ptr(slots))
 
     @classmethod
-    def from_host(cls, s, device="cuda") -> "Weights":
-        """Upload host streams (attributes fmt, experts, rows, cols, qs, scl, sch, sex, dv)."""
+    def from_host(cls, s, device="cuda", pack: bool = True) -> "Weights":
+        """Upload host streams (attributes fmt, experts, rows, cols, qs, scl, sch,
+        sex, dv); with `pack` and a CUDA device, also their scale-slot images
+        (iqk_pack_slots)."""
         torch = _torch()
 
         def up(a, dt):
@@ -149,9 +156,29 @@ class Weights:
                 return None
             return torch.from_numpy(np.ascontiguousarray(a).view(dt)).to(device)
 
-        return cls(s.fmt, s.experts, s.rows, s.cols, up(s.qs, np.int32), up(s.scl, np.int32),
-                   up(s.sch, np.uint8), up(s.sex, np.uint8 if s.fmt == "iq2_ks" else np.int16),
-                   up(s.dv, np.int16))
+        w = cls(s.fmt, s.experts, s.rows, s.cols, up(s.qs, np.int32), up(s.scl, np.int32),
+                up(s.sch, np.uint8), up(s.sex, np.uint8 if s.fmt == "iq2_ks" else np.int16),
+                up(s.dv, np.int16))
+        return w.packed() if pack and torch.device(device).type == "cuda" else w
+
+    def packed(self, stream=None) -> "Weights":
+        """These planes with their scale-slot images (iqk_pack_slots), packed on
+        `stream` and complete when this returns."""
+        torch = _torch()
+        plain = self.unpacked()
+        n = lib().iqk_slots_bytes(ctypes.byref(plain.c))
+        if n == 0:
+            raise ValueError("invalid weights")
+        slots = torch.empty((n,), dtype=torch.uint8, device=self.qs.device)
+        st = _stream(stream)
+        _check(lib().iqk_pack_slots(ctypes.byref(plain.c), slots.data_ptr(), n, st), "iqk_pack_slots")
+        torch.cuda.synchronize(self.qs.device)
+        return Weights(self.fmt, self.experts, self.rows, self.cols, self.qs, self.scl, self.sch, self.sex, self.dv,
+                       slots)
+
+    def unpacked(self) -> "Weights":
+        """The same planes without scale-slot images (per-lane scale copies)."""
+        return Weights(self.fmt, self.experts, self.rows, self.cols, self.qs, self.scl, self.sch, self.sex, self.dv)
 
     @property
     def c(self) -> IqkWeights:

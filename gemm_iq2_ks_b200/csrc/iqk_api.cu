@@ -55,11 +55,13 @@ int check_weights(const iqk_weights* w, WDev* out) {
   if (!aligned(w->qs, 16) || !aligned(w->scl, 16) || !aligned(w->sex, 16) || !aligned(w->dv, 16)) return IQK_EINVAL;
   if (w->sch && !aligned(w->sch, 16)) return IQK_EINVAL;
   if ((int64_t)w->experts * w->rows >= (int64_t)1 << 31) return IQK_ESHAPE;
+  if (w->slots && !aligned(w->slots, 16)) return IQK_EINVAL;
   out->qs = w->qs;
   out->scl = w->scl;
   out->sch = w->sch;
   out->sex = w->sex;
   out->dv = w->dv;
+  out->slots = w->slots;
   out->experts = w->experts;
   out->rows = w->rows;
   out->cols = w->cols;
@@ -108,13 +110,30 @@ const char* iqk_strerror(int s) {
 
 const char* iqk_last_cuda_error(void) { return g_cuda_err; }
 
-int iqk_version(void) { return 1; }
+int iqk_version(void) { return 2; }
 
 int64_t iqk_row_bytes(int32_t fmt, int32_t cols) {
   if (cols <= 0 || cols % 256) return -1;
   if (fmt == IQK_IQ2_KS) return 2 + (int64_t)70 * cols / 256;
   if (fmt == IQK_IQ2_K) return (int64_t)76 * cols / 256;
   return -1;
+}
+
+size_t iqk_slots_bytes(const iqk_weights* w) {
+  WDev wd;
+  if (check_weights(w, &wd)) return 0;
+  return slots_bytes(wd, w->fmt);
+}
+
+int iqk_pack_slots(const iqk_weights* w, uint8_t* out, size_t out_bytes, void* stream) {
+  WDev wd;
+  int rc;
+  if ((rc = check_weights(w, &wd))) return rc;
+  wd.slots = nullptr;  // packed from the planes
+  if (!out || !aligned(out, 16) || out_bytes < slots_bytes(wd, w->fmt)) return IQK_EWORKSPACE;
+  const int sms = num_sms();
+  if (sms < 0) return cuda_fail(cudaGetLastError());
+  return from_launch(launch_pack_slots(wd, w->fmt, out, (cudaStream_t)stream, sms));
 }
 
 int iqk_dequant(const iqk_weights* w, int32_t expert, const float* values, float* out, void* stream) {

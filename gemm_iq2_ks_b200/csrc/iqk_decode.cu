@@ -655,9 +655,19 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, kDecodeMinBlocks(NT)) k_str
     const int st = it % kStages;
     int u, tile, s;
     item_of(id, u, tile, s);
-    const int64_t R0 = (int64_t)expert_of(u) * rows + (int64_t)tile * kTile;
+    const int e = expert_of(u);
+    const int64_t R0 = (int64_t)e * rows + (int64_t)tile * kTile;
     const int valid = min(kTile, rows - tile * kTile);
     uint8_t* slot = ring_slots + (size_t)st * slot_b;
+    if (A.w0.slots) {  // the item's scale-slot image: one bulk copy beside the qs tile
+      if (lane == 0) {
+        const uint32_t sb = Slot<F0>::bytes(bpi);
+        mbar_arrive_expect_tx(&bar[st], (uint32_t)stage_words * 4 + sb);
+        tma_load_2d(ring_qs + (size_t)st * stage_words, &m0, s * ldw, (int)R0, &bar[st]);
+        bulk_load(slot, A.w0.slots + ((size_t)((int64_t)e * tiles + tile) * S + s) * sb, sb, &bar[st]);
+      }
+      return;
+    }
     stage_scales<F0>(slot, A.w0, R0, valid, s, bpi, A.async_sc, &bar[st], lane);
     __syncwarp();
     if (lane == 0) {
@@ -749,7 +759,7 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, kDecodeMinBlocks(NT)) k_str
       if (ks) {
         const uint8_t* sb = slot + Slot<FMT_KS>::b_off(bpi);
         const uint8_t* sc = slot + Slot<FMT_KS>::c_off(bpi);
-        const int o = A.async_sc ? (s * bpi) & 3 : 0;
+        const int o = (A.async_sc && !A.w0.slots) ? (s * bpi) & 3 : 0;  // window offset (0 in an image)
         for (int i = t; i < bpi; i += 4) {
           const int sh = 8 * ((s * bpi + i) & 3);
           xg ^= ((uint32_t)sb[g * 4 + o + i] ^ (uint32_t)sc[g * 4 + o + i]) << sh;
@@ -770,7 +780,7 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, kDecodeMinBlocks(NT)) k_str
         }
       }
     } else {
-      const int o = A.async_sc ? (s * bpi) & 3 : 0;
+      const int o = (A.async_sc && !A.w0.slots) ? (s * bpi) & 3 : 0;  // window offset (0 in an image)
       // IQ2_KS row scales of rows g and g + 8, applied after the slice's MMAs
       const float dg = kfmt ? 0.f : d_smem_ks(slot, bpi, g), dh = kfmt ? 0.f : d_smem_ks(slot, bpi, g + 8);
       // unrolled over the item's blocks where registers allow (one or two column groups)
@@ -967,9 +977,21 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, kDecodeMinBlocks(NT)) k_til
     const int st = q % kStages;
     int u, mat, tile, s;
     item_at(q, u, mat, tile, s);
-    const int64_t R0 = (int64_t)rt.uexp[u] * rows + (int64_t)tile * kTile;
+    const int e = rt.uexp[u];
+    const int64_t R0 = (int64_t)e * rows + (int64_t)tile * kTile;
     const int valid = min(kTile, rows - tile * kTile);
     uint8_t* slot = ring_slots + (size_t)st * slot_b;
+    issued = q + 1;
+    const uint8_t* images = mat ? A.w1.slots : A.w0.slots;
+    if (images) {  // the item's scale-slot image: one bulk copy beside the qs tile
+      if (lane == 0) {
+        const uint32_t sb = mat ? Slot<F1>::bytes(bpi) : Slot<F0>::bytes(bpi);
+        mbar_arrive_expect_tx(&bar[st], (uint32_t)stage_words * 4 + sb);
+        tma_load_2d(ring_qs + (size_t)st * stage_words, mat ? &m1 : &m0, s * ldw, (int)R0, &bar[st]);
+        bulk_load(slot, images + ((size_t)((int64_t)e * tiles + tile) * S + s) * sb, sb, &bar[st]);
+      }
+      return;
+    }
     if (mat == 0) stage_scales<F0>(slot, A.w0, R0, valid, s, bpi, A.async_sc, &bar[st], lane);
     else stage_scales<F1>(slot, A.w1, R0, valid, s, bpi, A.async_sc, &bar[st], lane);
     __syncwarp();
@@ -977,7 +999,6 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, kDecodeMinBlocks(NT)) k_til
       mbar_arrive_expect_tx(&bar[st], (uint32_t)stage_words * 4);
       tma_load_2d(ring_qs + (size_t)st * stage_words, mat ? &m1 : &m0, s * ldw, (int)R0, &bar[st]);
     }
-    issued = q + 1;
   };
   for (int q = 0; q < kStages; q++) issue(q);
   if (!A.first) griddep_wait();  // from here on: what the call's preceding kernels wrote, and the outputs
@@ -1076,7 +1097,7 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, kDecodeMinBlocks(NT)) k_til
         consumed = q + 1;
         const uint32_t* sq = ring_qs + (size_t)st * stage_words;
         const uint8_t* slot = ring_slots + (size_t)st * slot_b;
-        const int o = A.async_sc ? (s * bpi) & 3 : 0;
+        const int o = (A.async_sc && !(mat ? A.w1.slots : A.w0.slots)) ? (s * bpi) & 3 : 0;  // 0 in an image
         const float dg = kfmt ? 0.f : d_smem_ks(slot, bpi, g), dh = kfmt ? 0.f : d_smem_ks(slot, bpi, g + 8);
         if (bpi == 4)
           item_mma<F0, F1, NT, BSM, 4>(sq, slot, bpi, o, ldw, bsrc, fmt0, kfmt, lut0, lut1, dg, dh, g, t, k65536, acc);
@@ -1163,6 +1184,57 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, kDecodeMinBlocks(NT)) k_til
   }
   // let copies still in flight land before the CTA exits (only after a timeout)
   for (int qd = consumed; qd < issued; qd++) (void)mbar_wait_ns(&bar[qd % kStages], (uint32_t)((qd / kStages) & 1), kDrainWaitNs);
+}
+
+// ------------------------------------------------------ scale-slot images
+// For every (expert, 16-row tile, reduction slice of bpi blocks) of a weight
+// tensor, the bytes a decode item stages into its shared-memory slot, in the
+// slot layout above with window offset 0 and zeros past the last row (and in
+// the IQ2_KS sch / sex row windows past the slice's bpi bytes). Image
+// (e, tile, s) sits at ((e * tiles + tile) * S + s) * Slot<FMT>::bytes(bpi).
+// The bytes are the planes' own; only their order changes, as the page's
+// build-time stream relayout does, so an item fetches its scales with one
+// bulk copy. One thread per (image, row).
+template <int FMT>
+__global__ void __launch_bounds__(256) k_pack_slots(WDev w, int bpi, uint8_t* __restrict__ out) {
+  const int tiles = (w.rows + kTile - 1) / kTile;
+  const int nbk = w.cols / 256;
+  const int S = nbk / bpi;
+  const uint32_t SB = Slot<FMT>::bytes(bpi);
+  const int64_t n = (int64_t)w.experts * tiles * S * kTile;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
+    const int r = (int)(i % kTile);
+    const int64_t img = i / kTile;
+    const int s = (int)(img % S);
+    const int64_t et = img / S;  // e * tiles + tile
+    const int tile = (int)(et % tiles);
+    const int64_t e = et / tiles;
+    const int row = tile * kTile + r;
+    const bool valid = row < w.rows;
+    const int64_t R = e * w.rows + row;
+    uint8_t* slot = out + img * SB;
+    if (FMT == FMT_KS) {
+      uint32_t* d32 = reinterpret_cast<uint32_t*>(slot);
+      for (int b = 0; b < bpi; b++) d32[r * bpi + b] = valid ? __ldg(w.scl + R * nbk + s * bpi + b) : 0u;
+      uint8_t* sb = slot + Slot<FMT>::b_off(bpi);
+      uint8_t* sc = slot + Slot<FMT>::c_off(bpi);
+      for (int b = 0; b < 4; b++) {
+        const bool in = valid && b < bpi;
+        sb[4 * r + b] = in ? __ldg(w.sch + R * nbk + s * bpi + b) : (uint8_t)0;
+        sc[4 * r + b] = in ? __ldg(reinterpret_cast<const uint8_t*>(w.sex) + R * nbk + s * bpi + b) : (uint8_t)0;
+      }
+      reinterpret_cast<uint16_t*>(slot + Slot<FMT>::dv_off(bpi))[r] = valid ? __ldg(w.dv + R) : (uint16_t)0;
+    } else {
+      uint32_t* d32 = reinterpret_cast<uint32_t*>(slot);
+      for (int b = 0; b < 2 * bpi; b++) d32[r * 2 * bpi + b] = valid ? __ldg(w.scl + R * 2 * nbk + 2 * s * bpi + b) : 0u;
+      uint16_t* sb = reinterpret_cast<uint16_t*>(slot + Slot<FMT>::b_off(bpi));
+      uint16_t* sc = reinterpret_cast<uint16_t*>(slot + Slot<FMT>::c_off(bpi));
+      for (int b = 0; b < bpi; b++) {
+        sb[r * bpi + b] = valid ? __ldg(reinterpret_cast<const uint16_t*>(w.sex) + R * nbk + s * bpi + b) : (uint16_t)0;
+        sc[r * bpi + b] = valid ? __ldg(w.dv + R * nbk + s * bpi + b) : (uint16_t)0;
+      }
+    }
+  }
 }
 
 // ================================================================== host
@@ -1627,6 +1699,23 @@ int launch_switch_decode(const WDev& w, int fmt, const Values& V, const uint16_t
   IQK_SW(FMT_KS, 1) IQK_SW(FMT_KS, 2) IQK_SW(FMT_K, 1) IQK_SW(FMT_K, 2)
 #undef IQK_SW
   return -3;
+}
+
+size_t slots_bytes(const WDev& w, int fmt) {
+  const int bpi = item_blocks(w.cols);
+  const int64_t S = (w.cols / 256) / bpi;
+  const int64_t tiles = (w.rows + kTile - 1) / kTile;
+  const uint32_t sb = fmt == FMT_KS ? Slot<FMT_KS>::bytes(bpi) : Slot<FMT_K>::bytes(bpi);
+  return (size_t)((int64_t)w.experts * tiles * S * sb);
+}
+
+int launch_pack_slots(const WDev& w, int fmt, uint8_t* out, cudaStream_t st, int num_sms) {
+  const int bpi = item_blocks(w.cols);
+  const int64_t n = (int64_t)w.experts * ((w.rows + kTile - 1) / kTile) * ((w.cols / 256) / bpi) * kTile;
+  const int64_t blocks = std::max<int64_t>(1, std::min<int64_t>((n + 255) / 256, (int64_t)num_sms * 8));
+  if (fmt == FMT_KS) k_pack_slots<FMT_KS><<<(unsigned)blocks, 256, 0, st>>>(w, bpi, out);
+  else k_pack_slots<FMT_K><<<(unsigned)blocks, 256, 0, st>>>(w, bpi, out);
+  return cudaGetLastError() == cudaSuccess ? 0 : -4;
 }
 
 int launch_floor(const WDev& w, int fmt, const int32_t* experts, int n, uint32_t* out, cudaStream_t st,

@@ -101,6 +101,9 @@ size_t switch_gemm_ws(int T, int topk, int experts, int rows, int cols);
 int launch_switch_gemm(const WDev& w, int fmt, const Values& V, const uint16_t* x, int T, const int32_t* ids,
                        int topk, float* y, char* ws, cudaStream_t st, int num_sms);
 
+// Scale-slot images of w (iqk_pack_slots): their size, and the packing kernel.
+size_t slots_bytes(const WDev& w, int fmt);
+int launch_pack_slots(const WDev& w, int fmt, uint8_t* out, cudaStream_t st, int num_sms);
 int launch_floor(const WDev& w, int fmt, const int32_t* experts, int n, uint32_t* out, cudaStream_t st,
                  int num_sms);
 // The floor's timeout flag (cleared by every floor call), after syncing `st`.

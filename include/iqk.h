@@ -94,13 +94,20 @@ typedef struct {
   const uint8_t* sch;   /* IQ2_KS [E][rows][cols/256]; must be NULL for IQ2_K */
   const void* sex;      /* IQ2_KS uint8 [E][rows][cols/256]; IQ2_K uint16 [E][rows][cols/256] */
   const uint16_t* dv;   /* IQ2_KS [E][rows]; IQ2_K [E][rows][cols/256] */
+  /* Optional (NULL when unused): the scale-slot images of these planes,
+   * written by iqk_pack_slots, 16-byte aligned. When set, the decode paths
+   * (iqk_gemv, iqk_gemv_static, iqk_moe_decode, iqk_moe_decode_shard, the
+   * decode kernel of iqk_switch_linear, iqk_floor) fetch each work item's
+   * scales with one bulk copy instead of per-lane copies from the planes.
+   * The images must have been packed from these same planes. */
+  const uint8_t* slots;
 } iqk_weights;
 
 /* Human-readable text of a status code (static storage). */
 const char* iqk_strerror(int status);
 /* Text of the last CUDA error seen by this library in this thread ("" if none). */
 const char* iqk_last_cuda_error(void);
-/* Library ABI version: 1. */
+/* Library ABI version: 2 (iqk_weights gained `slots`). */
 int iqk_version(void);
 
 /*
@@ -108,6 +115,27 @@ int iqk_version(void);
  * Page: "IQ2_KS rows cost 2 + 70*n/256 bytes, IQ2_K rows cost 76*n/256 bytes".
  */
 int64_t iqk_row_bytes(int32_t fmt, int32_t cols);
+
+/*
+ * Scale-slot images. Page section "Format" (and its note that each stream is
+ * rearranged at build time so that values consumed together are contiguous,
+ * changing no reconstructed value and no stored byte): the decode kernels
+ * take a weight tensor in items of 16 rows x one reduction slice (a fixed
+ * number of 256-weight blocks per row, set by cols), and an item needs the
+ * slice's bytes of scl, sch and sex and the rows' dv. iqk_pack_slots copies
+ * those bytes, for every (expert, 16-row tile, slice), into one contiguous
+ * 16-byte-aligned image, zero past the last row. Only the order of the
+ * bytes changes.
+ *
+ * iqk_slots_bytes: bytes of the images of all experts of w (0 if w is
+ *   invalid; its `slots` field is ignored).
+ * iqk_pack_slots: writes them to `out` (device, 16-byte aligned, at least
+ *   iqk_slots_bytes(w) bytes, owned by the caller) on `stream`; IQK_EINVAL
+ *   or IQK_EWORKSPACE (out too small or misaligned) before any launch.
+ *   Once the copy is complete on the stream, set w.slots = out.
+ */
+size_t iqk_slots_bytes(const iqk_weights* w);
+int iqk_pack_slots(const iqk_weights* w, uint8_t* out, size_t out_bytes, void* stream);
 
 /*
  * iqk_dequant -- reconstruct expert `expert` of `w` to float32, bit-exact.

@@ -30,15 +30,37 @@ def test_library_exports_every_declared_symbol():
 
 def test_row_bytes_and_version():
     L = B.lib()
-    assert L.iqk_version() == 1
+    assert L.iqk_version() == 2
     assert L.iqk_row_bytes(0, 4096) == 2 + 70 * 4096 // 256
     assert L.iqk_row_bytes(1, 2048) == 76 * 2048 // 256
     assert L.iqk_row_bytes(0, 100) == -1
     assert L.iqk_row_bytes(7, 256) == -1
 
 
-def _w(fmt=0, experts=1, rows=16, cols=256, sch=True):
-    return B.IqkWeights(fmt, experts, rows, cols, 4096, 4096, 4096 if sch else None, 4096, 4096)
+def _w(fmt=0, experts=1, rows=16, cols=256, sch=True, slots=None):
+    return B.IqkWeights(fmt, experts, rows, cols, 4096, 4096, 4096 if sch else None, 4096, 4096, slots)
+
+
+def test_slot_image_sizes_and_checks():
+    """One image per (expert, 16-row tile, slice) of the decode kernels'
+    slice width: IQ2_KS 64*bpi + 160 bytes, IQ2_K 192*bpi bytes, with bpi
+    4 blocks at 4096 columns and 2 at 2048 (4 slices per row either way)."""
+    L = B.lib()
+    w = _w(fmt=0, experts=2, rows=2048, cols=4096)
+    assert L.iqk_slots_bytes(ctypes.byref(w)) == 2 * 128 * 4 * (64 * 4 + 160)
+    w = _w(fmt=1, experts=1, rows=4096, cols=2048, sch=False)
+    assert L.iqk_slots_bytes(ctypes.byref(w)) == 256 * 4 * (192 * 2)
+    w = _w(fmt=0, experts=3, rows=20, cols=512)  # ragged last tile; 2 blocks per row, bpi 2, one slice
+    assert L.iqk_slots_bytes(ctypes.byref(w)) == 3 * 2 * 1 * (64 * 2 + 160)
+    assert L.iqk_slots_bytes(ctypes.byref(_w(cols=100))) == 0
+    w = _w(fmt=0, experts=1, rows=16, cols=256)
+    n = L.iqk_slots_bytes(ctypes.byref(w))
+    assert L.iqk_pack_slots(ctypes.byref(w), 4096 + 8, n, None) == B.IQK_EWORKSPACE  # misaligned
+    assert L.iqk_pack_slots(ctypes.byref(w), 4096, n - 16, None) == B.IQK_EWORKSPACE  # too small
+    assert L.iqk_pack_slots(ctypes.byref(w), None, n, None) == B.IQK_EWORKSPACE
+    v = np.zeros(8, np.float32)
+    w = _w(slots=4096 + 4)  # images must be 16-byte aligned
+    assert L.iqk_dequant(ctypes.byref(w), 0, v.ctypes.data, 4096, None) == B.IQK_EINVAL
 
 
 def test_host_validation_rejects_before_any_launch():
