@@ -484,6 +484,7 @@ struct UnitArgs {
   int32_t* cnt;
   float* part;
   int32_t* status;
+  int32_t* ready;  // routed decode: per run, gate/up tile groups of h written (gate/up adds, down polls); or null
   int bpi;       // 256-weight blocks per item
   int splits;    // items per tile and matrix (blocks per row / bpi)
   int async_sc;  // scale slices by cp.async (blocks per row a multiple of four)
@@ -505,6 +506,18 @@ __device__ __forceinline__ void cp_async8(void* dst, const void* src) {
 }
 __device__ __forceinline__ void cp_async16(void* dst, const void* src) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait_group() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+// Wait until at most `pending` of this thread's cp.async groups are still in flight.
+__device__ __forceinline__ void cp_async_wait_upto(int pending) {
+  if (pending <= 0) cp_async_wait_group<0>();
+  else if (pending == 1) cp_async_wait_group<1>();
+  else if (pending == 2) cp_async_wait_group<2>();
+  else cp_async_wait_group<3>();
 }
 // The mbarrier's current phase also waits for this thread's earlier cp.async copies.
 __device__ __forceinline__ void cp_async_arrive(uint64_t* bar) {
@@ -911,8 +924,18 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, kDecodeMinBlocks(NT)) k_til
     if (wid == 0) mbar_init(never_bar, 1);
     fence_mbar_init();
   }
+  // Routed decode with per-run readiness (A.ready): the gate/up kernel adds
+  // one to a run's counter after each of the run's tile groups of h, and the
+  // down kernel, which has no dependency wait before its items, copies a
+  // run's h once the run's counter is complete; it waits for the gate/up
+  // kernel only before it writes y. The prep kernel zeroes the counters, and
+  // the gate/up kernel lets the down kernel launch only after its own
+  // dependency wait has seen the prep kernel complete, so the down kernel
+  // never reads a counter of an earlier call.
+  const bool publish = MODE == MODE_GATEUP && A.ready != nullptr;
+  const bool hready = MODE == MODE_DOWN && BSM && A.ready != nullptr;
   if (A.first) griddep_wait();
-  griddep_launch();
+  if (!publish) griddep_launch();
   // the call's inputs first (ids, routing weights, x), then the tables while they arrive
   const int my_id = (int)threadIdx.x < npairs ? __ldcg(A.ids + threadIdx.x) : 0;
   const float my_p = (MODE == MODE_DOWN && (int)threadIdx.x < npairs) ? __ldcg(A.p + threadIdx.x) : 0.f;
@@ -1001,7 +1024,10 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, kDecodeMinBlocks(NT)) k_til
     }
   };
   for (int q = 0; q < kStages; q++) issue(q);
-  if (!A.first) griddep_wait();  // from here on: what the call's preceding kernels wrote, and the outputs
+  // from here on: what the call's preceding kernels wrote, and the outputs
+  // (the down kernel with per-run readiness: h through the run counters)
+  if (!A.first && !hready) griddep_wait();
+  if (publish) griddep_launch();
   // The first kernel resets the call's status word (and records ids outside
   // [0, E)). Every other write to it is a timeout bit, set at least one wait
   // bound after this kernel's CTAs have passed their dependency wait, so
@@ -1010,7 +1036,7 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, kDecodeMinBlocks(NT)) k_til
     *reinterpret_cast<volatile int32_t*>(A.status) = (A.check_ids && rt.scalars[1] < npairs) ? 1 : 0;
   if constexpr (BSM) {  // activation rows, slot-transposed and padded, once per CTA
     const int gpr = K / 16;
-    for (int k = 0;; k++) {
+    for (int k = 0; !hready; k++) {
       const int gi = threadIdx.x + k * blockDim.x;
       if (gi >= act_groups) break;
       const int r = gi / gpr, c0 = (gi - r * gpr) * 16;
@@ -1046,6 +1072,7 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, kDecodeMinBlocks(NT)) k_til
     }
   }
   if (MODE == MODE_DOWN && D == 0) {  // no pair on these experts: the block output is zero
+    if (hready) griddep_wait();
     for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < A.T * rows; i += gridDim.x * blockDim.x) {
       if (A.yf) A.yf[i] = 0.f;
       else A.out16[i] = 0;
@@ -1061,6 +1088,51 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, kDecodeMinBlocks(NT)) k_til
     failed = true;  // keep taking part in the CTA barriers; stop loading
     if (lane == 0) atomicOr(A.status, 2);
   }
+  // Per-run readiness (down kernel): in the first round each warp copies,
+  // for each of its items (run u, slice s), that slice of the run's h rows
+  // into shared memory itself (cp.async through L2, one commit group per
+  // item, in item order) once the run's counter is complete; no other warp
+  // touches that slice, and later rounds reuse it. Lane j polls the counter
+  // of the warp's j-th pending item with a relaxed load, issued before the
+  // current item's arithmetic and read after it; an acquire fence follows a
+  // complete counter before any copy.
+  const int h_target = (K + kTile - 1) / kTile;  // gate/up tile groups per run
+  int h_issued = 0;
+  auto stage_h = [&](int k) {
+    int u, mat, tile, s;
+    item_at(k, u, mat, tile, s);
+    const int p0 = rt.ustart[u], ncols = rt.ustart[u + 1] - p0;
+    const int gps = bpi * 16;  // 16-element groups per slice row
+    for (int i = lane; i < ncols * gps; i += 32) {
+      const int c = i / gps;
+      const int c0 = (s * gps + (i - c * gps)) * 16;
+      const int pair = rt.sorted[p0 + c];
+      uint16_t* dst = act_s + (size_t)pair * KP + (c0 >> 6) * 80 + (c0 & 63);
+      const uint16_t* src = A.act + (size_t)pair * K + c0;
+      cp_async16(dst, src);
+      cp_async16(dst + 8, src + 8);
+    }
+    cp_async_commit();
+    h_issued = k + 1;
+  };
+  // relaxed poll of the counter of pending item h_issued + lane (-1: none)
+  auto poll = [&]() -> int32_t {
+    const int j = h_issued + lane;
+    if (j >= cnt_w) return -1;
+    int u, mat, tile, s;
+    item_at(j, u, mat, tile, s);
+    return ld_relaxed_s32(A.ready + u);
+  };
+  // stage the pending items whose runs are complete, in order, from polled values
+  auto stage_ready = [&](int32_t seen) {
+    const unsigned m = __ballot_sync(0xffffffffu, seen >= h_target);
+    const int n = ~m ? __ffs(~m) - 1 : 32;  // consecutive complete runs from h_issued
+    if (n == 0) return;
+    fence_acq_rel_gpu();
+    __syncwarp();
+    const int stop = min(h_issued + n, cnt_w);
+    while (h_issued < stop) stage_h(h_issued);
+  };
   int consumed = 0;
   int q = 0;
   for (int r = 0; r < rounds; r++) {
@@ -1088,6 +1160,27 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, kDecodeMinBlocks(NT)) k_til
       for (int n = 0; n < NT; n++)
 #pragma unroll
         for (int qq = 0; qq < 4; qq++) acc[n][qq] = 0.f;
+      int32_t ahead = -1;  // the next pending item's counter, polled during this item
+      if (hready && r == 0) {
+        failed = __any_sync(0xffffffffu, failed);  // the polls below take the whole warp
+        if (!failed && h_issued <= k) {  // this item's slice is not staged: wait (bounded) for its run
+          const uint64_t t0 = globaltimer_ns();
+          for (;;) {
+            stage_ready(poll());
+            if (h_issued > k) break;
+            if (__any_sync(0xffffffffu, globaltimer_ns() - t0 >= A.wait_ns)) {
+              failed = true;
+              if (lane == 0) atomicOr(A.status, 2);
+              break;
+            }
+            __nanosleep(64);
+          }
+        }
+        cp_async_wait_upto(h_issued - (k + 1));  // this item's group (and those before it) have landed
+        __syncwarp();
+        if (!failed && h_issued < cnt_w) ahead = poll();
+      }
+      const bool polled = hready && r == 0 && !failed && h_issued < cnt_w;
       const int st = q % kStages;
       if (!failed && !mbar_wait_ns(&bar[st], (uint32_t)((q / kStages) & 1), A.wait_ns)) {
         failed = true;  // keep taking part in the CTA barriers; stop loading
@@ -1108,6 +1201,7 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, kDecodeMinBlocks(NT)) k_til
         __syncwarp();
         issue(q + kStages);  // refill the stage just consumed
       }
+      if (polled) stage_ready(ahead);  // later items whose runs completed meanwhile
       // add into this warp's slot: (mat, column, row) for gate/up, (column, row)
       // for switch (a warp's items in a group share one tile), (token, row) for down
       if (MODE != MODE_DOWN) {
@@ -1133,6 +1227,7 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, kDecodeMinBlocks(NT)) k_til
       __syncwarp();
     }
     __syncthreads();  // every warp's slot of this group is complete
+    if (hready) griddep_wait();  // y only after the gate/up kernel has completed
     const int tg = (int)blockIdx.x + r * (int)gridDim.x;
     if (MODE == MODE_GATEUP) {
       const int u = (int)A.div_tiles.div((uint32_t)tg);
@@ -1181,9 +1276,14 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, kDecodeMinBlocks(NT)) k_til
       }
     }
     __syncthreads();  // slots free for the next group
+    if (publish && threadIdx.x == 0) {  // one more tile group of this run is in h
+      __threadfence();
+      atomicAdd(A.ready + (int)A.div_tiles.div((uint32_t)tg), 1);
+    }
   }
   // let copies still in flight land before the CTA exits (only after a timeout)
   for (int qd = consumed; qd < issued; qd++) (void)mbar_wait_ns(&bar[qd % kStages], (uint32_t)((qd / kStages) & 1), kDrainWaitNs);
+  if (hready) cp_async_wait_group<0>();
 }
 
 // ------------------------------------------------------ scale-slot images
@@ -1566,6 +1666,8 @@ DecodeWs decode_ws(int T, int topk, int experts, int hidden, int inter) {
   o = align256(o + (size_t)T * hidden * 2);
   ws.hperm = o;
   o = align256(o + (size_t)npairs * inter * 2);
+  ws.ready = o;
+  o = align256(o + (size_t)npairs * 4);
   ws.total = o;
   return ws;
 }
@@ -1588,11 +1690,18 @@ static int decode_impl(const WDev& g, const WDev& u, const WDev& d, const Values
   const int pblocks = std::max(1, std::min(num_sms, (int)(((int64_t)T * (g.cols / 16) + 63) / 64)));
   // a shard skips the ids of other shards silently, so it checks none
   const bool shard = yf != nullptr;
-  // With x staged in shared memory there is nothing to transpose: the gate/up
-  // kernel is the call's first kernel and resets the status word itself.
-  if (!ar && launch_prep(pblocks, st, x, T, g.cols, xp, nullptr, 0, ids, shard ? 0 : npairs, g.experts, status))
+  // h rows in the down kernel's shared memory: it takes each run of pairs as
+  // soon as the run's h is complete (per-run counters, zeroed by the prep
+  // kernel). Otherwise, with x staged in shared memory there is nothing to
+  // prepare: the gate/up kernel is the call's first kernel and resets the
+  // status word itself.
+  const int hrows = act_rows_smem(NT, npairs, d.cols);
+  int32_t* ready = hrows ? reinterpret_cast<int32_t*>(ws + L.ready) : nullptr;
+  if ((!ar || ready) && launch_prep(ar ? 1 : pblocks, st, x, ar ? 0 : T, g.cols, xp, ready, ready ? npairs : 0, ids,
+                                    shard ? 0 : npairs, g.experts, status))
     return -4;
-  a.first = ar ? 1 : 0;
+  a.first = (ar && !ready) ? 1 : 0;
+  a.ready = ready;
   a.check_ids = shard ? 0 : 1;
   a.ebase = ebase;
   a.w0 = g;
@@ -1619,7 +1728,7 @@ static int decode_impl(const WDev& g, const WDev& u, const WDev& d, const Values
   b.act = hp;
   b.out16 = y;
   b.yf = yf;
-  b.act_rows = act_rows_smem(NT, npairs, d.cols);
+  b.act_rows = hrows;
   return b.act_rows ? launch_tiles<MODE_DOWN, FD, FD, NT, true>(md, md, b, L.c3.tiles, st, num_sms, true)
                     : launch_tiles<MODE_DOWN, FD, FD, NT, false>(md, md, b, L.c3.tiles, st, num_sms, true);
 }

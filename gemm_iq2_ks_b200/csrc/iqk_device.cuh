@@ -124,6 +124,16 @@ __device__ __forceinline__ bool mbar_wait_ns(uint64_t* bar, uint32_t parity, uin
   }
 }
 
+// Device-scope relaxed load (polling a counter another SM adds to), and the
+// acquire fence that, after such a load has seen a writer's fence + add,
+// orders this thread's later loads after the writer's earlier stores.
+__device__ __forceinline__ int32_t ld_relaxed_s32(const int32_t* p) {
+  int32_t v;
+  asm volatile("ld.relaxed.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ void fence_acq_rel_gpu() { asm volatile("fence.acq_rel.gpu;" ::: "memory"); }
+
 // Bound of the waits that let a warp's copies still in flight land after one
 // of its waits expired (the copies complete on their own; this only guards
 // against a wedged copy engine).

@@ -68,9 +68,10 @@ struct GemvWs {
 GemvWs gemv_ws(int T, int rows, int cols);
 
 // Workspace carve-up for iqk_moe_decode: status word, transposed x (read
-// through L1 when it does not fit shared memory), h.
+// through L1 when it does not fit shared memory), h, and one counter per run
+// of pairs (gate/up tile groups of h written so far).
 struct DecodeWs {
-  size_t status, xperm, hperm, total;
+  size_t status, xperm, hperm, ready, total;
   Chunking c2, c3;
 };
 DecodeWs decode_ws(int T, int topk, int experts, int hidden, int inter);
