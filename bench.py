@@ -824,7 +824,7 @@ def main():
         for case in S.MATRIX_CASES:
             details[case] = gemv_leg(torch, B, case, device, stream)
 
-    launches = 2 * K  # per call: the gate/up kernel (the call's first) and the down kernel
+    launches = 3 * K  # per call: the prep kernel (run counters), the gate/up kernel and the down kernel
     line = {
         "metric": METRIC, "value": us_per_token, "unit": "us/token", "n_gpus": world, "steps": K, "warmup": W,
         "ms_per_step": t / K * 1e3, "higher_is_better": False, "scaling": "weak", "vs_baseline": None,
@@ -834,7 +834,7 @@ def main():
                   (t / K * 1e6) / floor_us, "status_ok": floor_status == B.IQK_OK},
         "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                      "frac": gbs / peaks["hbm_gbs"], "traffic": DECODE_CALL_TRAFFIC,
-                     "kernel": "one decode call (gate/up+SwiGLU, then down+combine, PDL-chained)",
+                     "kernel": "one decode call (prep, gate/up+SwiGLU, down+combine, PDL-chained)",
                      "peak_source": peaks["source"] + " hbm_gbs (copy)"},
         "e2e": {"value": e2e_us, "unit": "us/token", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": launches,
