@@ -26,6 +26,7 @@ EXPORTS = (
     "iqk_moe_prefill", "iqk_moe_prefill_shard", "iqk_moe_combine", "iqk_moe_status",
     "iqk_route_workspace_bytes", "iqk_moe_route", "iqk_floor", "iqk_floor_status", "iqk_set_wait_limit_ns",
     "iqk_switch_linear_workspace_bytes", "iqk_switch_linear", "iqk_slots_bytes", "iqk_pack_slots",
+    "iqk_prefill_a_tile",
 )
 
 
@@ -90,6 +91,7 @@ def lib(build_if_missing: bool = True) -> ctypes.CDLL:
             "iqk_switch_linear": (ctypes.c_int, [W, vp, vp, i32, vp, i32, vp, i32, vp, sz, vp]),
             "iqk_slots_bytes": (sz, [W]),
             "iqk_pack_slots": (ctypes.c_int, [W, vp, sz, vp]),
+            "iqk_prefill_a_tile": (ctypes.c_int, [W, i32, i32, i32, vp, vp, vp]),
         }
         for name, (res, args) in sig.items():
             f = getattr(L, name)
@@ -197,6 +199,17 @@ def _empty(shape, dtype, device):
 
 def iqk_row_bytes(fmt: str, cols: int) -> int:
     return lib().iqk_row_bytes(FMT[fmt], cols)
+
+
+def iqk_prefill_a_tile(w: Weights, expert: int, row0: int, nrows: int, values, out=None, stream=None):
+    """The prefill producer's bf16 A operand of rows [row0, row0 + nrows) of
+    one expert, in k order ([nrows, cols] bf16)."""
+    torch = _torch()
+    out = _empty((nrows, w.cols), torch.bfloat16, w.qs.device) if out is None else out
+    v = _values(values)
+    _check(lib().iqk_prefill_a_tile(ctypes.byref(w.c), expert, row0, nrows, v.ctypes.data, out.data_ptr(),
+                                    _stream(stream)), "iqk_prefill_a_tile")
+    return out
 
 
 def iqk_dequant(w: Weights, expert: int, values, out=None, stream=None):

@@ -136,6 +136,17 @@ int iqk_pack_slots(const iqk_weights* w, uint8_t* out, size_t out_bytes, void* s
   return from_launch(launch_pack_slots(wd, w->fmt, out, (cudaStream_t)stream, sms));
 }
 
+int iqk_prefill_a_tile(const iqk_weights* w, int32_t expert, int32_t row0, int32_t nrows, const float* values,
+                       uint16_t* out, void* stream) {
+  WDev wd;
+  Values V;
+  int rc;
+  if ((rc = check_weights(w, &wd)) || (rc = check_values(values, &V))) return rc;
+  if (expert < 0 || expert >= wd.experts || row0 < 0 || nrows < 1 || (int64_t)row0 + nrows > wd.rows) return IQK_EINVAL;
+  if (!out || !aligned(out, 16)) return IQK_EINVAL;
+  return from_launch(launch_pf_a_tile(wd, w->fmt, expert, row0, nrows, V, out, (cudaStream_t)stream));
+}
+
 int iqk_dequant(const iqk_weights* w, int32_t expert, const float* values, float* out, void* stream) {
   WDev wd;
   Values V;

@@ -138,6 +138,9 @@ int launch_moe_prefill(const WDev& g, int fg, const WDev& u, int fu, const WDev&
                        const Values& V, const uint16_t* x, int T, const int32_t* ids, const float* p,
                        int topk, uint16_t* y, float* yf, int ebase, char* ws, cudaStream_t st, int num_sms);
 // y[t] = bf16_rn(sum over slots j in order of p[t][j] * rows[t * topk + j]).
+// The prefill producer's A operand of rows [row0, row0 + nrows) of one expert, in k order.
+int launch_pf_a_tile(const WDev& w, int fmt, int expert, int row0, int nrows, const Values& V, uint16_t* out,
+                     cudaStream_t st);
 int launch_combine(const float* rows, const float* p, int T, int topk, int H, uint16_t* y, cudaStream_t st,
                    int num_sms);
 

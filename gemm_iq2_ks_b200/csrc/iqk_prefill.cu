@@ -122,6 +122,27 @@ __device__ __forceinline__ uint2 table_words(const BlkSc<FMT>& s, int cc, int m,
   }
 }
 
+// The A operand of one row for one chunk of 64 weights (the 4 qs words of the
+// chunk, cc = chunk index inside its 256-block): 32 registers of bf16 pairs.
+// regs[8m + 2i] holds weights (16m + i, 16m + 4 + i) and regs[8m + 2i + 1]
+// holds (16m + 8 + i, 16m + 12 + i) of the chunk, the slot order in which
+// the token rows are transposed (the byte-permute lookup emits codes i,
+// 4 + i, 8 + i, 12 + i of a word together).
+template <int FMT>
+__device__ __forceinline__ void decode_chunk(const BlkSc<FMT>& sc, int cc, const uint32_t (&qv)[4], const uint2* lut,
+                                             const Values& V, uint32_t (&regs)[32]) {
+#pragma unroll
+  for (int m = 0; m < 4; m++) {
+    const uint2 tw = table_words<FMT>(sc, cc, m, lut, V);
+#pragma unroll
+    for (int i = 0; i < 4; i++) {
+      const Pair2 pr = lookup_slot(qv[m], i, tw.x, tw.y);
+      regs[8 * m + 2 * i] = pr.lo;
+      regs[8 * m + 2 * i + 1] = pr.hi;
+    }
+  }
+}
+
 __device__ __forceinline__ bool pf_wait(uint64_t* bar, uint32_t par, volatile uint32_t* abort_flag, int32_t* status) {
   for (uint32_t i = 0; i < (1u << 24); i++) {
     if (mbar_try_wait(bar, par)) return true;
@@ -164,16 +185,7 @@ __device__ __forceinline__ bool pf_produce(const WDev& W, int64_t grow, int nch,
     const uint4 qw = *reinterpret_cast<const uint4*>(qbuf + (size_t)s * (PF_Q_BYTES / 4) + (tile ? 128 * 16 : 0) +
                                                      r * 16 + 4 * ((c & 3) ^ ((r >> 1) & 3)));
     const uint32_t qv[4] = {qw.x, qw.y, qw.z, qw.w};
-#pragma unroll
-    for (int m = 0; m < 4; m++) {
-      const uint2 tw = table_words<FMT>(sc, c & 3, m, lut, V);
-#pragma unroll
-      for (int i = 0; i < 4; i++) {
-        const Pair2 pr = lookup_slot(qv[m], i, tw.x, tw.y);
-        regs[8 * m + 2 * i] = pr.lo;
-        regs[8 * m + 2 * i + 1] = pr.hi;
-      }
-    }
+    decode_chunk<FMT>(sc, c & 3, qv, lut, V, regs);
     if ((c & 3) == 3) {  // the qs stage has been read in full
       __syncwarp();
       if (lane == 0) mbar_arrive(&qs_empty[s]);
@@ -730,6 +742,51 @@ int launch_switch_gemm(const WDev& w, int fmt, const Values& V, const uint16_t* 
     const int blocks = (int)std::min<int64_t>((n + 255) / 256, (int64_t)num_sms * 16);
     k_sw_scatter<<<std::max(blocks, 1), 256, 0, st>>>(outp, inv, P, R, y);
   }
+  return cudaGetLastError() == cudaSuccess ? 0 : -4;
+}
+
+// ------------------------------------------------------ A-operand inspection
+// The producer's A operand of rows [row0, row0 + nrows) of expert e, every
+// column, written to global memory in k order (out[r][k], bf16 bits): the
+// same block scales, tables and chunk decode (decode_chunk) the producers of
+// k_pf_gemm store into tensor memory, with the slot order undone. IQ2_K:
+// bf16_rn((d * float(idx)) * value); IQ2_KS: bf16_rn(float(idx) * value), its
+// row scale d being applied to the accumulator in the epilogue. One thread
+// per row.
+template <int FMT>
+__global__ void __launch_bounds__(128) k_pf_a_tile(WDev w, int expert, int row0, int nrows, Values V,
+                                                   uint16_t* __restrict__ out) {
+  __shared__ uint2 lut[64];
+  build_lut_pf<FMT>(lut, V);
+  __syncthreads();
+  const int r = blockIdx.x * blockDim.x + threadIdx.x;
+  if (r >= nrows) return;
+  const int64_t grow = (int64_t)expert * w.rows + row0 + r;
+  const int wpr = w.cols / 16;
+  BlkSc<FMT> sc = load_blk<FMT>(w, grow, 0);
+  for (int c = 0; c < w.cols / 64; c++) {
+    if ((c & 3) == 0) sc = load_blk<FMT>(w, grow, c >> 2);
+    uint32_t qv[4];
+    for (int m = 0; m < 4; m++) qv[m] = __ldg(w.qs + grow * wpr + 4 * c + m);
+    uint32_t regs[32];
+    decode_chunk<FMT>(sc, c & 3, qv, lut, V, regs);
+    uint16_t* o = out + (size_t)r * w.cols + 64 * c;
+    for (int m = 0; m < 4; m++)
+      for (int i = 0; i < 4; i++) {
+        const uint32_t lo = regs[8 * m + 2 * i], hi = regs[8 * m + 2 * i + 1];
+        o[16 * m + i] = (uint16_t)(lo & 0xffffu);
+        o[16 * m + 4 + i] = (uint16_t)(lo >> 16);
+        o[16 * m + 8 + i] = (uint16_t)(hi & 0xffffu);
+        o[16 * m + 12 + i] = (uint16_t)(hi >> 16);
+      }
+  }
+}
+
+int launch_pf_a_tile(const WDev& w, int fmt, int expert, int row0, int nrows, const Values& V, uint16_t* out,
+                     cudaStream_t st) {
+  const int blocks = (nrows + 127) / 128;
+  if (fmt == FMT_KS) k_pf_a_tile<FMT_KS><<<blocks, 128, 0, st>>>(w, expert, row0, nrows, V, out);
+  else k_pf_a_tile<FMT_K><<<blocks, 128, 0, st>>>(w, expert, row0, nrows, V, out);
   return cudaGetLastError() == cudaSuccess ? 0 : -4;
 }
 

@@ -138,6 +138,24 @@ size_t iqk_slots_bytes(const iqk_weights* w);
 int iqk_pack_slots(const iqk_weights* w, uint8_t* out, size_t out_bytes, void* stream);
 
 /*
+ * iqk_prefill_a_tile -- inspection: the bf16 A operand that iqk_moe_prefill's
+ * producer warps decode into tensor memory (page sections "Format" and
+ * "Surface": weights dequantized once per expert into the grouped matmul's
+ * operand), for rows [row0, row0 + nrows) of expert `expert` of w, all
+ * columns, written in k order to out (device, [nrows][cols] bf16 bits).
+ *   IQ2_K:  out = bf16_rn((d * float(scale_index)) * values[4*alphabet + code])
+ *           (d changes every 256 weights, so it is folded in per weight);
+ *   IQ2_KS: out = bf16_rn(float(scale_index) * values[4*alphabet + code]);
+ *           the row scale d is applied to the float32 accumulator in the
+ *           GEMM epilogue instead.
+ * The decode is the producers' own (same tables and per-chunk routine);
+ * only the store target differs. IQK_EINVAL before any launch for bad
+ * arguments (rows out of range, nrows < 1, out NULL or not 16-byte aligned).
+ */
+int iqk_prefill_a_tile(const iqk_weights* w, int32_t expert, int32_t row0, int32_t nrows,
+                       const float* values /* host [8] */, uint16_t* out, void* stream);
+
+/*
  * iqk_dequant -- reconstruct expert `expert` of `w` to float32, bit-exact.
  * Defines: the reconstruction formula above (page section "Format").
  * out:    device float32 [rows][cols], row-major, written completely.

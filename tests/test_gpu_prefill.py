@@ -123,3 +123,31 @@ def test_prefill_full_all_tokens(B, full_prefill, parity_report):
     ref = O.moe(gate, up, down, values, x, ids, p)
     out = check_block(y, h, ref, down, values, ids, p, "prefill 2048 tokens, all")
     parity_report("prefill 2048, all tokens", flat_stats(out))
+
+
+@pytest.mark.parametrize("fmt,rows,cols,table", [("iq2_k", 200, 512, "f16"), ("iq2_ks", 200, 512, "int"),
+                                                 ("iq2_k", 160, 4096, "int"), ("iq2_ks", 272, 2048, "f16")])
+def test_producer_tile_is_the_rounded_weight(B, fmt, rows, cols, table):
+    """The prefill A operand (what the producer warps store into tensor
+    memory) is the oracle's float32 weight rounded to bf16, bit for bit.
+    IQ2_K: bf16_rn((d*idx)*value). IQ2_KS: bf16_rn(idx*value), the row
+    scale d going to the epilogue; pinned with d = 1 (fp16 0x3C00), where the
+    oracle's weight is exactly float(idx)*value. Rows from an offset to a
+    ragged end; a row of zero scale (IQ2_K) for the signs of zero."""
+    rng = S.rng_for(700 + rows)
+    host = S.random_streams(rng, fmt, 3, rows, cols)
+    if fmt == "iq2_ks":
+        host.dv[...] = 0x3C00
+    else:
+        host.dv[1, 7, :] = 0  # every weight of row 7 of expert 1 is +-0
+    values = S.value_table(table, 11)
+    w = B.Weights.from_host(host)
+    e, row0 = 1, 5
+    nrows = rows - row0
+    a = B.iqk_prefill_a_tile(w, e, row0, nrows, values)
+    torch.cuda.synchronize()
+    got = a.view(torch.int16).cpu().numpy().view(np.uint16)
+    ref = O.bf16_round(O.dequant_expert(host, e, values)[row0:row0 + nrows])
+    assert got.shape == ref.shape
+    bad = np.argwhere(got != ref)
+    assert bad.size == 0, f"{len(bad)} mismatches, first at {bad[:3].tolist()}"
