@@ -51,15 +51,17 @@
  *     are staged into shared memory by TMA and bulk copies); IQK_EINVAL if not.
  *   - Consecutive calls overlap their launches: the decode, GEMV,
  *     switch-linear and floor paths launch their kernels as programmatic
- *     dependents of whatever precedes them on the stream, and each kernel
- *     lets its dependents launch as soon as it starts. Every kernel of this
- *     library waits (griddepcontrol.wait) for its predecessor before it reads
- *     or writes any memory other than its launch parameters, so stream order
- *     holds as usual: a call may read the previous call's output. A caller's
- *     own kernel launched with programmatic stream serialization right after
- *     one of these calls must likewise wait before touching the call's
- *     outputs; kernels launched without that attribute, copies and events
- *     see the call complete, as always.
+ *     dependents of whatever precedes them on the stream. The first kernel
+ *     of every call waits (griddepcontrol.wait) for all earlier work on the
+ *     stream before it touches any memory, and only then lets the call's
+ *     other kernels launch; those read the call's inputs and the weights as
+ *     soon as they start, and write outputs only after their own wait. So
+ *     stream order holds as usual: a call may read the previous call's
+ *     output, and weights written by earlier work on the stream are seen. A
+ *     caller's own kernel launched with programmatic stream serialization
+ *     right after one of these calls must likewise wait before touching the
+ *     call's outputs; kernels launched without that attribute, copies and
+ *     events see the call complete, as always.
  */
 #ifndef IQK_H_
 #define IQK_H_
