@@ -1093,9 +1093,11 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, kDecodeMinBlocks(NT)) k_til
   // into shared memory itself (cp.async through L2, one commit group per
   // item, in item order) once the run's counter is complete; no other warp
   // touches that slice, and later rounds reuse it. Lane j polls the counter
-  // of the warp's j-th pending item with a relaxed load, issued before the
-  // current item's arithmetic and read after it; an acquire fence follows a
-  // complete counter before any copy.
+  // of the warp's j-th pending item: with an acquire load where the warp
+  // waits for an item, and with a relaxed load issued before the current
+  // item's arithmetic and read after it (look-ahead), in which case the
+  // lanes that saw a complete counter read it again with acquire before any
+  // copy. A warp barrier passes the acquiring lanes' ordering to the others.
   const int h_target = (K + kTile - 1) / kTile;  // gate/up tile groups per run
   int h_issued = 0;
   auto stage_h = [&](int k) {
@@ -1115,20 +1117,24 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, kDecodeMinBlocks(NT)) k_til
     cp_async_commit();
     h_issued = k + 1;
   };
-  // relaxed poll of the counter of pending item h_issued + lane (-1: none)
-  auto poll = [&]() -> int32_t {
+  // the counter of pending item h_issued + lane (-1: none)
+  auto poll = [&](bool acquire) -> int32_t {
     const int j = h_issued + lane;
     if (j >= cnt_w) return -1;
     int u, mat, tile, s;
     item_at(j, u, mat, tile, s);
-    return ld_relaxed_s32(A.ready + u);
+    return acquire ? ld_acquire_s32(A.ready + u) : ld_relaxed_s32(A.ready + u);
   };
   // stage the pending items whose runs are complete, in order, from polled values
-  auto stage_ready = [&](int32_t seen) {
+  auto stage_ready = [&](int32_t seen, bool acquired) {
     const unsigned m = __ballot_sync(0xffffffffu, seen >= h_target);
     const int n = ~m ? __ffs(~m) - 1 : 32;  // consecutive complete runs from h_issued
     if (n == 0) return;
-    fence_acq_rel_gpu();
+    if (!acquired && lane < n) {  // counters only grow: this read is complete too, now with acquire
+      int u, mat, tile, s;
+      item_at(h_issued + lane, u, mat, tile, s);
+      (void)ld_acquire_s32(A.ready + u);
+    }
     __syncwarp();
     const int stop = min(h_issued + n, cnt_w);
     while (h_issued < stop) stage_h(h_issued);
@@ -1166,7 +1172,7 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, kDecodeMinBlocks(NT)) k_til
         if (!failed && h_issued <= k) {  // this item's slice is not staged: wait (bounded) for its run
           const uint64_t t0 = globaltimer_ns();
           for (;;) {
-            stage_ready(poll());
+            stage_ready(poll(true), true);
             if (h_issued > k) break;
             if (__any_sync(0xffffffffu, globaltimer_ns() - t0 >= A.wait_ns)) {
               failed = true;
@@ -1178,7 +1184,7 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, kDecodeMinBlocks(NT)) k_til
         }
         cp_async_wait_upto(h_issued - (k + 1));  // this item's group (and those before it) have landed
         __syncwarp();
-        if (!failed && h_issued < cnt_w) ahead = poll();
+        if (!failed && h_issued < cnt_w) ahead = poll(false);
       }
       const bool polled = hready && r == 0 && !failed && h_issued < cnt_w;
       const int st = q % kStages;
@@ -1201,7 +1207,7 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, kDecodeMinBlocks(NT)) k_til
         __syncwarp();
         issue(q + kStages);  // refill the stage just consumed
       }
-      if (polled) stage_ready(ahead);  // later items whose runs completed meanwhile
+      if (polled) stage_ready(ahead, false);  // later items whose runs completed meanwhile
       // add into this warp's slot: (mat, column, row) for gate/up, (column, row)
       // for switch (a warp's items in a group share one tile), (token, row) for down
       if (MODE != MODE_DOWN) {

@@ -133,6 +133,13 @@ __device__ __forceinline__ int32_t ld_relaxed_s32(const int32_t* p) {
   return v;
 }
 __device__ __forceinline__ void fence_acq_rel_gpu() { asm volatile("fence.acq_rel.gpu;" ::: "memory"); }
+// Device-scope acquire load: once it reads a value a writer's fence + add
+// produced, this thread's later loads see what the writer stored before.
+__device__ __forceinline__ int32_t ld_acquire_s32(const int32_t* p) {
+  int32_t v;
+  asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
 
 // Bound of the waits that let a warp's copies still in flight land after one
 // of its waits expired (the copies complete on their own; this only guards
