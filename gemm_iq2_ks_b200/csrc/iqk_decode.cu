@@ -1282,9 +1282,10 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, kDecodeMinBlocks(NT)) k_til
       }
     }
     __syncthreads();  // slots free for the next group
-    if (publish && threadIdx.x == 0) {  // one more tile group of this run is in h
-      __threadfence();
-      atomicAdd(A.ready + (int)A.div_tiles.div((uint32_t)tg), 1);
+    if (publish && threadIdx.x == 0) {  // one more tile group of this run is in h (the barrier above
+      // orders every thread's h stores before this release)
+      asm volatile("red.release.gpu.global.add.s32 [%0], 1;" ::"l"(A.ready + (int)A.div_tiles.div((uint32_t)tg))
+                   : "memory");
     }
   }
   // let copies still in flight land before the CTA exits (only after a timeout)
