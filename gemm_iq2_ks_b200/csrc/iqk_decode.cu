@@ -1025,9 +1025,12 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, kDecodeMinBlocks(NT)) k_til
   };
   for (int q = 0; q < kStages; q++) issue(q);
   // from here on: what the call's preceding kernels wrote, and the outputs
-  // (the down kernel with per-run readiness: h through the run counters)
-  if (!A.first && !hready) griddep_wait();
-  if (publish) griddep_launch();
+  // (the down kernel with per-run readiness: h through the run counters).
+  // A gate/up kernel that publishes runs and stages x itself needs nothing
+  // the prep kernel writes before its first counter add: it waits there.
+  const bool late_wait = publish && BSM;
+  if (!A.first && !hready && !late_wait) griddep_wait();
+  if (publish && !late_wait) griddep_launch();
   // The first kernel resets the call's status word (and records ids outside
   // [0, E)). Every other write to it is a timeout bit, set at least one wait
   // bound after this kernel's CTAs have passed their dependency wait, so
@@ -1282,6 +1285,10 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, kDecodeMinBlocks(NT)) k_til
       }
     }
     __syncthreads();  // slots free for the next group
+    if (late_wait && r == 0) {  // the prep kernel has zeroed the run counters: the down kernel may start
+      griddep_wait();
+      griddep_launch();
+    }
     if (publish && threadIdx.x == 0) {  // one more tile group of this run is in h (the barrier above
       // orders every thread's h stores before this release)
       asm volatile("red.release.gpu.global.add.s32 [%0], 1;" ::"l"(A.ready + (int)A.div_tiles.div((uint32_t)tg))
