@@ -467,5 +467,5 @@ extern "C" int iqk_gemv_static(const iqk_weights* w, int32_t expert, const float
   const int sms = num_sms();
   if (sms < 0) return cuda_fail(cudaGetLastError());
   return from_launch(
-      launch_gemv(wd, w->fmt, expert, V, x, T, y, static_cast<char*>(scratch), (cudaStream_t)stream, sms));
+      launch_gemv(wd, w->fmt, expert, V, x, T, y, static_cast<char*>(scratch), (cudaStream_t)stream, sms, false));
 }

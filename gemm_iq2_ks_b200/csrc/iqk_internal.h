@@ -80,8 +80,10 @@ DecodeWs decode_ws(int T, int topk, int experts, int hidden, int inter);
 // box [16 rows][nb*16 words]. Returns 0 on success.
 int make_qs_map(CUtensorMap* map, const WDev& w, int nb);
 
+// tiles_ok: a tall matrix with few tokens may take the tile kernel (one
+// launch); otherwise the prep and stream kernels.
 int launch_gemv(const WDev& w, int fmt, int expert, const Values& V, const uint16_t* x, int T,
-                float* y, char* ws, cudaStream_t st, int num_sms);
+                float* y, char* ws, cudaStream_t st, int num_sms, bool tiles_ok = true);
 
 // yf non-null: an expert-parallel shard holding experts [ebase, ebase + E)
 // writes its float32 partial to yf (y unused) and skips other ids silently.
