@@ -663,7 +663,7 @@ def main():
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work for cpu_baseline")
     ap.add_argument("--no-details", action="store_true")
     ap.add_argument("--no-price", action="store_true", help="skip the pricing table (kernels vs own floors)")
-    ap.add_argument("--profile", choices=["decode", "prefill", "dequant"], default=None,
+    ap.add_argument("--profile", choices=["decode", "prefill", "dequant", "gemv"], default=None,
                     help="plain launches without graphs or reporting (for ncu captures)")
     ap.add_argument("--experts", type=int, default=S.EXPERTS,
                     help="experts resident in --profile mode (fewer keeps ncu captures small)")
@@ -708,6 +708,18 @@ def main():
         with torch.cuda.stream(stream):
             for c in range(args.warmup + args.steps):
                 B.iqk_dequant(dw, c % args.experts, S.value_table("int", 2), out=out, stream=stream)
+        torch.cuda.synchronize()
+        return 0
+    if args.profile == "gemv":  # iqk_gemv of one 2048x4096 IQ2_K matrix per call, rotating over --experts copies
+        w, x, values = S.matrix_case("gemv_iq2_k_2048x4096")
+        stack = S.random_streams(S.rng_for(S.seed_of("gemv_iq2_k_2048x4096") + 50), w.fmt, args.experts, w.rows, w.cols)
+        dw = B.Weights.from_host(stack, device)
+        xd = torch.from_numpy(x.view(np.int16)).to(device).view(torch.bfloat16)
+        y = torch.empty((xd.shape[0], w.rows), dtype=torch.float32, device=device)
+        ws = B.workspace(B.iqk_gemv_workspace_bytes(xd.shape[0], w.rows, w.cols), device)
+        with torch.cuda.stream(stream):
+            for c in range(args.warmup + args.steps):
+                B.iqk_gemv(dw, c % args.experts, values, xd, y=y, ws=ws, stream=stream)
         torch.cuda.synchronize()
         return 0
     if args.profile == "prefill":

@@ -1645,14 +1645,26 @@ static int gemv_impl(const WDev& w, int expert, const Values& V, const uint16_t*
     // A tall matrix with up to 4 tokens: the switch tile kernel with every
     // pair on `expert` (no ids array). One launch, the call's first: x rows
     // in shared memory, each CTA sums a tile group's slices in its own
-    // shared memory (no prep kernel, no device-wide counters). 2048x4096 at
-    // one token: 5.5 against 7.4 us; small matrices stay on the stream kernel.
+    // shared memory (no prep kernel, no device-wide counters). Items of two
+    // blocks (half the usual 16-row x 1024-weight slice where rows have a
+    // multiple of four blocks): one tile per CTA, twice the CTAs, half the
+    // decode per warp; the scales then come from the planes, since the
+    // images hold four-block slices. 2048x4096 at one token: 4.75 against
+    // 5.57 us with four-block items and 7.4 us on the stream kernel; small
+    // matrices stay on the stream kernel.
     if (tiles_ok && T <= 4 && tiles >= 64 && act_rows_smem(1, T, w.cols)) {
+      CUtensorMap map2 = map;
+      if (a.bpi == 4) {
+        a.bpi = 2;
+        a.splits *= 2;
+        if (make_qs_map(&map2, w, a.bpi)) return -4;
+      }
       UnitArgs b = a;
       b.first = 1;
       b.check_ids = 0;
       b.w0 = w;
       b.w1 = w;
+      if (b.bpi != item_blocks(w.cols)) b.w0.slots = b.w1.slots = nullptr;
       b.V = V;
       b.ids = nullptr;
       b.expert = expert;
@@ -1664,7 +1676,7 @@ static int gemv_impl(const WDev& w, int expert, const Values& V, const uint16_t*
       b.status = status;
       b.act_rows = T;
       b.tpg = std::max(1, kDecodeWarps / b.splits);
-      return launch_tiles<MODE_SWITCH, FMT, FMT, 1, true>(map, map, b, (tiles + b.tpg - 1) / b.tpg, st, num_sms,
+      return launch_tiles<MODE_SWITCH, FMT, FMT, 1, true>(map2, map2, b, (tiles + b.tpg - 1) / b.tpg, st, num_sms,
                                                           true);
     }
   }

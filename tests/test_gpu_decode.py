@@ -91,6 +91,23 @@ def test_gemv_matrix_cases(B, case, T):
 
 
 @pytest.mark.parametrize("fmt", ["iq2_ks", "iq2_k"])
+@pytest.mark.parametrize("rows,cols,T", [(2048, 4096, 1), (2048, 4096, 4), (1030, 5120, 1), (1030, 5120, 2)])
+def test_gemv_tile_path(B, fmt, rows, cols, T):
+    """Tall matrices with at most 4 tokens take the tile kernel with
+    two-block items (scales from the planes): 2048 x 4096 gives one tile per
+    CTA and one item per warp; 1030 x 5120 gives a ragged last tile and ten
+    slices, so two warps take a second item. Expert 2 of 3, f16 table."""
+    rng = S.rng_for(rows + cols + T)
+    w = S.random_streams(rng, fmt, 3, rows, cols)
+    x = S.random_bf16(rng, (T, cols))
+    values = S.value_table("f16", 5)
+    dw = B.Weights.from_host(w)
+    y = B.iqk_gemv(dw, 2, values, to_dev_bf16(x)).cpu().numpy()
+    y_ref, Sabs = O.gemv(O.dequant_expert(w, 2, values), x)
+    check_fp32(y, y_ref, Sabs, f"gemv tile path {fmt} {rows}x{cols} T={T}")
+
+
+@pytest.mark.parametrize("fmt", ["iq2_ks", "iq2_k"])
 @pytest.mark.parametrize("T", [9, 16, 33, 64])
 def test_gemv_ragged_and_many_tokens(B, fmt, T):
     rng = S.rng_for(7 + T)
