@@ -22,7 +22,8 @@ FMT = {"iq2_ks": 0, "iq2_k": 1}
 EXPORTS = (
     "iqk_strerror", "iqk_last_cuda_error", "iqk_version", "iqk_row_bytes",
     "iqk_dequant", "iqk_dequant_bf16", "iqk_dequant_floor", "iqk_gemv_workspace_bytes", "iqk_gemv", "iqk_gemv_static",
-    "iqk_moe_workspace_bytes", "iqk_moe_workspace_layout", "iqk_moe_decode", "iqk_moe_decode_shard", "iqk_f32_to_bf16",
+    "iqk_moe_workspace_bytes", "iqk_moe_workspace_layout", "iqk_moe_decode", "iqk_moe_decode_host",
+    "iqk_moe_decode_shard", "iqk_f32_to_bf16",
     "iqk_moe_prefill", "iqk_moe_prefill_shard", "iqk_moe_combine", "iqk_moe_status",
     "iqk_route_workspace_bytes", "iqk_moe_route", "iqk_floor", "iqk_floor_status", "iqk_set_wait_limit_ns",
     "iqk_switch_linear_workspace_bytes", "iqk_switch_linear", "iqk_slots_bytes", "iqk_pack_slots",
@@ -76,6 +77,7 @@ def lib(build_if_missing: bool = True) -> ctypes.CDLL:
             "iqk_moe_workspace_layout": (ctypes.c_int, [i32, i32, i32, i32, i32, i32,
                                                         ctypes.POINTER(IqkWsLayout)]),
             "iqk_moe_decode": (ctypes.c_int, [W, W, W, vp, vp, i32, vp, vp, i32, vp, vp, sz, vp]),
+            "iqk_moe_decode_host": (ctypes.c_int, [W, W, W, vp, vp, i32, vp, vp, i32, vp, vp, sz, vp]),
             "iqk_moe_decode_shard": (ctypes.c_int, [W, W, W, vp, vp, i32, vp, vp, i32, i32, vp, vp, sz, vp]),
             "iqk_f32_to_bf16": (ctypes.c_int, [vp, vp, ctypes.c_int64, vp]),
             "iqk_moe_prefill": (ctypes.c_int, [W, W, W, vp, vp, i32, vp, vp, i32, vp, vp, sz, vp]),
@@ -321,6 +323,26 @@ def _moe(fn, mode, gate, up, down, values, x, ids, p, y, ws, stream):
 
 def iqk_moe_decode(gate: Weights, up: Weights, down: Weights, values, x, ids, p, y=None, ws=None, stream=None):
     return _moe(lib().iqk_moe_decode, 0, gate, up, down, values, x, ids, p, y, ws, stream)
+
+
+def iqk_moe_decode_host(gate: Weights, up: Weights, down: Weights, values, x, ids, p, y=None, ws=None, stream=None):
+    """iqk_moe_decode on page-locked host tensors (x, ids, p and y pinned CPU
+    tensors); the call's kernels read the inputs and write y over the host
+    link. y is complete once the stream has passed the call. The workspace is
+    device memory on the current device."""
+    torch = _torch()
+    T, topk = ids.shape
+    if y is None:
+        y = torch.empty((T, down.rows), dtype=torch.bfloat16, pin_memory=True)
+    if ws is None:
+        ws = workspace(iqk_moe_workspace_bytes(0, T, topk, gate.experts, gate.cols, gate.rows),
+                       torch.device("cuda", torch.cuda.current_device()))
+    v = _values(values)
+    _check(lib().iqk_moe_decode_host(ctypes.byref(gate.c), ctypes.byref(up.c), ctypes.byref(down.c), v.ctypes.data,
+                                     x.data_ptr(), T, ids.data_ptr(), p.data_ptr(), topk, y.data_ptr(),
+                                     ws.data_ptr(), ws.numel(), _stream(stream)),
+           "iqk_moe_decode_host")
+    return y
 
 
 def iqk_moe_prefill(gate: Weights, up: Weights, down: Weights, values, x, ids, p, y=None, ws=None, stream=None):

@@ -406,14 +406,29 @@ __device__ __forceinline__ void build_route_warp(int my_id, int n, int E, RouteV
 }
 
 // ------------------------------------------------------------- prep kernel
+// Inputs that a routed call reads from page-locked host memory, copied once
+// into the workspace by the prep kernel (n = 0, nx = 0: nothing to copy).
+struct PrepStage {
+  const int32_t* ids;
+  const float* p;
+  int32_t* ids_out;
+  float* p_out;
+  int n;  // pairs
+  const uint4* xraw;
+  uint4* xraw_out;
+  int nx;  // 16-byte words of x copied as they are
+};
+
 // Resets the status word and records out-of-range expert ids, zeroes the
 // stream kernel's tile counters (GEMV) and slot-transposes the activations
 // read through L1 (x[t][16w + i + 4j] -> xp[t][16w + 4i + j]); T = 0 skips
 // the transposition (x staged in shared memory), npairs = 0 the id check.
+// With host-resident inputs it also copies ids, p and (for x staged in
+// shared memory) x into the workspace.
 __global__ void __launch_bounds__(256) k_prep(const uint16_t* __restrict__ x, int T, int cols,
                                               uint16_t* __restrict__ xp, int32_t* __restrict__ zero,
                                               int nzero, const int32_t* __restrict__ ids, int npairs, int E,
-                                              int32_t* __restrict__ status) {
+                                              int32_t* __restrict__ status, PrepStage sg) {
   // Launched as a dependent of whatever precedes it (the previous call's last
   // kernel may still be writing this call's x or ids, or reading the
   // workspace written below): nothing is read or written before the wait.
@@ -424,6 +439,11 @@ __global__ void __launch_bounds__(256) k_prep(const uint16_t* __restrict__ x, in
   const int tid = blockIdx.x * blockDim.x + threadIdx.x;
   const int nth = gridDim.x * blockDim.x;
   for (int i = tid; i < nzero; i += nth) zero[i] = 0;
+  for (int i = tid; i < sg.n; i += nth) {
+    sg.ids_out[i] = sg.ids[i];
+    sg.p_out[i] = sg.p[i];
+  }
+  for (int i = tid; i < sg.nx; i += nth) sg.xraw_out[i] = sg.xraw[i];
   if (blockIdx.x == 0 && threadIdx.x < 32) {
     int bad = 0;
     for (int p = threadIdx.x; p < npairs; p += 32) bad |= (ids[p] < 0 || ids[p] >= E);
@@ -492,6 +512,7 @@ struct UnitArgs {
   int tpg;       // tile kernel, SWITCH: tiles per group (items per group = splits * tpg)
   int ebase;     // routed modes: first expert id the weights hold (expert-parallel shard)
   int first;     // tile kernel launched as the call's first kernel (no prep kernel before it)
+  int wait_in;   // tile kernel: ids, p (and x) are the prep kernel's copies: wait for it before reading them
   int check_ids; // first: record out-of-range ids in the status word
   int expire;    // testing hook: warp 0 of every CTA also waits on a barrier nothing arrives on
   uint64_t wait_ns;  // bound of every wait on a data barrier (global-timer ns)
@@ -934,7 +955,7 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, kDecodeMinBlocks(NT)) k_til
   // never reads a counter of an earlier call.
   const bool publish = MODE == MODE_GATEUP && A.ready != nullptr;
   const bool hready = MODE == MODE_DOWN && BSM && A.ready != nullptr;
-  if (A.first) griddep_wait();
+  if (A.first || A.wait_in) griddep_wait();
   if (!publish) griddep_launch();
   // the call's inputs first (ids, routing weights, x), then the tables while they arrive
   // (switch mode without an ids array: every pair is on expert A.expert, a
@@ -1491,7 +1512,8 @@ static cudaLaunchAttribute pdl_attr() {
 // stream (the previous call's last kernel triggers early); it waits before
 // its first read or write.
 static int launch_prep(int blocks, cudaStream_t st, const uint16_t* x, int T, int cols, uint16_t* xp, int32_t* zero,
-                       int nzero, const int32_t* ids, int npairs, int E, int32_t* status) {
+                       int nzero, const int32_t* ids, int npairs, int E, int32_t* status,
+                       const PrepStage& sg = PrepStage{}) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(blocks);
   cfg.blockDim = dim3(256);
@@ -1499,7 +1521,8 @@ static int launch_prep(int blocks, cudaStream_t st, const uint16_t* x, int T, in
   cudaLaunchAttribute at[1] = {pdl_attr()};
   cfg.attrs = at;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, k_prep, x, T, cols, xp, zero, nzero, ids, npairs, E, status) == cudaSuccess ? 0 : -4;
+  return cudaLaunchKernelEx(&cfg, k_prep, x, T, cols, xp, zero, nzero, ids, npairs, E, status, sg) == cudaSuccess ? 0
+                                                                                                               : -4;
 }
 
 // Zeroes n words and the floor's timeout flag after the preceding kernel
@@ -1725,6 +1748,8 @@ DecodeWs decode_ws(int T, int topk, int experts, int hidden, int inter) {
   o = align256(o + (size_t)npairs * inter * 2);
   ws.ready = o;
   o = align256(o + (size_t)npairs * 4);
+  ws.hin = o;  // ids and p copied from host memory
+  o = align256(o + (size_t)npairs * 8);
   ws.total = o;
   return ws;
 }
@@ -1732,7 +1757,7 @@ DecodeWs decode_ws(int T, int topk, int experts, int hidden, int inter) {
 template <int FG, int FU, int FD, int NT>
 static int decode_impl(const WDev& g, const WDev& u, const WDev& d, const Values& V, const uint16_t* x, int T,
                        const int32_t* ids, const float* p, int topk, uint16_t* y, float* yf, int ebase, char* ws,
-                       cudaStream_t st, int num_sms) {
+                       cudaStream_t st, int num_sms, bool host_io) {
   static_assert(NT == 1 || NT == 2, "routed decode: one or two MMA column groups");
   const DecodeWs L = decode_ws(T, topk, g.experts, g.cols, g.rows);
   const int npairs = T * topk;
@@ -1754,20 +1779,46 @@ static int decode_impl(const WDev& g, const WDev& u, const WDev& d, const Values
   // status word itself.
   const int hrows = act_rows_smem(NT, npairs, d.cols);
   int32_t* ready = hrows ? reinterpret_cast<int32_t*>(ws + L.ready) : nullptr;
-  if ((!ar || ready) && launch_prep(ar ? 1 : pblocks, st, x, ar ? 0 : T, g.cols, xp, ready, ready ? npairs : 0, ids,
-                                    shard ? 0 : npairs, g.experts, status))
+  // Host-resident inputs: the prep kernel reads each input byte once over the
+  // host link into the workspace (x as it is where its rows are staged in
+  // shared memory, else slot-transposed as usual), and the tile kernels read
+  // the copies after waiting for it. y is written to host memory directly.
+  PrepStage sg = {};
+  const int32_t* ids_k = ids;
+  const float* p_k = p;
+  const uint16_t* x_k = x;
+  if (host_io) {
+    int32_t* ids_s = reinterpret_cast<int32_t*>(ws + L.hin);
+    float* p_s = reinterpret_cast<float*>(ws + L.hin + (size_t)npairs * 4);
+    sg.ids = ids;
+    sg.p = p;
+    sg.ids_out = ids_s;
+    sg.p_out = p_s;
+    sg.n = npairs;
+    if (ar) {
+      sg.xraw = reinterpret_cast<const uint4*>(x);
+      sg.xraw_out = reinterpret_cast<uint4*>(xp);
+      sg.nx = T * g.cols / 8;
+      x_k = xp;
+    }
+    ids_k = ids_s;
+    p_k = p_s;
+  }
+  if ((!ar || ready || host_io) && launch_prep(ar ? 1 : pblocks, st, x, ar ? 0 : T, g.cols, xp, ready,
+                                               ready ? npairs : 0, ids, shard ? 0 : npairs, g.experts, status, sg))
     return -4;
-  a.first = (ar && !ready) ? 1 : 0;
+  a.first = (ar && !ready && !host_io) ? 1 : 0;
+  a.wait_in = host_io ? 1 : 0;
   a.ready = ready;
   a.check_ids = shard ? 0 : 1;
   a.ebase = ebase;
   a.w0 = g;
   a.w1 = u;
   a.V = V;
-  a.ids = ids;
-  a.p = p;
+  a.ids = ids_k;
+  a.p = p_k;
   a.act = xp;
-  a.xraw = x;
+  a.xraw = x_k;
   a.T = T;
   a.topk = topk;
   a.out16 = hp;
@@ -1792,12 +1843,12 @@ static int decode_impl(const WDev& g, const WDev& u, const WDev& d, const Values
 
 int launch_moe_decode(const WDev& g, int fg, const WDev& u, int fu, const WDev& d, int fd, const Values& V,
                       const uint16_t* x, int T, const int32_t* ids, const float* p, int topk, uint16_t* y, float* yf,
-                      int ebase, char* ws, cudaStream_t st, int num_sms) {
+                      int ebase, char* ws, cudaStream_t st, int num_sms, bool host_io) {
   const int NT = routed_nt(T * topk, g.experts);
   const int key = fg * 4 + fu * 2 + fd;
 #define IQK_DEC(G, U, D, N)                  \
   if (key == G * 4 + U * 2 + D && NT == N) \
-    return decode_impl<G, U, D, N>(g, u, d, V, x, T, ids, p, topk, y, yf, ebase, ws, st, num_sms);
+    return decode_impl<G, U, D, N>(g, u, d, V, x, T, ids, p, topk, y, yf, ebase, ws, st, num_sms, host_io);
 #define IQK_DEC_N(G, U, D) IQK_DEC(G, U, D, 1) IQK_DEC(G, U, D, 2)
   IQK_DEC_N(0, 0, 0) IQK_DEC_N(0, 0, 1) IQK_DEC_N(0, 1, 0) IQK_DEC_N(0, 1, 1)
   IQK_DEC_N(1, 0, 0) IQK_DEC_N(1, 0, 1) IQK_DEC_N(1, 1, 0) IQK_DEC_N(1, 1, 1)

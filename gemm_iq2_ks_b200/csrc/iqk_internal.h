@@ -71,7 +71,7 @@ GemvWs gemv_ws(int T, int rows, int cols);
 // through L1 when it does not fit shared memory), h, and one counter per run
 // of pairs (gate/up tile groups of h written so far).
 struct DecodeWs {
-  size_t status, xperm, hperm, ready, total;
+  size_t status, xperm, hperm, ready, hin, total;
   Chunking c2, c3;
 };
 DecodeWs decode_ws(int T, int topk, int experts, int hidden, int inter);
@@ -87,9 +87,12 @@ int launch_gemv(const WDev& w, int fmt, int expert, const Values& V, const uint1
 
 // yf non-null: an expert-parallel shard holding experts [ebase, ebase + E)
 // writes its float32 partial to yf (y unused) and skips other ids silently.
+// host_io: x, ids, p and y are page-locked host memory; the prep kernel
+// copies the inputs into the workspace and the down kernel writes y there.
 int launch_moe_decode(const WDev& g, int fg, const WDev& u, int fu, const WDev& d, int fd,
                       const Values& V, const uint16_t* x, int T, const int32_t* ids, const float* p,
-                      int topk, uint16_t* y, float* yf, int ebase, char* ws, cudaStream_t st, int num_sms);
+                      int topk, uint16_t* y, float* yf, int ebase, char* ws, cudaStream_t st, int num_sms,
+                      bool host_io = false);
 int launch_to_bf16(const float* in, uint16_t* out, int64_t n, cudaStream_t st, int num_sms);
 
 // Routed single projection (switch linear), per (token, slot) pair, fp32.

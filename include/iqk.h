@@ -301,6 +301,26 @@ int iqk_moe_prefill(const iqk_weights* gate, const iqk_weights* up, const iqk_we
                     void* workspace, size_t ws_bytes, void* stream);
 
 /*
+ * iqk_moe_decode_host -- iqk_moe_decode with x, ids, p and y in page-locked
+ * host memory (cudaHostAlloc, cudaMallocHost or cudaHostRegister; reachable
+ * from the device at the same address). The call's kernels move the data
+ * themselves: its first kernel reads each input byte once over the host link
+ * into the workspace, the others read those copies, and the down kernel
+ * writes y to host memory. No copy-engine transfer and no host
+ * synchronisation is involved: y is complete once `stream` has passed the
+ * call (synchronise the stream, or an event recorded after it, before
+ * reading y). The caller must not modify x, ids or p until then. Same
+ * arguments, accuracy and results as iqk_moe_decode, bit for bit. x must be
+ * 16-byte aligned. Returns IQK_EINVAL where one of the four pointers is not
+ * page-locked host memory (cudaPointerGetAttributes reports another type),
+ * otherwise as iqk_moe_decode. Workspace as iqk_moe_decode (device memory).
+ */
+int iqk_moe_decode_host(const iqk_weights* gate, const iqk_weights* up, const iqk_weights* down,
+                        const float* values /* host [8] */, const uint16_t* x /* host */, int32_t T,
+                        const int32_t* ids /* host */, const float* p /* host */, int32_t topk,
+                        uint16_t* y /* host */, void* workspace, size_t ws_bytes, void* stream);
+
+/*
  * iqk_moe_workspace_layout -- where a routed-block call (mode 0 decode,
  * mode 1 prefill; iqk_moe_decode_shard uses the decode layout) keeps its
  * intermediates inside the caller's workspace, for inspection: the tests
