@@ -98,10 +98,13 @@ typedef struct {
   const uint16_t* dv;   /* IQ2_KS [E][rows]; IQ2_K [E][rows][cols/256] */
   /* Optional (NULL when unused): the scale-slot images of these planes,
    * written by iqk_pack_slots, 16-byte aligned. When set, the decode paths
-   * (iqk_gemv, iqk_gemv_static, iqk_moe_decode, iqk_moe_decode_shard, the
-   * decode kernel of iqk_switch_linear, iqk_floor) fetch each work item's
-   * scales with one bulk copy instead of per-lane copies from the planes.
-   * The images must have been packed from these same planes. */
+   * (iqk_gemv, iqk_gemv_static, iqk_moe_decode, iqk_moe_decode_host,
+   * iqk_moe_decode_shard, the decode kernel of iqk_switch_linear, iqk_floor)
+   * fetch each work item's scales with one bulk copy instead of per-lane
+   * copies from the planes; iqk_gemv on a matrix of at least 64 row tiles at
+   * up to 4 tokens splits rows of a multiple of four blocks into two-block
+   * items, whose scales it copies from the planes. The images must have been
+   * packed from these same planes. */
   const uint8_t* slots;
 } iqk_weights;
 
