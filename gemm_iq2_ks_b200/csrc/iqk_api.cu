@@ -234,24 +234,6 @@ int iqk_moe_workspace_layout(int32_t mode, int32_t T, int32_t topk, int32_t expe
   return IQK_OK;
 }
 
-int iqk_moe_decode(const iqk_weights* gate, const iqk_weights* up, const iqk_weights* down, const float* values,
-                   const uint16_t* x, int32_t T, const int32_t* ids, const float* p, int32_t topk, uint16_t* y,
-                   void* workspace, size_t ws_bytes, void* stream) {
-  WDev g, u, d;
-  Values V;
-  int rc;
-  if ((rc = check_moe(gate, up, down, &g, &u, &d)) || (rc = check_values(values, &V))) return rc;
-  if (!x || !ids || !p || !y) return IQK_EINVAL;
-  if (T == 0) return IQK_OK;
-  if (T < 0 || topk < 1 || topk > 16) return IQK_EINVAL;
-  if (T > 64 || T * topk > kMaxPairs) return IQK_EUNSUPPORTED;
-  if ((rc = check_ws(workspace, ws_bytes, decode_ws(T, topk, g.experts, g.cols, g.rows).total))) return rc;
-  const int sms = num_sms();
-  if (sms < 0) return cuda_fail(cudaGetLastError());
-  return from_launch(launch_moe_decode(g, gate->fmt, u, up->fmt, d, down->fmt, V, x, T, ids, p, topk, y, nullptr, 0,
-                                       (char*)workspace, (cudaStream_t)stream, sms));
-}
-
 static bool host_locked(const void* ptr) {
   cudaPointerAttributes at;
   if (cudaPointerGetAttributes(&at, ptr) != cudaSuccess) {
@@ -261,9 +243,11 @@ static bool host_locked(const void* ptr) {
   return at.type == cudaMemoryTypeHost;
 }
 
-int iqk_moe_decode_host(const iqk_weights* gate, const iqk_weights* up, const iqk_weights* down, const float* values,
-                        const uint16_t* x, int32_t T, const int32_t* ids, const float* p, int32_t topk, uint16_t* y,
-                        void* workspace, size_t ws_bytes, void* stream) {
+// iqk_moe_decode and iqk_moe_decode_host: the same checks, then the same launch
+// (host_io: x, ids, p and y in page-locked host memory).
+static int moe_decode(const iqk_weights* gate, const iqk_weights* up, const iqk_weights* down, const float* values,
+                      const uint16_t* x, int32_t T, const int32_t* ids, const float* p, int32_t topk, uint16_t* y,
+                      void* workspace, size_t ws_bytes, void* stream, bool host_io) {
   WDev g, u, d;
   Values V;
   int rc;
@@ -272,13 +256,26 @@ int iqk_moe_decode_host(const iqk_weights* gate, const iqk_weights* up, const iq
   if (T == 0) return IQK_OK;
   if (T < 0 || topk < 1 || topk > 16) return IQK_EINVAL;
   if (T > 64 || T * topk > kMaxPairs) return IQK_EUNSUPPORTED;
-  if (reinterpret_cast<uintptr_t>(x) % 16) return IQK_EINVAL;
-  if (!host_locked(x) || !host_locked(ids) || !host_locked(p) || !host_locked(y)) return IQK_EINVAL;
+  if (host_io && (reinterpret_cast<uintptr_t>(x) % 16 || !host_locked(x) || !host_locked(ids) || !host_locked(p) ||
+                  !host_locked(y)))
+    return IQK_EINVAL;
   if ((rc = check_ws(workspace, ws_bytes, decode_ws(T, topk, g.experts, g.cols, g.rows).total))) return rc;
   const int sms = num_sms();
   if (sms < 0) return cuda_fail(cudaGetLastError());
   return from_launch(launch_moe_decode(g, gate->fmt, u, up->fmt, d, down->fmt, V, x, T, ids, p, topk, y, nullptr, 0,
-                                       (char*)workspace, (cudaStream_t)stream, sms, true));
+                                       (char*)workspace, (cudaStream_t)stream, sms, host_io));
+}
+
+int iqk_moe_decode(const iqk_weights* gate, const iqk_weights* up, const iqk_weights* down, const float* values,
+                   const uint16_t* x, int32_t T, const int32_t* ids, const float* p, int32_t topk, uint16_t* y,
+                   void* workspace, size_t ws_bytes, void* stream) {
+  return moe_decode(gate, up, down, values, x, T, ids, p, topk, y, workspace, ws_bytes, stream, false);
+}
+
+int iqk_moe_decode_host(const iqk_weights* gate, const iqk_weights* up, const iqk_weights* down, const float* values,
+                        const uint16_t* x, int32_t T, const int32_t* ids, const float* p, int32_t topk, uint16_t* y,
+                        void* workspace, size_t ws_bytes, void* stream) {
+  return moe_decode(gate, up, down, values, x, T, ids, p, topk, y, workspace, ws_bytes, stream, true);
 }
 
 int iqk_moe_decode_shard(const iqk_weights* gate, const iqk_weights* up, const iqk_weights* down,

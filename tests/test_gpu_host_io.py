@@ -98,6 +98,42 @@ def test_host_io_chained_calls_on_one_workspace(B, weights):
         assert np.array_equal(hy.numpy(), want)
 
 
+def test_host_io_output_feeds_the_next_call(B):
+    """Four layers chained through host memory, no synchronisation: call
+    N+1's x is call N's y. Each call's prep kernel reads x only after the
+    previous call's kernels have completed, so the chain must equal, bit for
+    bit, the same chain through device tensors."""
+    rng = S.rng_for(990)
+    # small row scales keep four chained layers (quadratic through SwiGLU) finite and non-zero
+    g, u, d = (B.Weights.from_host(S.random_streams(rng, "iq2_ks", E, r, c, dv_range=(3e-4, 5e-4)))
+               for r, c in ((F, H), (F, H), (H, F)))
+    values = S.value_table("dyadic", 8)
+    layers = 4
+    x0 = S.random_bf16(rng, (1, H))
+    routes = [S.routing(rng, 1, E, K) for _ in range(layers)]
+    ws_d = B.workspace(B.iqk_moe_workspace_bytes(0, 1, K, E, H, F))
+    xd = to_dev_bf16(x0)
+    want = []
+    for ids, p in routes:
+        xd = B.iqk_moe_decode(g, u, d, values, xd, torch.from_numpy(ids).cuda(), torch.from_numpy(p).cuda(), ws=ws_d)
+        want.append(xd.cpu().view(torch.int16).numpy())
+    torch.cuda.synchronize()
+    ws_h = B.workspace(B.iqk_moe_workspace_bytes(0, 1, K, E, H, F))
+    hx = _pinned(x0.view(np.int16), torch.bfloat16)
+    keep, outs = [hx], []
+    for ids, p in routes:
+        hids, hp = _pinned(ids), _pinned(p)
+        hy = torch.zeros((1, H), dtype=torch.int16).pin_memory()
+        B.iqk_moe_decode_host(g, u, d, values, hx, hids, hp, y=hy.view(torch.bfloat16), ws=ws_h)
+        keep += [hids, hp, hy]
+        outs.append(hy)
+        hx = hy.view(torch.bfloat16)
+    torch.cuda.synchronize()
+    for n, (hy, w) in enumerate(zip(outs, want)):
+        assert np.array_equal(hy.numpy(), w), f"layer {n}"
+    assert np.any(want[-1] != 0)
+
+
 def test_host_io_rejects_other_memory(B, weights):
     values = S.value_table("int", 9)
     g, u, d = weights
