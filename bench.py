@@ -39,7 +39,7 @@ RING = 420  # calls per captured graph (10 permutation cycles of 42 calls)
 # call (IQ2_KS, 256 experts, top-6, one token), from one ncu capture of
 # `bench.py --profile decode --experts 24` (its summary is kept under
 # profiles/); per call, not per resident expert.
-DECODE_CALL_TRAFFIC = 42_277_376  # 27,817,984 (gate/up, 6,400 B of it written) + 14,459,392 (down)
+DECODE_CALL_TRAFFIC = 42_272_768  # 27,812,864 (gate/up) + 14,459,904 (down), all reads
 
 
 def env_int(k, d):
